@@ -1,0 +1,254 @@
+"""Pins for the CPU oracle: each check holds it to something other than itself.
+
+Hand-worked examples (tests/golden/), closed forms, special cases that reduce
+to textbook or library routines, brute force on tiny inputs, and the
+agreement of the three independently written forms of retention.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import read_golden, slice_rel_err
+
+rng = np.random.default_rng(7)
+
+
+def _rand(*shape, scale=1.0):
+    return rng.standard_normal(shape) * scale
+
+
+# ---------------------------------------------------------------- constants
+def test_gammas_match_golden_table():
+    g = read_golden("gammas_h16.txt")
+    table = {}
+    # each data line is "h gamma": keys are the head indices
+    for key, val in g.items():
+        table[int(key)] = val[0]
+    got = oracle.decay_gammas(16)
+    for h in range(16):
+        assert got[h] == table[h], (h, got[h], table[h])
+    # the first four are the 200M-layer heads
+    assert list(oracle.decay_gammas(4)) == [0.96875, 0.984375, 0.9921875, 0.99609375]
+
+
+def test_decay_mask_closed_form():
+    D = oracle.decay_mask(8, 0.5)
+    for a in range(8):
+        for b in range(8):
+            want = 2.0 ** (-(a - b)) if a >= b else 0.0
+            assert D[a, b] == want
+    assert np.array_equal(oracle.decay_mask(5, 0.0), np.eye(5))   # 0^0 = 1 on the diagonal
+    assert np.array_equal(oracle.decay_mask(4, 1.0), np.tril(np.ones((4, 4))))
+
+
+def test_thetas_closed_form():
+    # d = 8: theta_j = 10000^(-2j/8) = 10^-j exactly
+    assert np.allclose(oracle.rotation_thetas(8), [1.0, 0.1, 0.01, 0.001], rtol=1e-15, atol=0)
+    assert oracle.rotation_thetas(2)[0] == 1.0
+
+
+# ------------------------------------------------------- hand-worked examples
+def _scalar_case():
+    g = read_golden("scalar_retention_n4.txt")
+    q = g["q"].reshape(1, 4, 1, 1)
+    k = g["k"].reshape(1, 4, 1, 1)
+    v = g["v"].reshape(1, 4, 1, 1)
+    return g, q, k, v
+
+
+@pytest.mark.parametrize("form", ["parallel", "recurrent", "chunk1", "chunk2", "chunk3", "chunk4"])
+def test_scalar_golden(form):
+    g, q, k, v = _scalar_case()
+    gam = [g["gamma"][0]]
+    for state_in, o_key, s_key in [(None, "o", "state"),
+                                   (g["state_in"].reshape(1, 1, 1, 1), "o_with_state", "state_with_state")]:
+        if form == "parallel":
+            o, s = oracle.retention_parallel(q, k, v, gam, state_in)
+        elif form == "recurrent":
+            o, s = oracle.retention_recurrent(q, k, v, gam, state_in)
+        else:
+            o, s = oracle.retention_chunkwise(q, k, v, gam, int(form[5:]), state_in)
+        assert np.allclose(o.ravel(), g[o_key], rtol=0, atol=1e-14), (form, o.ravel())
+        assert np.allclose(s.ravel(), g[s_key], rtol=0, atol=1e-14), (form, s.ravel())
+
+
+@pytest.mark.parametrize("form", ["parallel", "recurrent", "chunk1", "chunk2", "chunk3"])
+def test_matrix_golden(form):
+    g = read_golden("matrix_retention_n3.txt")
+    q = g["q"].reshape(1, 3, 1, 2)
+    k = g["k"].reshape(1, 3, 1, 2)
+    v = g["v"].reshape(1, 3, 1, 2)
+    gam = [g["gamma"][0]]
+    if form == "parallel":
+        o, s = oracle.retention_parallel(q, k, v, gam)
+    elif form == "recurrent":
+        o, s = oracle.retention_recurrent(q, k, v, gam)
+    else:
+        o, s = oracle.retention_chunkwise(q, k, v, gam, int(form[5:]))
+    assert np.allclose(o.ravel(), g["o"], rtol=0, atol=1e-14), o.ravel()
+    assert np.allclose(s.ravel(), g["state"], rtol=0, atol=1e-14), s.ravel()
+
+
+# ------------------------------------------------------- forms agree (pages)
+@pytest.mark.parametrize("chunk", [1, 2, 4, 5, 13, 16])
+@pytest.mark.parametrize("with_state", [False, True])
+def test_three_forms_agree(chunk, with_state):
+    B, n, H, dk, dv = 2, 13, 3, 4, 6        # dk != dv catches a transposed state
+    q, k, v = _rand(B, n, H, dk), _rand(B, n, H, dk), _rand(B, n, H, dv)
+    gam = [0.5, 0.96875, 1.0]
+    s0 = _rand(B, H, dk, dv) if with_state else None
+    o_p, s_p = oracle.retention_parallel(q, k, v, gam, s0)
+    o_r, s_r = oracle.retention_recurrent(q, k, v, gam, s0)
+    o_c, s_c = oracle.retention_chunkwise(q, k, v, gam, chunk, s0)
+    assert np.allclose(o_p, o_r, rtol=0, atol=1e-12)
+    assert np.allclose(o_c, o_r, rtol=0, atol=1e-12)
+    assert np.allclose(s_p, s_r, rtol=0, atol=1e-12)
+    assert np.allclose(s_c, s_r, rtol=0, atol=1e-12)
+
+
+def test_state_brute_force():
+    B, n, H, dk, dv = 1, 9, 2, 3, 5
+    q, k, v = _rand(B, n, H, dk), _rand(B, n, H, dk), _rand(B, n, H, dv)
+    gam = [0.75, 0.9]
+    _, S = oracle.retention_recurrent(q, k, v, gam)
+    for h in range(H):
+        for a in range(dk):
+            for c in range(dv):
+                want = 0.0
+                for m in range(n):
+                    want += gam[h] ** (n - 1 - m) * k[0, m, h, a] * v[0, m, h, c]
+                assert abs(S[0, h, a, c] - want) < 1e-12
+
+
+def test_step_is_one_token_of_the_recurrence():
+    B, n, H, d = 2, 7, 2, 4
+    q, k, v = _rand(B, n + 1, H, d), _rand(B, n + 1, H, d), _rand(B, n + 1, H, d)
+    gam = [0.9, 0.99]
+    o_full, s_full = oracle.retention_recurrent(q, k, v, gam)
+    _, s_pref = oracle.retention_chunkwise(q[:, :n], k[:, :n], v[:, :n], gam, 4)
+    o_step, s_step = oracle.retention_step(q[:, n], k[:, n], v[:, n], gam, s_pref)
+    assert np.allclose(o_step, o_full[:, n], atol=1e-12)
+    assert np.allclose(s_step, s_full, atol=1e-12)
+
+
+# --------------------------------------------- special cases (textbook forms)
+def test_gamma_one_is_causal_linear_attention():
+    B, n, H, dk, dv = 1, 11, 2, 3, 4
+    q, k, v = _rand(B, n, H, dk), _rand(B, n, H, dk), _rand(B, n, H, dv)
+    o, _ = oracle.retention_chunkwise(q, k, v, [1.0, 1.0], 4)
+    outer = k[..., :, None] * v[..., None, :]               # [B, n, H, dk, dv]
+    prefix = np.cumsum(outer, axis=1)                        # library prefix sum
+    want = np.einsum("bnhk,bnhkv->bnhv", q, prefix)
+    assert np.allclose(o, want, atol=1e-12)
+
+
+def test_gamma_zero_is_diagonal():
+    B, n, H, dk, dv = 2, 10, 1, 3, 2
+    q, k, v = _rand(B, n, H, dk), _rand(B, n, H, dk), _rand(B, n, H, dv)
+    for fn in (lambda: oracle.retention_chunkwise(q, k, v, [0.0], 3),
+               lambda: oracle.retention_parallel(q, k, v, [0.0]),
+               lambda: oracle.retention_recurrent(q, k, v, [0.0])):
+        o, s = fn()
+        want = (q * k).sum(-1, keepdims=True) * v
+        assert np.allclose(o, want, atol=1e-12)
+        assert np.allclose(s[:, 0], k[:, -1, 0, :, None] * v[:, -1, 0, None, :], atol=1e-12)
+
+
+def test_rotation_d2_is_complex_multiplication():
+    n = 6
+    x = _rand(1, n, 1, 2)
+    for pos0 in (0, 3, 1000):
+        y = oracle.xpos_rotate(x, pos0)
+        z = (x[..., 0] + 1j * x[..., 1]) * np.exp(1j * (pos0 + np.arange(n)))[None, :, None]
+        assert np.allclose(y[..., 0], z.real, atol=1e-12)
+        assert np.allclose(y[..., 1], z.imag, atol=1e-12)
+
+
+def test_rotation_d4_hand_values():
+    x = np.array([1.0, 0.0, 0.0, 1.0]).reshape(1, 1, 1, 4)
+    for p in (0, 1, 7, 123):
+        y = oracle.xpos_rotate(x, p).ravel()
+        want = [math.cos(p), math.sin(p), -math.sin(0.01 * p), math.cos(0.01 * p)]
+        assert np.allclose(y, want, atol=1e-12)
+
+
+def test_rotation_d8_complex_pairs_and_norm():
+    x = _rand(2, 5, 3, 8)
+    y = oracle.xpos_rotate(x, 11)
+    theta = np.array([1.0, 0.1, 0.01, 0.001])
+    pos = 11 + np.arange(5)
+    z = (x[..., 0::2] + 1j * x[..., 1::2]) * np.exp(1j * pos[None, :, None, None] * theta)
+    assert np.allclose(y[..., 0::2], z.real, atol=1e-12)
+    assert np.allclose(y[..., 1::2], z.imag, atol=1e-12)
+    assert np.allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1), atol=1e-12)
+
+
+def test_rotation_only_relative_positions_matter():
+    B, n, H, d = 1, 12, 2, 8
+    q, k, v = _rand(B, n, H, d), _rand(B, n, H, d), _rand(B, n, H, d)
+    gam = oracle.decay_gammas(H)
+    o0, s0 = oracle.retention_prefill(q, k, v, gam, 4, pos0=0)
+    o1, s1 = oracle.retention_prefill(q, k, v, gam, 4, pos0=517)
+    assert np.allclose(o0, o1, atol=1e-10)
+    # the state is in absolute (rotated) coordinates, so it does change
+    assert not np.allclose(s0, s1, atol=1e-6)
+
+
+def test_split_prefill_through_state():
+    B, n, H, d, m = 2, 20, 2, 8, 12
+    q, k, v = _rand(B, n, H, d), _rand(B, n, H, d), _rand(B, n, H, d)
+    gam = oracle.decay_gammas(H)
+    o_full, s_full = oracle.retention_prefill(q, k, v, gam, 8)
+    o_a, s_a = oracle.retention_prefill(q[:, :m], k[:, :m], v[:, :m], gam, 8)
+    o_b, s_b = oracle.retention_prefill(q[:, m:], k[:, m:], v[:, m:], gam, 8, pos0=m, state_in=s_a)
+    assert np.allclose(np.concatenate([o_a, o_b], axis=1), o_full, atol=1e-12)
+    assert np.allclose(s_b, s_full, atol=1e-12)
+
+
+# ---------------------------------------------------------- gate epilogue
+def test_groupnorm_swish_against_torch_library():
+    N, H, dv = 7, 3, 16
+    o, g = _rand(N, H, dv), _rand(N, H, dv, scale=3.0)
+    w, b = _rand(H, dv), _rand(H, dv)
+    got = oracle.groupnorm_swish(o, g, w, b, eps=1e-5)
+    t = torch.from_numpy(o.reshape(N, H * dv))
+    gn = torch.nn.functional.group_norm(t, H, torch.from_numpy(w.ravel()),
+                                        torch.from_numpy(b.ravel()), eps=1e-5)
+    want = torch.nn.functional.silu(torch.from_numpy(g.reshape(N, H * dv))) * gn
+    assert np.allclose(got.reshape(N, H * dv), want.numpy(), atol=1e-12)
+
+
+def test_groupnorm_swish_hand_values():
+    o = np.array([1.0, 2.0, 3.0, 4.0]).reshape(1, 1, 4)
+    # mean 2.5, biased variance 1.25; a gate of 0 gives swish(0) = 0
+    assert np.all(oracle.groupnorm_swish(o, np.zeros_like(o), eps=0.0) == 0.0)
+    big = np.full_like(o, 60.0)          # swish(60) = 60 to double precision
+    y = oracle.groupnorm_swish(o, big, eps=0.0).ravel() / 60.0
+    assert np.allclose(y, np.array([-1.5, -0.5, 0.5, 1.5]) / math.sqrt(1.25), atol=1e-14)
+    # unit gate: swish(1) = 1 / (1 + e^-1)
+    y1 = oracle.groupnorm_swish(o, np.ones_like(o), eps=0.0).ravel()
+    assert np.allclose(y1, np.array([-1.5, -0.5, 0.5, 1.5]) / math.sqrt(1.25) / (1 + math.exp(-1)),
+                       atol=1e-14)
+
+
+def test_groupnorm_output_moments():
+    o = _rand(50, 4, 32, scale=5.0) + 3.0
+    y = oracle.groupnorm_swish(o, np.full_like(o, 60.0), eps=1e-5) / 60.0
+    assert np.allclose(y.mean(-1), 0.0, atol=1e-12)
+    var = o.var(-1)
+    assert np.allclose(y.var(-1), var / (var + 1e-5), atol=1e-12)
+
+
+# ------------------------------------------------------- parity measure
+def test_slice_rel_err_measure():
+    ref = _rand(2, 5, 3, 4)
+    assert slice_rel_err(ref, ref) == 0.0
+    bad = ref.copy()
+    bad[1, 2, 2, 3] += 0.5 * np.abs(ref[1, :, 2, :]).max()
+    assert abs(slice_rel_err(bad, ref) - 0.5) < 1e-12
+    nan = ref.copy()
+    nan[0, 0, 0, 0] = np.nan
+    assert slice_rel_err(nan, ref) == float("inf")
