@@ -1,0 +1,437 @@
+"""Benchmark of the retention hot path on B200: prints one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload layer200m|layer3b|long7b] [--chunk C]
+
+One step = one pass of the whole hot path over one batch of the workload:
+rotation prologue, chunkwise prefill with the state carried out, the
+GroupNorm + swish gate epilogue (when the workload has a gate), then one
+recurrent decode step for every sequence from that state.  `value` counts
+the tokens of the step (batch * seqlen prefill tokens + batch decode
+tokens) per second of device time, max over ranks; inputs are resident in
+HBM.  Three input sets rotate so that every step reads inputs that are not
+in L2 (each set is larger than a third of the 126 MB L2 and three together
+are well beyond it).
+
+Under torchrun each rank runs its own replica (no data-path collective;
+weak scaling).  `--impl reference` times the CPU oracle (float64 numpy) on
+rank 0 on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "retention prefill tokens/s and decode steps/s on 1 B200; % of roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def workload_config(w: wl.Workload, chunk: int) -> dict:
+    return {
+        "workload": f"{w.name}: B={w.batch} H={w.heads} n={w.seqlen} d={w.d} {w.dtype} "
+                    f"chunk {chunk}" + (" + GroupNorm/swish gate" if w.hidden else "") +
+                    " + 1 decode step",
+        "batch": w.batch, "heads": w.heads, "seqlen": w.seqlen, "dk": w.d, "dv": w.d,
+        "chunk": chunk, "gate": bool(w.hidden),
+        "l2": "3 rotating input sets, each beyond 1/3 of the 126 MB L2",
+    }
+
+
+def algorithmic_flops_per_token_head(d: int, chunk: int) -> int:
+    # causal Q K^T and P V inside a chunk, plus the state update and the
+    # cross-chunk product: (dk + dv)(C + 1) + 4 dk dv
+    return 2 * d * (chunk + 1) + 4 * d * d
+
+
+def output_kernel_flops_per_token_head(d: int, chunk: int) -> int:
+    return 2 * d * (chunk + 1) + 2 * d * d
+
+
+def state_kernel_flops_per_token_head(d: int) -> int:
+    return 2 * d * d
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML on a thread."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index: int, period_s: float = 0.002):
+        self.samples = []
+        self.period = period_s
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _sample(self):
+        nv = self.nv
+        mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+        try:
+            reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            reasons = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        self.samples.append((mhz, int(reasons)))
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                return
+            time.sleep(self.period)
+
+    def start(self):
+        if self.nv is None:
+            return
+        self._sample()
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+
+    def stop(self) -> dict:
+        if self.nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+        self._sample()
+        mhz = [s[0] for s in self.samples]
+        active = set()
+        for _, r in self.samples:
+            for name, bit in self.REASONS.items():
+                if r & bit and name != "gpu_idle":
+                    active.add(name)
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(active), "samples": len(mhz)}
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ oracle arm
+def oracle_step(inputs, gam, chunk, b):
+    """The hot path on the CPU oracle for sequence b: prefill + 1 decode step."""
+    import oracle
+    q, k, v, g, qd, kd, vd = inputs
+    sl = slice(b, b + 1)
+    y, s = oracle.retention_prefill(q[sl], k[sl], v[sl], gam, chunk,
+                                    gate=None if g is None else g[sl])
+    n = q.shape[1]
+    o, _ = oracle.retention_step(oracle.xpos_rotate(qd[sl][:, None], n)[:, 0],
+                                 oracle.xpos_rotate(kd[sl][:, None], n)[:, 0], vd[sl], gam, s)
+    return y, o
+
+
+def host_inputs(w: wl.Workload):
+    q, k, v, g = wl.make_prefill_inputs(w.batch, w.heads, w.seqlen, w.d, w.dtype, w.scale,
+                                        w.seed, hidden=w.hidden)
+    qd, kd, vd = (x[0] for x in wl.make_decode_inputs(w.batch, w.heads, 1, w.d, w.dtype,
+                                                      w.scale, w.seed + 100))
+    return q, k, v, g, qd, kd, vd
+
+
+def cpu_baseline(w, chunk, min_seconds=10.0):
+    inputs = host_inputs(w)
+    gam = np.float32([1 - 2.0 ** (-5 - h) for h in range(w.heads)])
+    t0 = time.perf_counter()
+    seqs = 0
+    while True:
+        oracle_step(inputs, gam, chunk, seqs % w.batch)
+        seqs += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or seqs >= 4 * w.batch:
+            break
+    tokens = seqs * (w.seqlen + 1)
+    return {"value": tokens / el, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{seqs} sequence(s) of {w.seqlen} prefill tokens + 1 decode step each, "
+                      f"all {w.heads} heads, float64 numpy, {el:.1f} s"}
+
+
+def run_reference(args, w, chunk):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    inputs = host_inputs(w)
+    gam = np.float32([1 - 2.0 ** (-5 - h) for h in range(w.heads)])
+    for i in range(args.warmup):
+        oracle_step(inputs, gam, chunk, i % w.batch)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle_step(inputs, gam, chunk, i % w.batch)
+    el = time.perf_counter() - t0
+    value = args.steps * (w.seqlen + 1) / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * el / max(args.steps, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, chunk),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
+                         "kind": "oracle",
+                         "sample": f"each step: 1 of {w.batch} sequences ({w.seqlen} prefill "
+                                   f"tokens + 1 decode step), all heads, float64 numpy"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_ours(args, w, chunk):
+    import torch
+    import torch.distributed as dist
+
+    import linear_recurrent_sequence_02_b200 as rn
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    from linear_recurrent_sequence_02_b200.build import build
+    if rank == 0:
+        build()
+    if world > 1:
+        dist.barrier()
+    rn.load_library()
+
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    q, k, v, g, qd, kd, vd = host_inputs(w)
+
+    def pinned(x):
+        return torch.from_numpy(x).to(tdt).pin_memory()
+
+    host = [pinned(x) if x is not None else None for x in (q, k, v, g, qd, kd, vd)]
+    nsets = 3
+    sets = []
+    for _ in range(nsets):
+        sets.append([None if x is None else x.to(dev, non_blocking=True) for x in host])
+    B, n, H, d = w.batch, w.seqlen, w.heads, w.d
+    gam = rn.retnet_default_gammas(H)
+    y = torch.empty(B, n, H, d, dtype=tdt, device=dev)
+    o = torch.empty(B, H, d, dtype=tdt, device=dev)
+    state = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
+    wsb = rn.retnet_chunkwise_workspace_size(B, H, n, d, d, tdt, chunk, args.algo)
+    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=dev)
+
+    def step(s):
+        qq, kk, vv, gg, q1, k1, v1 = s
+        rn.retnet_retention_chunkwise(qq, kk, vv, gam, chunk, state_out=state, gate=gg, out=y,
+                                      workspace=ws, algo=args.algo)
+        rn.retnet_retention_step(q1, k1, v1, gam, state, n, out=o)
+
+    torch.cuda.synchronize()
+    for i in range(args.warmup):
+        step(sets[i % nsets])
+    torch.cuda.synchronize()
+    rn.retnet_check_device_errors(dev)
+
+    # ---- device-timed region
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    stream = torch.cuda.current_stream(dev)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    rn.retnet_profiler_reset()
+    rn.retnet_profiler_enable(True)
+    launches0 = rn.retnet_kernel_launch_count()
+    clocks.start()
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(sets[i % nsets])
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    launches = rn.retnet_kernel_launch_count() - launches0
+    rn.retnet_profiler_enable(False)
+    kern = rn.retnet_profiler_read()
+    if world > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    rn.retnet_check_device_errors(dev)
+
+    tokens_per_step = B * n + B
+    value = world * tokens_per_step * args.steps / (ms / 1e3)
+
+    # ---- end to end through the public API with host buffers
+    h2d = sum(x.numel() * x.element_size() for x in host if x is not None)
+    d2h = y.numel() * y.element_size() + o.numel() * o.element_size()
+    y_host = torch.empty_like(y, device="cpu").pin_memory()
+    o_host = torch.empty_like(o, device="cpu").pin_memory()
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+
+    def e2e_step():
+        s = [None if x is None else x.to(dev, non_blocking=True) for x in host]
+        step(s)
+        y_host.copy_(y, non_blocking=True)
+        o_host.copy_(o, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ev0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * tokens_per_step * e2e_steps / (e2e_ms / 1e3)
+
+    # ---- roofline of the dominant kernel
+    peaks, peak_src = load_peaks()
+    dom = max(kern.items(), key=lambda kv: kv[1][0])[0] if kern else None
+    roof = None
+    kernels_json = {}
+    for name, (tot, cnt) in kern.items():
+        kernels_json[name] = {"avg_us": 1e3 * tot / cnt, "launches": cnt,
+                              "share": tot / max(sum(v[0] for v in kern.values()), 1e-12)}
+    if dom is not None:
+        tot, cnt = kern[dom]
+        avg_s = tot / cnt / 1e3
+        th = B * n * H
+        if dom in ("tc_output", "simt_output"):
+            flops = output_kernel_flops_per_token_head(d, chunk) * th
+            achieved = flops / avg_s / 1e12
+            bound = "tensor" if dom.startswith("tc") else "alu"
+            if bound == "tensor":
+                peak = peaks["bf16_tflops"]
+            else:   # float32 FFMA: 148 SMs x 128 lanes x 2 flop x max SM clock
+                peak = 148 * 128 * 2 * (peaks.get("sm_max_mhz", 1965.0) * 1e6) / 1e12
+            roof = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak,
+                    "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                    "peak_source": peak_src, "work_per_launch": flops}
+        elif dom in ("tc_state", "simt_state"):
+            flops = state_kernel_flops_per_token_head(d) * th
+            achieved = flops / avg_s / 1e12
+            bound = "tensor" if dom.startswith("tc") else "alu"
+            peak = peaks["bf16_tflops"] if bound == "tensor" else \
+                148 * 128 * 2 * (peaks.get("sm_max_mhz", 1965.0) * 1e6) / 1e12
+            roof = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak,
+                    "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                    "peak_source": peak_src, "work_per_launch": flops}
+        else:
+            roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": None, "traffic": None, "peak_source": peak_src}
+
+    # whole prefill against the tensor peak (algorithmic flops at this chunk)
+    pre_names = [nm for nm in kern if nm != "retention_step"]
+    pre_ms = sum(kern[nm][0] for nm in pre_names) / max(args.steps, 1)
+    prefill = None
+    if pre_ms > 0:
+        alg = algorithmic_flops_per_token_head(d, chunk) * B * n * H
+        prefill = {"tokens_per_s": B * n / (pre_ms / 1e3),
+                   "ms": pre_ms,
+                   "tflops_algorithmic": alg / (pre_ms / 1e3) / 1e12,
+                   "frac_of_bf16_peak": alg / (pre_ms / 1e3) / 1e12 / peaks["bf16_tflops"]}
+    decode = None
+    if "retention_step" in kern:
+        tot, cnt = kern["retention_step"]
+        avg_s = tot / cnt / 1e3
+        esz = 2 if w.dtype == "bf16" else 4
+        bytes_step = B * H * (8 * d * d + esz * 4 * d)
+        decode = {"steps_per_s": 1.0 / avg_s, "batch": B, "us_per_step": avg_s * 1e6,
+                  "gbs": bytes_step / avg_s / 1e9, "hbm_frac": bytes_step / avg_s / 1e9 /
+                  peaks["hbm_gbs"], "note": "state just written by the prefill (L2-warm)"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, chunk)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic", "config": workload_config(w, chunk),
+            "algo": args.algo, "roofline": roof, "prefill": prefill, "decode": decode,
+            "kernels": kernels_json, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": launches, "clocks": clock_info,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["layer200m", "layer3b", "long7b"], default="layer200m")
+    ap.add_argument("--chunk", type=int, default=0)
+    ap.add_argument("--algo", choices=["auto", "simt", "tensor"], default="auto")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = wl.WORKLOADS[args.workload]
+    chunk = args.chunk or w.chunk
+    if args.impl == "reference":
+        run_reference(args, w, chunk)
+    else:
+        run_ours(args, w, chunk)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,212 @@
+/*
+ * retnet.h -- C ABI of the B200 (sm_100a) multi-scale retention library.
+ *
+ * The operation is RetNet's retention: a linear recurrence with exponential
+ * decay that can be evaluated in a parallel, a recurrent (O(1) per token,
+ * no KV cache) and a chunkwise form (parallel inside a chunk, a recurrent
+ * state passed between chunks), with a per-head decay gamma, xPos-like
+ * relative positions, and a swish gate plus GroupNorm on the output
+ * ("Retentive Network: A Successor to Transformer for Large Language
+ * Models", research summary page, sections "Summary" and "Key points").
+ *
+ * For one head with decay g, row vectors q_t, k_t (length dk), v_t (dv):
+ *   recurrent : S_t = g S_{t-1} + k_t^T v_t ,  o_t = q_t S_t
+ *   chunkwise : per chunk of L tokens, local indices i, j,
+ *               O = (Q K^T (.) D) V + (Q (.) xi) S_prev,  D_ij = g^(i-j) (i >= j),
+ *               xi_i = g^(i+1);  S = g^L S_prev + K^T (V (.) zeta), zeta_j = g^(L-1-j)
+ *   rotation  : pairs (2j, 2j+1) of q and k turned by pos * theta_j,
+ *               theta_j = 10000^(-2j/dk), pos = pos0 + token index
+ *   epilogue  : Y = swish(G) (.) GroupNorm(O), one group per head (dv channels)
+ *
+ * Conventions for every entry point
+ *   - Tensors are caller-owned device memory, densely packed, row-major:
+ *       q, k         [batch, seqlen, heads, dk]
+ *       v, out, g, y [batch, seqlen, heads, dv]
+ *       state        [batch, heads, dk, dv]   always float32
+ *     Decode-step tensors drop the seqlen axis: q, k [batch, heads, dk], ...
+ *   - Device pointers must be 16-byte aligned.
+ *   - Element type: RETNET_F32 (float) or RETNET_BF16 (bfloat16).  Math and
+ *     accumulation are float32; outputs take the input element type.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and the call returns without synchronising.  Argument errors
+ *     are detected on the host before anything is enqueued and leave every
+ *     buffer untouched.  Faults inside kernels surface at the caller's next
+ *     synchronisation, as with any CUDA work.
+ *   - The library allocates no device memory in these calls; scratch space
+ *     comes from a caller-provided workspace.
+ *   - Calls are thread-safe; concurrent calls must not share output or
+ *     workspace buffers.
+ */
+#ifndef RETNET_H
+#define RETNET_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define RETNET_API __attribute__((visibility("default")))
+#else
+#define RETNET_API
+#endif
+
+struct CUstream_st;
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *retnet_stream_t;
+
+typedef enum retnet_status {
+    RETNET_OK = 0,
+    RETNET_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size or dtype */
+    RETNET_ERR_UNSUPPORTED = 2,  /* well-formed request this build does not implement */
+    RETNET_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
+    RETNET_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up */
+    RETNET_ERR_WORKSPACE = 5     /* workspace missing or smaller than required */
+} retnet_status;
+
+typedef enum retnet_dtype {
+    RETNET_F32 = 0,
+    RETNET_BF16 = 1
+} retnet_dtype;
+
+/* Kernel family for the chunkwise prefill. */
+typedef enum retnet_algo {
+    RETNET_ALGO_AUTO = 0,    /* tensor-core path where it applies, else SIMT */
+    RETNET_ALGO_SIMT = 1,    /* float32 CUDA-core path, any supported shape   */
+    RETNET_ALGO_TENSOR = 2   /* tcgen05/TMEM path: bf16, dk = dv = 256         */
+} retnet_algo;
+
+typedef struct retnet_shape {
+    int batch;       /* >= 0 */
+    int heads;       /* 1 .. 256 */
+    int seqlen;      /* >= 0 tokens */
+    int dk;          /* key/query head dimension: 64, 128 or 256 */
+    int dv;          /* value head dimension: 64, 128 or 256 */
+    retnet_dtype dtype;
+} retnet_shape;
+
+/* Optional output epilogue Y = swish(G) (.) GroupNorm(O).
+ * g: [batch, seqlen, heads, dv] device tensor of the prefill's dtype.
+ * weight, bias: device float32 [heads * dv] affine (NULL = 1 and 0).
+ * eps: added to the biased variance (for example 1e-5). */
+typedef struct retnet_gate {
+    const void *g;
+    const float *weight;
+    const float *bias;
+    float eps;
+} retnet_gate;
+
+/* Human-readable name of a status code (static string, never NULL). */
+RETNET_API const char *retnet_status_string(retnet_status status);
+
+/* Number of kernels this library has launched in this process (all
+ * devices, all threads).  Used to count launches inside a timed region. */
+RETNET_API unsigned long long retnet_kernel_launch_count(void);
+
+/* Per-head decay constants gamma_h = 1 - 2^(-5-h), h = 0..heads-1, written
+ * to the HOST array gammas[heads] ("Key points": gamma = 1 - 2^(-5-i)).
+ * Errors: INVALID_ARG if gammas is NULL or heads is outside 1..256. */
+RETNET_API retnet_status retnet_default_gammas(int heads, float *gammas);
+
+/* xPos-like rotation prologue ("Summary": positions encoded similarly to
+ * xPos).  y[b, t, h, :] = rotation of x[b, t, h, :] by (pos0 + t) * theta_j
+ * on each adjacent pair (2j, 2j+1).  x and y are [batch, seqlen, heads, d]
+ * device tensors of `dtype`; y == x (in place) is allowed, any other
+ * overlap is not.  d must be a multiple of 8 and at most 1024; pos0 >= 0.
+ * Angles are reduced in float64 before a float32 sine/cosine. */
+RETNET_API retnet_status retnet_xpos_rotate(const void *x, void *y, int batch, int seqlen, int heads,
+                                 int d, retnet_dtype dtype, long long pos0,
+                                 retnet_stream_t stream);
+
+/* Bytes of device workspace retnet_retention_chunkwise needs for this shape,
+ * chunk length and algorithm (RETNET_ALGO_AUTO resolves as the call would).
+ * Errors: as retnet_retention_chunkwise's shape checks. */
+RETNET_API retnet_status retnet_chunkwise_workspace_size(const retnet_shape *shape, int chunk,
+                                              retnet_algo algo, size_t *bytes);
+
+/* Chunkwise-recurrent prefill ("Summary": computes in parallel within a
+ * chunk and passes the recurrent state between chunks; "Key points": cost
+ * O(d n (b + h)) with chunk b).
+ *   q, k, v    device inputs (layouts above); not modified.
+ *   gammas     HOST float array [heads]: the per-head decay, each in [0, 1].
+ *   chunk      chunk length b, 1..1024; seqlen need not be a multiple
+ *              (the last chunk is then shorter).  The tensor path takes
+ *              chunk in {128, 256, 512, 1024}.
+ *   out        device output [batch, seqlen, heads, dv]: O, or Y when `gate`
+ *              is given.
+ *   pos0       position of token 0 for the rotation (split prefills pass
+ *              the number of tokens already consumed).
+ *   rotate     1: rotate q and k by position first; 0: use them as given.
+ *   state_in   device float32 [batch, heads, dk, dv] state before token 0,
+ *              or NULL for a zero state.
+ *   state_out  device float32 [batch, heads, dk, dv] state after the last
+ *              token, or NULL.  May equal state_in.
+ *   gate       optional epilogue (NULL: out = O).
+ *   algo       kernel family, see retnet_algo.
+ *   workspace  device scratch of at least retnet_chunkwise_workspace_size()
+ *              bytes, 256-byte aligned; contents on entry are ignored.
+ * Errors: INVALID_ARG (null or misaligned pointers, sizes out of range,
+ * gamma outside [0,1]), UNSUPPORTED (dk/dv not in {64,128,256}, or a tensor
+ * path request it cannot serve), WORKSPACE, CUDA. */
+RETNET_API retnet_status retnet_retention_chunkwise(const void *q, const void *k, const void *v,
+                                         const float *gammas, int chunk, void *out,
+                                         const retnet_shape *shape, long long pos0, int rotate,
+                                         const float *state_in, float *state_out,
+                                         const retnet_gate *gate, retnet_algo algo,
+                                         void *workspace, size_t workspace_bytes,
+                                         retnet_stream_t stream);
+
+/* One recurrent decode step for every (sequence, head) ("Summary": the
+ * recurrent form costs O(1) per step and needs no KV cache).
+ *   q, k [batch, heads, dk], v [batch, heads, dv]: this token, device, dtype.
+ *   gammas   HOST float array [heads].
+ *   state    device float32 [batch, heads, dk, dv], updated in place:
+ *            S <- gamma S + k^T v.
+ *   out      device [batch, heads, dv]: o = q S (after the update).
+ *   pos      rotation position of this token (prefill length + steps done).
+ *   rotate   1: rotate q and k by pos first; 0: use them as given.
+ * Errors: INVALID_ARG, UNSUPPORTED (dk/dv not in {64,128,256}), CUDA. */
+RETNET_API retnet_status retnet_retention_step(const void *q, const void *k, const void *v,
+                                    const float *gammas, float *state, void *out,
+                                    int batch, int heads, int dk, int dv, retnet_dtype dtype,
+                                    long long pos, int rotate, retnet_stream_t stream);
+
+/* Output epilogue Y = swish(G) (.) GroupNorm(O) ("Summary": a swish gate
+ * and GroupNorm are added).  o, g, y: device [rows, heads, dv] of `dtype`
+ * (rows = batch * seqlen); one group per (row, head) over its dv channels,
+ * biased variance, then the per-channel affine weight/bias (device float32
+ * [heads * dv], NULL = 1 / 0), times swish(g) = g * sigmoid(g).
+ * y may equal o.  dv must be a multiple of 8 and at most 1024. */
+RETNET_API retnet_status retnet_groupnorm_swish(const void *o, const void *g, const float *weight,
+                                     const float *bias, float eps, long long rows, int heads,
+                                     int dv, retnet_dtype dtype, void *y,
+                                     retnet_stream_t stream);
+
+/* Reads and clears the library's device-side error word on the current
+ * device after synchronising `stream`.  Returns RETNET_OK when no kernel
+ * reported a problem, RETNET_ERR_TIMEOUT when a bounded wait inside a
+ * kernel gave up (its results are then invalid), RETNET_ERR_CUDA when the
+ * read itself failed. */
+RETNET_API retnet_status retnet_check_device_errors(retnet_stream_t stream);
+
+/* ---- Kernel timer (diagnostics; off by default) ----------------------
+ * While enabled, every kernel this library launches is bracketed by CUDA
+ * events on its own stream, and per-kernel totals accumulate until reset.
+ * Adds a few microseconds of host work per launch; do not enable it while
+ * capturing a CUDA graph. */
+RETNET_API retnet_status retnet_profiler_enable(int on);
+/* Drops accumulated totals (waits for pending events first). */
+RETNET_API retnet_status retnet_profiler_reset(void);
+/* Totals of the index-th kernel name (0-based, sorted by name): copies the
+ * name (NUL-terminated, truncated to name_len) and writes the summed device
+ * milliseconds and the launch count.  Waits for pending events.
+ * Returns INVALID_ARG past the last index or for NULL outputs. */
+RETNET_API retnet_status retnet_profiler_read(int index, char *name, size_t name_len,
+                                              double *total_ms, unsigned long long *launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RETNET_H */

@@ -1,0 +1,199 @@
+// C ABI entry points: host-side validation, then dispatch to the kernels.
+//
+// Every check runs before anything is enqueued, so a rejected call leaves
+// all buffers untouched and launches nothing.
+#include <atomic>
+#include <cmath>
+
+#include "kernels.h"
+
+namespace retnet {
+
+static std::atomic<unsigned long long> g_launches{0};
+void count_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+__device__ unsigned g_device_error = 0u;
+
+unsigned *device_error_word() {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    return (unsigned *)p;
+}
+
+static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+static bool head_dim_ok(int d) { return d == 64 || d == 128 || d == 256; }
+static bool dtype_ok(retnet_dtype t) { return t == RETNET_F32 || t == RETNET_BF16; }
+static size_t elem_size(retnet_dtype t) { return t == RETNET_BF16 ? 2 : 4; }
+
+static retnet_status load_gammas(const float *gammas, int heads, HeadGammas *out) {
+    if (!gammas || heads < 1 || heads > kMaxHeads) return RETNET_ERR_INVALID_ARG;
+    for (int h = 0; h < kMaxHeads; ++h) out->g[h] = 0.f;
+    for (int h = 0; h < heads; ++h) {
+        float g = gammas[h];
+        if (!(g >= 0.f && g <= 1.f)) return RETNET_ERR_INVALID_ARG;   // also rejects NaN
+        out->g[h] = g;
+    }
+    return RETNET_OK;
+}
+
+static retnet_status check_shape(const retnet_shape *s, int chunk) {
+    if (!s) return RETNET_ERR_INVALID_ARG;
+    if (s->batch < 0 || s->seqlen < 0 || s->heads < 1 || s->heads > kMaxHeads)
+        return RETNET_ERR_INVALID_ARG;
+    if (!dtype_ok(s->dtype)) return RETNET_ERR_INVALID_ARG;
+    if (chunk < 1 || chunk > 1024) return RETNET_ERR_INVALID_ARG;
+    if (s->dk <= 0 || s->dv <= 0) return RETNET_ERR_INVALID_ARG;
+    if (!head_dim_ok(s->dk) || !head_dim_ok(s->dv)) return RETNET_ERR_UNSUPPORTED;
+    return RETNET_OK;
+}
+
+static retnet_algo resolve_algo(const retnet_shape *s, int chunk, retnet_algo algo) {
+    (void)s; (void)chunk;
+    if (algo == RETNET_ALGO_AUTO) return RETNET_ALGO_SIMT;
+    return algo;
+}
+
+}  // namespace retnet
+
+using namespace retnet;
+
+extern "C" {
+
+const char *retnet_status_string(retnet_status status) {
+    switch (status) {
+        case RETNET_OK: return "ok";
+        case RETNET_ERR_INVALID_ARG: return "invalid argument";
+        case RETNET_ERR_UNSUPPORTED: return "unsupported shape or option";
+        case RETNET_ERR_CUDA: return "CUDA error";
+        case RETNET_ERR_TIMEOUT: return "device-side wait timed out";
+        case RETNET_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+unsigned long long retnet_kernel_launch_count(void) {
+    return g_launches.load(std::memory_order_relaxed);
+}
+
+retnet_status retnet_default_gammas(int heads, float *gammas) {
+    if (!gammas || heads < 1 || heads > kMaxHeads) return RETNET_ERR_INVALID_ARG;
+    for (int h = 0; h < heads; ++h) gammas[h] = (float)(1.0 - std::ldexp(1.0, -5 - h));
+    return RETNET_OK;
+}
+
+retnet_status retnet_xpos_rotate(const void *x, void *y, int batch, int seqlen, int heads, int d,
+                                 retnet_dtype dtype, long long pos0, retnet_stream_t stream) {
+    if (batch < 0 || seqlen < 0 || heads < 1 || pos0 < 0 || !dtype_ok(dtype))
+        return RETNET_ERR_INVALID_ARG;
+    if (d <= 0 || d % 8 != 0 || d > 1024) return RETNET_ERR_INVALID_ARG;
+    if ((long long)batch * seqlen == 0) return RETNET_OK;
+    if (!x || !y || !aligned16(x) || !aligned16(y)) return RETNET_ERR_INVALID_ARG;
+    RETNET_CUDA_TRY(launch_xpos_rotate(x, y, (long long)batch * seqlen, heads, d, dtype, seqlen,
+                                       pos0, (cudaStream_t)stream));
+    return RETNET_OK;
+}
+
+retnet_status retnet_chunkwise_workspace_size(const retnet_shape *shape, int chunk,
+                                              retnet_algo algo, size_t *bytes) {
+    if (!bytes) return RETNET_ERR_INVALID_ARG;
+    retnet_status st = check_shape(shape, chunk);
+    if (st != RETNET_OK) return st;
+    retnet_algo a = resolve_algo(shape, chunk, algo);
+    if (a != RETNET_ALGO_SIMT) return RETNET_ERR_UNSUPPORTED;
+    *bytes = simt_workspace_bytes(shape->batch, shape->heads, shape->seqlen, shape->dk,
+                                  shape->dv, chunk);
+    return RETNET_OK;
+}
+
+retnet_status retnet_retention_chunkwise(const void *q, const void *k, const void *v,
+                                         const float *gammas, int chunk, void *out,
+                                         const retnet_shape *shape, long long pos0, int rotate,
+                                         const float *state_in, float *state_out,
+                                         const retnet_gate *gate, retnet_algo algo,
+                                         void *workspace, size_t workspace_bytes,
+                                         retnet_stream_t stream) {
+    retnet_status st = check_shape(shape, chunk);
+    if (st != RETNET_OK) return st;
+    if (pos0 < 0 || (rotate != 0 && rotate != 1)) return RETNET_ERR_INVALID_ARG;
+    if (algo != RETNET_ALGO_AUTO && algo != RETNET_ALGO_SIMT && algo != RETNET_ALGO_TENSOR)
+        return RETNET_ERR_INVALID_ARG;
+    ChunkwiseArgs a;
+    st = load_gammas(gammas, shape->heads, &a.gam);
+    if (st != RETNET_OK) return st;
+    const long long tokens = (long long)shape->batch * shape->seqlen;
+    if (tokens > 0) {
+        if (!q || !k || !v || !out) return RETNET_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+            return RETNET_ERR_INVALID_ARG;
+    }
+    if ((state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out)))
+        return RETNET_ERR_INVALID_ARG;
+    if (gate) {
+        if (tokens > 0 && (!gate->g || !aligned16(gate->g))) return RETNET_ERR_INVALID_ARG;
+        if (!(gate->eps >= 0.f)) return RETNET_ERR_INVALID_ARG;
+    }
+    retnet_algo resolved = resolve_algo(shape, chunk, algo);
+    if (resolved != RETNET_ALGO_SIMT) return RETNET_ERR_UNSUPPORTED;
+    size_t need = simt_workspace_bytes(shape->batch, shape->heads, shape->seqlen, shape->dk,
+                                       shape->dv, chunk);
+    if (need > 0 && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)))
+        return RETNET_ERR_WORKSPACE;
+    if (shape->batch == 0) return RETNET_OK;
+
+    a.q = q; a.k = k; a.v = v; a.out = out;
+    a.state_in = state_in; a.state_out = state_out; a.gate = gate;
+    a.batch = shape->batch; a.heads = shape->heads; a.seqlen = shape->seqlen;
+    a.dk = shape->dk; a.dv = shape->dv; a.chunk = chunk; a.dtype = shape->dtype;
+    a.pos0 = pos0; a.rotate = rotate; a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
+    RETNET_CUDA_TRY(launch_chunkwise_simt(a, (cudaStream_t)stream));
+    return RETNET_OK;
+}
+
+retnet_status retnet_retention_step(const void *q, const void *k, const void *v,
+                                    const float *gammas, float *state, void *out, int batch,
+                                    int heads, int dk, int dv, retnet_dtype dtype, long long pos,
+                                    int rotate, retnet_stream_t stream) {
+    if (batch < 0 || heads < 1 || heads > kMaxHeads || !dtype_ok(dtype) || pos < 0 ||
+        (rotate != 0 && rotate != 1))
+        return RETNET_ERR_INVALID_ARG;
+    if (dk <= 0 || dv <= 0) return RETNET_ERR_INVALID_ARG;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return RETNET_ERR_UNSUPPORTED;
+    HeadGammas gam;
+    retnet_status st = load_gammas(gammas, heads, &gam);
+    if (st != RETNET_OK) return st;
+    if (batch == 0) return RETNET_OK;
+    if (!q || !k || !v || !state || !out) return RETNET_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(out))
+        return RETNET_ERR_INVALID_ARG;
+    RETNET_CUDA_TRY(launch_retention_step(q, k, v, gam, state, out, batch, heads, dk, dv, dtype,
+                                          pos, rotate, (cudaStream_t)stream));
+    return RETNET_OK;
+}
+
+retnet_status retnet_groupnorm_swish(const void *o, const void *g, const float *weight,
+                                     const float *bias, float eps, long long rows, int heads,
+                                     int dv, retnet_dtype dtype, void *y,
+                                     retnet_stream_t stream) {
+    if (rows < 0 || heads < 1 || !dtype_ok(dtype) || !(eps >= 0.f)) return RETNET_ERR_INVALID_ARG;
+    if (dv <= 0 || dv % 8 != 0 || dv > 1024) return RETNET_ERR_INVALID_ARG;
+    if (rows == 0) return RETNET_OK;
+    if (!o || !g || !y || !aligned16(o) || !aligned16(g) || !aligned16(y))
+        return RETNET_ERR_INVALID_ARG;
+    RETNET_CUDA_TRY(launch_groupnorm_swish(o, g, weight, bias, eps, rows, heads, dv, dtype, y,
+                                           (cudaStream_t)stream));
+    return RETNET_OK;
+}
+
+retnet_status retnet_check_device_errors(retnet_stream_t stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return RETNET_ERR_CUDA;
+    unsigned word = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word)) != cudaSuccess)
+        return RETNET_ERR_CUDA;
+    if (word == 0) return RETNET_OK;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+        return RETNET_ERR_CUDA;
+    return (word & kDevErrTimeout) ? RETNET_ERR_TIMEOUT : RETNET_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,107 @@
+// Shared device helpers for the retention kernels (internal header).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/retnet.h"
+
+namespace retnet {
+
+constexpr int kMaxHeads = 256;
+
+// Per-head decay constants travel by value in the kernel parameter block.
+struct HeadGammas {
+    float g[kMaxHeads];
+};
+
+// Device-side error word (bit flags), read by retnet_check_device_errors.
+enum DeviceError : unsigned {
+    kDevErrTimeout = 1u,
+};
+unsigned *device_error_word();   // device address of this device's error word
+
+// Counts host-side kernel launches (see retnet_kernel_launch_count).
+void count_launch(unsigned n = 1);
+
+// Records CUDA events around one launch on `stream` while the profiler is
+// enabled (retnet_profiler_enable); a no-op otherwise.  `name` must be a
+// string literal.
+class KernelTimer {
+  public:
+    KernelTimer(const char *name, cudaStream_t stream);
+    ~KernelTimer();
+    KernelTimer(const KernelTimer &) = delete;
+    KernelTimer &operator=(const KernelTimer &) = delete;
+
+  private:
+    cudaStream_t stream_;
+    const char *name_ = nullptr;
+    void *start_ = nullptr;
+    void *stop_ = nullptr;
+};
+
+// ---------------------------------------------------------------- element IO
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+    return __bfloat162float(x);
+}
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Loads 8 consecutive elements as float (16-byte aligned for bf16, 32 for f32).
+__device__ __forceinline__ void load8(const float *p, float *out) {
+    float4 a = reinterpret_cast<const float4 *>(p)[0];
+    float4 b = reinterpret_cast<const float4 *>(p)[1];
+    out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
+    out[4] = b.x; out[5] = b.y; out[6] = b.z; out[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float *out) {
+    uint4 u = *reinterpret_cast<const uint4 *>(p);
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 f = __bfloat1622float2(h[i]);
+        out[2 * i] = f.x;
+        out[2 * i + 1] = f.y;
+    }
+}
+__device__ __forceinline__ void store8(float *p, const float *v) {
+    reinterpret_cast<float4 *>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4 *>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+__device__ __forceinline__ void store8(__nv_bfloat16 *p, const float *v) {
+    uint4 u;
+    __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    *reinterpret_cast<uint4 *>(p) = u;
+}
+
+// ---------------------------------------------------------------- rotation
+// (cos, sin) of pos * theta_j with theta_j = 10000^(-2j/d).  The angle is
+// formed and reduced to [-pi, pi] in float64, then a float32 sincos is
+// taken, so the result is accurate to a few 1e-7 for any position.
+__device__ __forceinline__ float2 rotation_cs(long long pos, int j, int d) {
+    const double two_pi = 6.283185307179586476925286766559;
+    double theta = pow(10000.0, -2.0 * (double)j / (double)d);
+    double a = (double)pos * theta;
+    double r = a - two_pi * rint(a / two_pi);
+    float s, c;
+    sincosf((float)r, &s, &c);
+    return make_float2(c, s);
+}
+
+// ---------------------------------------------------------------- launches
+#define RETNET_CUDA_TRY(expr)                                  \
+    do {                                                       \
+        cudaError_t err__ = (expr);                            \
+        if (err__ != cudaSuccess) return RETNET_ERR_CUDA;      \
+    } while (0)
+
+}  // namespace retnet

@@ -1,0 +1,45 @@
+// Internal launcher declarations shared between api.cu and the kernel files.
+#pragma once
+
+#include "common.cuh"
+
+namespace retnet {
+
+// rotate.cu ---------------------------------------------------------------
+// table[t * (d/2) + j] = (cos, sin) of (pos0 + t) * theta_j, t < n.
+cudaError_t launch_rotation_table(float2 *table, int n, int d, long long pos0,
+                                  cudaStream_t stream);
+cudaError_t launch_xpos_rotate(const void *x, void *y, long long rows_bt, int heads, int d,
+                               retnet_dtype dtype, int seqlen, long long pos0,
+                               cudaStream_t stream);
+
+// step.cu ----------------------------------------------------------------
+cudaError_t launch_retention_step(const void *q, const void *k, const void *v,
+                                  const HeadGammas &gam, float *state, void *out, int batch,
+                                  int heads, int dk, int dv, retnet_dtype dtype, long long pos,
+                                  int rotate, cudaStream_t stream);
+
+// groupnorm.cu -------------------------------------------------------------
+cudaError_t launch_groupnorm_swish(const void *o, const void *g, const float *weight,
+                                   const float *bias, float eps, long long rows, int heads,
+                                   int dv, retnet_dtype dtype, void *y, cudaStream_t stream);
+
+// chunkwise_simt.cu --------------------------------------------------------
+struct ChunkwiseArgs {
+    const void *q, *k, *v;
+    void *out;
+    const float *state_in;
+    float *state_out;
+    const retnet_gate *gate;     // may be null
+    int batch, heads, seqlen, dk, dv, chunk;
+    retnet_dtype dtype;
+    long long pos0;
+    int rotate;
+    HeadGammas gam;
+    void *workspace;
+    size_t workspace_bytes;
+};
+size_t simt_workspace_bytes(int batch, int heads, int seqlen, int dk, int dv, int chunk);
+cudaError_t launch_chunkwise_simt(const ChunkwiseArgs &a, cudaStream_t stream);
+
+}  // namespace retnet

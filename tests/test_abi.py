@@ -1,0 +1,140 @@
+"""CPU checks of the C ABI: the library loads, exports every declared symbol,
+and host-side validation rejects bad calls before touching CUDA."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import linear_recurrent_sequence_02_b200 as rn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "retnet.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"RETNET_API[^;(]*?\b(retnet_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from linear_recurrent_sequence_02_b200.build import build
+    build()
+    return rn.load_library()
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for want in ("retnet_retention_chunkwise", "retnet_retention_step", "retnet_groupnorm_swish",
+                 "retnet_xpos_rotate", "retnet_default_gammas", "retnet_chunkwise_workspace_size",
+                 "retnet_check_device_errors", "retnet_status_string",
+                 "retnet_kernel_launch_count"):
+        assert want in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    # nothing else leaks out of the shared object under a retnet_ prefix
+    out = os.popen(f"nm -D --defined-only {rn.LIB_PATH}").read()
+    exported = sorted(set(re.findall(r"\b(retnet_\w+)\b", out)))
+    assert exported == declared_functions()
+
+
+def test_status_strings(lib):
+    assert rn.retnet_status_string(0) == "ok"
+    assert "invalid" in rn.retnet_status_string(1)
+    assert rn.retnet_status_string(99) == "unknown status"
+
+
+def test_default_gammas_match_closed_form(lib):
+    g = rn.retnet_default_gammas(16)
+    assert g[0] == 0.96875 and g[3] == 0.99609375
+    assert g[15] == np.float32(1 - 2.0 ** -20)
+    buf = (ctypes.c_float * 1)()
+    assert lib.retnet_default_gammas(0, buf) == 1
+    assert lib.retnet_default_gammas(257, buf) == 1
+    assert lib.retnet_default_gammas(4, None) == 1
+
+
+def _shape(B=1, H=4, n=256, dk=64, dv=64, dt=0):
+    return rn._Shape(B, H, n, dk, dv, dt)
+
+
+def test_workspace_size_validation(lib):
+    n = ctypes.c_size_t(0)
+    s = _shape()
+    assert lib.retnet_chunkwise_workspace_size(ctypes.byref(s), 64, 1, ctypes.byref(n)) == 0
+    assert n.value > 0
+    assert lib.retnet_chunkwise_workspace_size(ctypes.byref(s), 0, 1, ctypes.byref(n)) == 1
+    assert lib.retnet_chunkwise_workspace_size(ctypes.byref(s), 2048, 1, ctypes.byref(n)) == 1
+    bad = _shape(dk=96)
+    assert lib.retnet_chunkwise_workspace_size(ctypes.byref(bad), 64, 1, ctypes.byref(n)) == 2
+    neg = _shape(B=-1)
+    assert lib.retnet_chunkwise_workspace_size(ctypes.byref(neg), 64, 1, ctypes.byref(n)) == 1
+    assert lib.retnet_chunkwise_workspace_size(None, 64, 1, ctypes.byref(n)) == 1
+
+
+def _chunkwise(lib, q=16, k=16, v=16, out=16, gam=(0.9,) * 4, chunk=64, shape=None, pos0=0,
+               rotate=1, sin=None, sout=None, algo=1, ws=256, wsb=1 << 30):
+    s = shape or _shape()
+    g = None if gam is None else (ctypes.c_float * len(gam))(*gam)
+    P = ctypes.c_void_p
+    return lib.retnet_retention_chunkwise(P(q), P(k), P(v), g, chunk, P(out), ctypes.byref(s),
+                                          pos0, rotate, P(sin), P(sout), None, algo, P(ws), wsb,
+                                          None)
+
+
+def test_chunkwise_rejects_before_launch(lib):
+    # Fake, aligned, never-dereferenced addresses: every case must fail validation
+    assert _chunkwise(lib, q=None) == 1                    # null input
+    assert _chunkwise(lib, q=18) == 1                      # misaligned input
+    assert _chunkwise(lib, gam=None) == 1                  # no gammas
+    assert _chunkwise(lib, gam=(0.9, 0.9, 0.9, 1.5)) == 1  # gamma outside [0, 1]
+    assert _chunkwise(lib, gam=(0.9, 0.9, 0.9, float("nan"))) == 1
+    assert _chunkwise(lib, chunk=0) == 1
+    assert _chunkwise(lib, pos0=-1) == 1
+    assert _chunkwise(lib, rotate=2) == 1
+    assert _chunkwise(lib, sin=8) == 1                     # misaligned state
+    assert _chunkwise(lib, algo=7) == 1
+    assert _chunkwise(lib, shape=_shape(dk=80)) == 2       # unsupported head dim
+    assert _chunkwise(lib, ws=None) == 5                   # missing workspace
+    assert _chunkwise(lib, wsb=16) == 5                    # too small
+    assert _chunkwise(lib, ws=272) == 5                    # not 256-byte aligned
+    # an empty batch is a no-op that succeeds without touching memory
+    assert _chunkwise(lib, q=None, k=None, v=None, out=None, shape=_shape(B=0)) == 0
+
+
+def test_step_and_groupnorm_reject_before_launch(lib):
+    P = ctypes.c_void_p
+    g4 = (ctypes.c_float * 4)(0.9, 0.9, 0.9, 0.9)
+    assert lib.retnet_retention_step(None, P(16), P(16), g4, P(16), P(16), 2, 4, 64, 64, 0, 0, 1,
+                                     None) == 1
+    assert lib.retnet_retention_step(P(16), P(16), P(16), g4, P(20), P(16), 2, 4, 64, 64, 0, 0,
+                                     1, None) == 1
+    assert lib.retnet_retention_step(P(16), P(16), P(16), g4, P(16), P(16), 2, 4, 96, 64, 0, 0,
+                                     1, None) == 2
+    assert lib.retnet_retention_step(P(16), P(16), P(16), g4, P(16), P(16), 2, 4, 64, 64, 5, 0,
+                                     1, None) == 1
+    assert lib.retnet_retention_step(P(16), P(16), P(16), None, P(16), P(16), 2, 4, 64, 64, 0, 0,
+                                     1, None) == 1
+    assert lib.retnet_retention_step(None, None, None, g4, None, None, 0, 4, 64, 64, 0, 0, 1,
+                                     None) == 0
+    assert lib.retnet_groupnorm_swish(P(16), P(16), None, None, 1e-5, 10, 4, 60, 1, P(16),
+                                      None) == 1
+    assert lib.retnet_groupnorm_swish(P(16), None, None, None, 1e-5, 10, 4, 64, 1, P(16),
+                                      None) == 1
+    assert lib.retnet_groupnorm_swish(P(16), P(16), None, None, -1.0, 10, 4, 64, 1, P(16),
+                                      None) == 1
+    assert lib.retnet_groupnorm_swish(None, None, None, None, 1e-5, 0, 4, 64, 1, None, None) == 0
+    assert lib.retnet_xpos_rotate(P(16), P(16), 1, 4, 2, 6, 0, 0, None) == 1    # d % 8 != 0
+    assert lib.retnet_xpos_rotate(P(16), P(16), 1, 4, 2, 8, 0, -3, None) == 1   # pos0 < 0
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(1, 4, 2, 8)
+    with pytest.raises(ValueError):
+        rn.retnet_xpos_rotate(x)
