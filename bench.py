@@ -413,13 +413,89 @@ def run_ours(args, w, chunk):
         dist.destroy_process_group()
 
 
+def run_decode(args, w):
+    """Decode-only measurement: one timed step = one recurrent step for every
+    sequence of the batch (state seeded by an 8192-token GPU prefill)."""
+    import torch
+
+    import linear_recurrent_sequence_02_b200 as rn
+    from linear_recurrent_sequence_02_b200.build import build
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    build()
+    rn.load_library()
+    B, H, d, n = args.batch, w.heads, w.d, w.seqlen
+    gam = rn.retnet_default_gammas(H)
+    state = torch.empty(B, H, d, d, device=dev)
+    for b0 in range(0, B, 16):                       # seed the state slice by slice
+        b1 = min(B, b0 + 16)
+        q, k, v = wl.make_prefill_inputs_device(b1 - b0, H, n, d, w.scale, w.seed + b0, dev)
+        rn.retnet_retention_chunkwise(q, k, v, gam, w.chunk, state_out=state[b0:b1])
+        del q, k, v
+    torch.cuda.synchronize()
+    steps = w.decode_steps
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed + 7)
+    qd, kd, vd = ((torch.randn(steps, B, H, d, generator=gen, device=dev) * w.scale)
+                  .to(torch.bfloat16) for _ in range(3))
+    o = torch.empty(B, H, d, dtype=torch.bfloat16, device=dev)
+
+    def step(i):
+        rn.retnet_retention_step(qd[i % steps], kd[i % steps], vd[i % steps], gam, state,
+                                 n + i, out=o)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index or 0)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    stream = torch.cuda.current_stream(dev)
+    rn.retnet_profiler_reset()
+    rn.retnet_profiler_enable(True)
+    launches0 = rn.retnet_kernel_launch_count()
+    clocks.start()
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    rn.retnet_profiler_enable(False)
+    kern = rn.retnet_profiler_read()
+    ms = ev0.elapsed_time(ev1)
+    peaks, src = load_peaks()
+    tot, cnt = kern["retention_step"]
+    avg_s = tot / cnt / 1e3
+    bytes_step = B * H * (8 * d * d + 2 * 4 * d)
+    line = {
+        "metric": "decode steps/s (all sequences advance one token)", "value": args.steps / (ms / 1e3),
+        "unit": "steps/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 state, bf16 q/k/v", "data": "synthetic",
+        "config": {"workload": f"decode7b: H={H} d={d} batch {B}, state from an {n}-token prefill",
+                   "batch": B, "l2": "state larger than L2" if bytes_step > 126e6 else
+                   "state fits in L2 (L2-resident)"},
+        "tokens_per_s": B * args.steps / (ms / 1e3),
+        "roofline": {"kernel": "retention_step", "bound": "hbm", "achieved": bytes_step / avg_s / 1e9,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": bytes_step / avg_s / 1e9 / peaks["hbm_gbs"], "traffic": None,
+                     "peak_source": src, "work_per_launch": bytes_step},
+        "kernel_avg_us": avg_s * 1e6,
+        "gpu_launches": rn.retnet_kernel_launch_count() - launches0, "clocks": clock_info,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["layer200m", "layer3b", "long7b"], default="layer200m")
+    ap.add_argument("--workload", choices=["layer200m", "layer3b", "long7b", "decode7b"],
+                    default="layer200m")
+    ap.add_argument("--batch", type=int, default=128, help="decode7b batch")
     ap.add_argument("--chunk", type=int, default=0)
     ap.add_argument("--algo", choices=["auto", "simt", "tensor"], default="auto")
     ap.add_argument("--e2e-steps", type=int, default=20)
@@ -429,6 +505,8 @@ def main():
     chunk = args.chunk or w.chunk
     if args.impl == "reference":
         run_reference(args, w, chunk)
+    elif args.workload == "decode7b":
+        run_decode(args, w)
     else:
         run_ours(args, w, chunk)
 

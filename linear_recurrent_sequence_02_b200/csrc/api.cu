@@ -47,10 +47,18 @@ static retnet_status check_shape(const retnet_shape *s, int chunk) {
     return RETNET_OK;
 }
 
-static retnet_algo resolve_algo(const retnet_shape *s, int chunk, retnet_algo algo) {
-    (void)s; (void)chunk;
-    if (algo == RETNET_ALGO_AUTO) return RETNET_ALGO_SIMT;
+// Kernel family for a call; gammas == nullptr answers for any admissible decay.
+static retnet_algo resolve_algo(const retnet_shape *s, int chunk, retnet_algo algo,
+                                const float *gammas) {
+    const bool shape_ok = tc_shape_ok(s->dk, s->dv, s->dtype, chunk);
+    const bool gam_ok = !gammas || tc_gammas_ok(chunk, gammas, s->heads);
+    if (algo == RETNET_ALGO_AUTO) return shape_ok && gam_ok ? RETNET_ALGO_TENSOR : RETNET_ALGO_SIMT;
     return algo;
+}
+
+static size_t workspace_for(const retnet_shape *s, int chunk, retnet_algo resolved) {
+    if (resolved == RETNET_ALGO_TENSOR) return tc_workspace_bytes(s->batch, s->heads, s->seqlen, chunk);
+    return simt_workspace_bytes(s->batch, s->heads, s->seqlen, s->dk, s->dv, chunk);
 }
 
 }  // namespace retnet
@@ -98,10 +106,17 @@ retnet_status retnet_chunkwise_workspace_size(const retnet_shape *shape, int chu
     if (!bytes) return RETNET_ERR_INVALID_ARG;
     retnet_status st = check_shape(shape, chunk);
     if (st != RETNET_OK) return st;
-    retnet_algo a = resolve_algo(shape, chunk, algo);
-    if (a != RETNET_ALGO_SIMT) return RETNET_ERR_UNSUPPORTED;
-    *bytes = simt_workspace_bytes(shape->batch, shape->heads, shape->seqlen, shape->dk,
-                                  shape->dv, chunk);
+    if (algo != RETNET_ALGO_AUTO && algo != RETNET_ALGO_SIMT && algo != RETNET_ALGO_TENSOR)
+        return RETNET_ERR_INVALID_ARG;
+    if (algo == RETNET_ALGO_TENSOR && !tc_shape_ok(shape->dk, shape->dv, shape->dtype, chunk))
+        return RETNET_ERR_UNSUPPORTED;
+    size_t n = workspace_for(shape, chunk, RETNET_ALGO_SIMT);
+    if (resolve_algo(shape, chunk, algo, nullptr) == RETNET_ALGO_TENSOR) {
+        // AUTO may still pick SIMT at call time (decays outside the fold's range)
+        size_t t = workspace_for(shape, chunk, RETNET_ALGO_TENSOR);
+        n = algo == RETNET_ALGO_TENSOR ? t : (t > n ? t : n);
+    }
+    *bytes = n;
     return RETNET_OK;
 }
 
@@ -132,10 +147,12 @@ retnet_status retnet_retention_chunkwise(const void *q, const void *k, const voi
         if (tokens > 0 && (!gate->g || !aligned16(gate->g))) return RETNET_ERR_INVALID_ARG;
         if (!(gate->eps >= 0.f)) return RETNET_ERR_INVALID_ARG;
     }
-    retnet_algo resolved = resolve_algo(shape, chunk, algo);
-    if (resolved != RETNET_ALGO_SIMT) return RETNET_ERR_UNSUPPORTED;
-    size_t need = simt_workspace_bytes(shape->batch, shape->heads, shape->seqlen, shape->dk,
-                                       shape->dv, chunk);
+    retnet_algo resolved = resolve_algo(shape, chunk, algo, gammas);
+    if (resolved == RETNET_ALGO_TENSOR &&
+        (!tc_shape_ok(shape->dk, shape->dv, shape->dtype, chunk) ||
+         !tc_gammas_ok(chunk, gammas, shape->heads)))
+        return RETNET_ERR_UNSUPPORTED;
+    size_t need = workspace_for(shape, chunk, resolved);
     if (need > 0 && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)))
         return RETNET_ERR_WORKSPACE;
     if (shape->batch == 0) return RETNET_OK;
@@ -146,7 +163,12 @@ retnet_status retnet_retention_chunkwise(const void *q, const void *k, const voi
     a.dk = shape->dk; a.dv = shape->dv; a.chunk = chunk; a.dtype = shape->dtype;
     a.pos0 = pos0; a.rotate = rotate; a.workspace = workspace;
     a.workspace_bytes = workspace_bytes;
-    RETNET_CUDA_TRY(launch_chunkwise_simt(a, (cudaStream_t)stream));
+    if (resolved == RETNET_ALGO_TENSOR) {
+        if ((uintptr_t)workspace & 1023u) return RETNET_ERR_WORKSPACE;
+        RETNET_CUDA_TRY(launch_chunkwise_tc(a, gammas, (cudaStream_t)stream));
+    } else {
+        RETNET_CUDA_TRY(launch_chunkwise_simt(a, (cudaStream_t)stream));
+    }
     return RETNET_OK;
 }
 

@@ -42,4 +42,12 @@ struct ChunkwiseArgs {
 size_t simt_workspace_bytes(int batch, int heads, int seqlen, int dk, int dv, int chunk);
 cudaError_t launch_chunkwise_simt(const ChunkwiseArgs &a, cudaStream_t stream);
 
+// chunkwise_tc.cu ----------------------------------------------------------
+// Shape/dtype/chunk admitted by the tensor-core path.
+bool tc_shape_ok(int dk, int dv, retnet_dtype dtype, int chunk);
+// Every head's decay admits the decay fold: gamma > 0 and chunk*log2(1/gamma) <= 100.
+bool tc_gammas_ok(int chunk, const float *gammas, int heads);
+size_t tc_workspace_bytes(int batch, int heads, int seqlen, int chunk);
+cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cudaStream_t stream);
+
 }  // namespace retnet

@@ -9,26 +9,37 @@
 
 namespace retnet {
 
-__global__ void rotation_table_kernel(float2 *__restrict__ table, int n, int half,
-                                      int d, long long pos0) {
-    long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    long long total = (long long)n * half;
-    if (idx >= total) return;
-    int t = (int)(idx / half);
-    int j = (int)(idx - (long long)t * half);
-    table[idx] = rotation_cs(pos0 + t, j, d);
+// Grid (ceil(n / kTablePositions), ceil(half / 128)): each thread owns one
+// pair index j, forms theta_j once and fills kTablePositions positions, so
+// the float64 power is paid once per 32 table entries.
+constexpr int kTablePositions = 32;
+
+__global__ void __launch_bounds__(128)
+rotation_table_kernel(float2 *__restrict__ table, int n, int half, int d, long long pos0) {
+    const int j = blockIdx.y * 128 + threadIdx.x;
+    if (j >= half) return;
+    const double two_pi = 6.283185307179586476925286766559;
+    const double theta = pow(10000.0, -2.0 * (double)j / (double)d);
+    const int t0 = blockIdx.x * kTablePositions;
+    const int t1 = min(n, t0 + kTablePositions);
+    for (int t = t0; t < t1; ++t) {
+        const double a = (double)(pos0 + t) * theta;
+        const double r = a - two_pi * rint(a / two_pi);
+        float sn, cs;
+        sincosf((float)r, &sn, &cs);
+        table[(size_t)t * half + j] = make_float2(cs, sn);
+    }
 }
 
 cudaError_t launch_rotation_table(float2 *table, int n, int d, long long pos0,
                                   cudaStream_t stream) {
-    int half = d / 2;
-    long long total = (long long)n * half;
-    if (total == 0) return cudaSuccess;
-    int threads = 256;
-    long long blocks = (total + threads - 1) / threads;
+    const int half = d / 2;
+    if (n == 0 || half == 0) return cudaSuccess;
+    dim3 grid((unsigned)((n + kTablePositions - 1) / kTablePositions),
+              (unsigned)((half + 127) / 128));
     {
         KernelTimer timer("rotation_table", stream);
-        rotation_table_kernel<<<(unsigned)blocks, threads, 0, stream>>>(table, n, half, d, pos0);
+        rotation_table_kernel<<<grid, 128, 0, stream>>>(table, n, half, d, pos0);
     }
     count_launch();
     return cudaGetLastError();

@@ -13,6 +13,8 @@
 // across the cluster through distributed shared memory, by cluster rank 0.
 #include <cooperative_groups.h>
 
+#include <cmath>
+
 #include "kernels.h"
 
 namespace cg = cooperative_groups;
@@ -22,87 +24,107 @@ namespace retnet {
 constexpr int kStepThreads = 256;
 constexpr int kStepRows = 32;       // state rows per CTA
 
+// (cos, sin) of pos * theta_j for the pairs of this step, formed on the host
+// in float64 (the position is a host scalar), j < dk / 2 <= 128.
+struct StepRotation {
+    float2 cs[128];
+};
+
 template <typename T>
+__device__ __forceinline__ void load4(const T *p, float *o);
+template <>
+__device__ __forceinline__ void load4<float>(const float *p, float *o) {
+    float4 f = *reinterpret_cast<const float4 *>(p);
+    o[0] = f.x; o[1] = f.y; o[2] = f.z; o[3] = f.w;
+}
+template <>
+__device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16 *p, float *o) {
+    uint2 u = *reinterpret_cast<const uint2 *>(p);
+    float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&u.x));
+    float2 b = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&u.y));
+    o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y;
+}
+
+template <typename T, int DV>
 __global__ void __launch_bounds__(kStepThreads)
 retention_step_kernel(const T *__restrict__ q, const T *__restrict__ k,
-                      const T *__restrict__ v, HeadGammas gam, float *__restrict__ state,
-                      T *__restrict__ out, int heads, int dk, int dv, long long pos,
+                      const T *__restrict__ v, HeadGammas gam, StepRotation rot,
+                      float *__restrict__ state, T *__restrict__ out, int heads, int dk,
                       int rotate) {
+    constexpr int NCG = DV / 4;                      // float4 column groups
+    constexpr int NRL = kStepThreads / NCG;          // row lanes
+    constexpr int RPL = kStepRows / NRL;             // rows per lane: 2, 4 or 8
     cg::cluster_group cluster = cg::this_cluster();
     const int bh = blockIdx.x;                       // sequence * heads + head
     const int h = bh % heads;
-    const int slab = blockIdx.y;                     // == rank in the (1, dk/32) cluster
-    const int row0 = slab * kStepRows;
+    const int row0 = blockIdx.y * kStepRows;         // blockIdx.y == cluster rank
     const float g = gam.g[h];
+    const int cgi = threadIdx.x % NCG;
+    const int rl = threadIdx.x / NCG;
 
     __shared__ float qs[kStepRows], ks[kStepRows];
     __shared__ float4 red[kStepThreads];
-    __shared__ float4 partial[64];                   // dv / 4 <= 64
+    __shared__ float4 partial[NCG];
 
-    // Rotated q, k entries of this CTA's rows (row pairs are never split:
-    // kStepRows is even and row0 is a multiple of it).
-    const T *qh = q + (size_t)bh * dk;
-    const T *kh = k + (size_t)bh * dk;
+    // Issue this thread's state loads first: they do not depend on q, k, v.
+    float *S = state + (size_t)bh * dk * DV;
+    float4 s[RPL];
+#pragma unroll
+    for (int i = 0; i < RPL; ++i)
+        s[i] = reinterpret_cast<const float4 *>(S + (size_t)(row0 + rl + i * NRL) * DV)[cgi];
+
+    // Rotated q, k entries of this CTA's rows (pairs never straddle CTAs).
     if (threadIdx.x < kStepRows / 2) {
-        int r = row0 + 2 * threadIdx.x;
-        float q0 = to_f32(qh[r]), q1 = to_f32(qh[r + 1]);
-        float k0 = to_f32(kh[r]), k1 = to_f32(kh[r + 1]);
+        const int r = row0 + 2 * threadIdx.x;
+        const T *qh = q + (size_t)bh * dk + r;
+        const T *kh = k + (size_t)bh * dk + r;
+        float q0 = to_f32(qh[0]), q1 = to_f32(qh[1]);
+        float k0 = to_f32(kh[0]), k1 = to_f32(kh[1]);
         if (rotate) {
-            float2 cs = rotation_cs(pos, r / 2, dk);
-            float a = q0, b = q1;
-            q0 = a * cs.x - b * cs.y;
-            q1 = a * cs.y + b * cs.x;
-            a = k0; b = k1;
-            k0 = a * cs.x - b * cs.y;
-            k1 = a * cs.y + b * cs.x;
+            const float2 cs = rot.cs[r / 2];
+            float a = q0;
+            q0 = a * cs.x - q1 * cs.y;
+            q1 = a * cs.y + q1 * cs.x;
+            a = k0;
+            k0 = a * cs.x - k1 * cs.y;
+            k1 = a * cs.y + k1 * cs.x;
         }
         qs[2 * threadIdx.x] = q0; qs[2 * threadIdx.x + 1] = q1;
         ks[2 * threadIdx.x] = k0; ks[2 * threadIdx.x + 1] = k1;
     }
-
-    const int ncg = dv / 4;                          // float4 column groups
-    const int nrl = kStepThreads / ncg;              // row lanes
-    const int cgi = threadIdx.x % ncg;
-    const int rl = threadIdx.x / ncg;
     float vv[4];
-    {
-        const T *vh = v + (size_t)bh * dv + cgi * 4;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) vv[i] = to_f32(vh[i]);
-    }
+    load4<T>(v + (size_t)bh * DV + cgi * 4, vv);
     __syncthreads();
 
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float *S = state + (size_t)bh * dk * dv;
-    const int rows_per_lane = kStepRows / nrl;       // 2, 4 or 8
-#pragma unroll 8
-    for (int i = 0; i < rows_per_lane; ++i) {
-        int rr = rl + i * nrl;                       // row within the slab
-        float4 *p = reinterpret_cast<float4 *>(S + (size_t)(row0 + rr) * dv) + cgi;
-        float4 s = *p;
-        float kr = ks[rr], qr = qs[rr];
-        s.x = fmaf(g, s.x, kr * vv[0]);
-        s.y = fmaf(g, s.y, kr * vv[1]);
-        s.z = fmaf(g, s.z, kr * vv[2]);
-        s.w = fmaf(g, s.w, kr * vv[3]);
-        *p = s;
-        acc.x = fmaf(qr, s.x, acc.x);
-        acc.y = fmaf(qr, s.y, acc.y);
-        acc.z = fmaf(qr, s.z, acc.z);
-        acc.w = fmaf(qr, s.w, acc.w);
+#pragma unroll
+    for (int i = 0; i < RPL; ++i) {
+        const int rr = rl + i * NRL;
+        const float kr = ks[rr], qr = qs[rr];
+        float4 t = s[i];
+        t.x = fmaf(g, t.x, kr * vv[0]);
+        t.y = fmaf(g, t.y, kr * vv[1]);
+        t.z = fmaf(g, t.z, kr * vv[2]);
+        t.w = fmaf(g, t.w, kr * vv[3]);
+        reinterpret_cast<float4 *>(S + (size_t)(row0 + rr) * DV)[cgi] = t;
+        acc.x = fmaf(qr, t.x, acc.x);
+        acc.y = fmaf(qr, t.y, acc.y);
+        acc.z = fmaf(qr, t.z, acc.z);
+        acc.w = fmaf(qr, t.w, acc.w);
     }
     red[threadIdx.x] = acc;
     __syncthreads();
-    if (threadIdx.x < ncg) {
+    if (threadIdx.x < NCG) {
         float4 t = red[threadIdx.x];
-        for (int l = 1; l < nrl; ++l) {
-            float4 u = red[l * ncg + threadIdx.x];
+#pragma unroll
+        for (int l = 1; l < NRL; ++l) {
+            float4 u = red[l * NCG + threadIdx.x];
             t.x += u.x; t.y += u.y; t.z += u.z; t.w += u.w;
         }
         partial[threadIdx.x] = t;
     }
     cluster.sync();
-    if (cluster.block_rank() == 0 && threadIdx.x < ncg) {
+    if (cluster.block_rank() == 0 && threadIdx.x < NCG) {
         float4 t = partial[threadIdx.x];
         const unsigned nblk = cluster.num_blocks();
         for (unsigned r = 1; r < nblk; ++r) {
@@ -110,7 +132,7 @@ retention_step_kernel(const T *__restrict__ q, const T *__restrict__ k,
             float4 u = rp[threadIdx.x];
             t.x += u.x; t.y += u.y; t.z += u.z; t.w += u.w;
         }
-        T *oh = out + (size_t)bh * dv + threadIdx.x * 4;
+        T *oh = out + (size_t)bh * DV + threadIdx.x * 4;
         oh[0] = from_f32<T>(t.x);
         oh[1] = from_f32<T>(t.y);
         oh[2] = from_f32<T>(t.z);
@@ -119,11 +141,11 @@ retention_step_kernel(const T *__restrict__ q, const T *__restrict__ k,
     cluster.sync();       // keep every CTA's shared memory alive until rank 0 has read it
 }
 
-cudaError_t launch_retention_step(const void *q, const void *k, const void *v,
-                                  const HeadGammas &gam, float *state, void *out, int batch,
-                                  int heads, int dk, int dv, retnet_dtype dtype, long long pos,
-                                  int rotate, cudaStream_t stream) {
-    if (batch == 0) return cudaSuccess;
+template <typename T, int DV>
+static cudaError_t launch_step_typed(const void *q, const void *k, const void *v,
+                                     const HeadGammas &gam, const StepRotation &rot,
+                                     float *state, void *out, int batch, int heads, int dk,
+                                     int rotate, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(batch * heads), (unsigned)(dk / kStepRows), 1);
     cfg.blockDim = dim3(kStepThreads, 1, 1);
@@ -136,17 +158,45 @@ cudaError_t launch_retention_step(const void *q, const void *k, const void *v,
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t err;
     KernelTimer timer("retention_step", stream);
-    if (dtype == RETNET_BF16)
-        err = cudaLaunchKernelEx(&cfg, retention_step_kernel<__nv_bfloat16>,
-                                 (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k,
-                                 (const __nv_bfloat16 *)v, gam, state, (__nv_bfloat16 *)out,
-                                 heads, dk, dv, pos, rotate);
-    else
-        err = cudaLaunchKernelEx(&cfg, retention_step_kernel<float>, (const float *)q,
-                                 (const float *)k, (const float *)v, gam, state, (float *)out,
-                                 heads, dk, dv, pos, rotate);
+    return cudaLaunchKernelEx(&cfg, retention_step_kernel<T, DV>, (const T *)q, (const T *)k,
+                              (const T *)v, gam, rot, state, (T *)out, heads, dk, rotate);
+}
+
+template <typename T>
+static cudaError_t launch_step_t(const void *q, const void *k, const void *v,
+                                 const HeadGammas &gam, const StepRotation &rot, float *state,
+                                 void *out, int batch, int heads, int dk, int dv, int rotate,
+                                 cudaStream_t stream) {
+    switch (dv) {
+        case 64: return launch_step_typed<T, 64>(q, k, v, gam, rot, state, out, batch, heads, dk, rotate, stream);
+        case 128: return launch_step_typed<T, 128>(q, k, v, gam, rot, state, out, batch, heads, dk, rotate, stream);
+        case 256: return launch_step_typed<T, 256>(q, k, v, gam, rot, state, out, batch, heads, dk, rotate, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_retention_step(const void *q, const void *k, const void *v,
+                                  const HeadGammas &gam, float *state, void *out, int batch,
+                                  int heads, int dk, int dv, retnet_dtype dtype, long long pos,
+                                  int rotate, cudaStream_t stream) {
+    if (batch == 0) return cudaSuccess;
+    StepRotation rot;
+    const double two_pi = 6.283185307179586476925286766559;
+    for (int j = 0; j < 128; ++j) rot.cs[j] = make_float2(1.f, 0.f);
+    if (rotate) {
+        for (int j = 0; j < dk / 2; ++j) {
+            const double theta = std::pow(10000.0, -2.0 * j / dk);
+            const double a = (double)pos * theta;
+            const double r = a - two_pi * std::nearbyint(a / two_pi);
+            rot.cs[j] = make_float2((float)std::cos(r), (float)std::sin(r));
+        }
+    }
+    cudaError_t err = dtype == RETNET_BF16
+                          ? launch_step_t<__nv_bfloat16>(q, k, v, gam, rot, state, out, batch,
+                                                         heads, dk, dv, rotate, stream)
+                          : launch_step_t<float>(q, k, v, gam, rot, state, out, batch, heads,
+                                                 dk, dv, rotate, stream);
     count_launch();
     return err;
 }

@@ -28,7 +28,7 @@ from dataclasses import dataclass, field
 import numpy as np
 
 __all__ = ["Workload", "WORKLOADS", "round_to_bf16", "make_prefill_inputs",
-           "make_decode_inputs", "normal"]
+           "make_decode_inputs", "make_prefill_inputs_device", "normal"]
 
 
 @dataclass(frozen=True)
@@ -117,3 +117,25 @@ def make_decode_inputs(batch: int, heads: int, steps: int, d: int, dtype: str,
     k = normal(rng, (steps, batch, heads, d), scale, dtype)
     v = normal(rng, (steps, batch, heads, d), scale, dtype)
     return q, k, v
+
+
+def make_prefill_inputs_device(batch: int, heads: int, seqlen: int, d: int, scale: float,
+                               seed: int, device, dtype=None):
+    """q, k, v [B, n, H, d] drawn on `device` with torch's seeded generator.
+
+    Same distribution as make_prefill_inputs (standard normal times `scale`,
+    rounded to the storage dtype, bf16 by default), for workloads too large
+    to draw on the host (the 8192-token prefills that seed decode states at
+    batch 32 and 128).  The draw order is q, k, v.
+    """
+    import torch
+    dtype = torch.bfloat16 if dtype is None else dtype
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    shape = (batch, seqlen, heads, d)
+    out = []
+    for _ in range(3):
+        x = torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
+        out.append((x * scale).to(dtype))
+        del x
+    return tuple(out)
