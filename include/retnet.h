@@ -157,6 +157,33 @@ RETNET_API retnet_status retnet_retention_chunkwise(const void *q, const void *k
                                          void *workspace, size_t workspace_bytes,
                                          retnet_stream_t stream);
 
+/* ---- Prefill without any allocation ---------------------------------
+ * No counterpart on the pages: an addition for callers that cannot
+ * allocate device memory at run time -- for example a plugin inside a
+ * serving process that reserves all device memory at start-up and hands
+ * its plugins no allocator, or a latency-critical path where cudaMalloc's
+ * implicit device-wide synchronisation is not allowed.  It runs exactly the
+ * kernels of retnet_retention_chunkwise (same arguments and semantics, minus
+ * the workspace) on a scratch array compiled into the library:
+ *   - at most RETNET_NOALLOC_SCRATCH_BYTES of scratch per call; a call that
+ *     would need more (see retnet_chunkwise_workspace_size for the chosen
+ *     kernel family) returns RETNET_ERR_WORKSPACE and enqueues nothing;
+ *   - every GPU that loads the library holds that array until exit;
+ *   - it calls no cudaMalloc, cudaFree or other allocating routine;
+ *   - it works on the current device (`stream` must belong to it).  Its
+ *     first call on a device looks up the array's device address there
+ *     (cudaGetSymbolAddress); make that first call before any stream
+ *     capture on that device;
+ *   - all calls on a device share the one array and it keeps the last
+ *     call's contents (nothing in it needs to start at zero): calls whose
+ *     work overlaps on the GPU (different streams, no ordering) race on it
+ *     and must be serialised by the caller. */
+#define RETNET_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+RETNET_API retnet_status retnet_retention_chunkwise_noalloc(
+    const void *q, const void *k, const void *v, const float *gammas, int chunk, void *out,
+    const retnet_shape *shape, long long pos0, int rotate, const float *state_in,
+    float *state_out, const retnet_gate *gate, retnet_algo algo, retnet_stream_t stream);
+
 /* One recurrent decode step for every (sequence, head) ("Summary": the
  * recurrent form costs O(1) per step and needs no KV cache).
  *   q, k [batch, heads, dk], v [batch, heads, dv]: this token, device, dtype.
