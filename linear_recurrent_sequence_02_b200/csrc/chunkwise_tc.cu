@@ -48,55 +48,84 @@ struct TcHeadParams {
 };
 
 // ------------------------------------------------------------------ prep
-// One thread: 8 consecutive elements (4 rotation pairs) of q and of k for
-// one (b, t, h).  Writes Qt, Kt in [b*H + h][t][:] layout.
+// One CTA per token t: its 128 (cos, sin) pairs are formed once (angle
+// (pos0 + t) * theta_j in float64, reduced to [-pi, pi], then a float32
+// sincos) and applied to every (sequence, head) row of q and k at that
+// token, together with the decay fold.  Writes Qt, Kt in [b*H + h][t][:].
+struct TcPrepParams {
+    double theta[kD / 2];          // 10000^(-2j/256), formed on the host
+    float log2g[kMaxHeads];        // log2(gamma_h)
+};
+
 __global__ void __launch_bounds__(256)
 tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-               const float2 *__restrict__ table, TcHeadParams hp, __nv_bfloat16 *__restrict__ qt,
-               __nv_bfloat16 *__restrict__ kt, int batch, int heads, int n, int chunk,
-               int rotate) {
-    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    const long long total = (long long)batch * n * heads * (kD / 8);
-    if (idx >= total) return;
-    const int part = (int)(idx % (kD / 8));
-    const long long bth = idx / (kD / 8);
-    const int h = (int)(bth % heads);
-    const long long bt = bth / heads;
-    const int t = (int)(bt % n);
-    const int b = (int)(bt / n);
-    const int i = t % chunk;
-    const float e = (float)(i + 1) * hp.log2g[h];
-    const float sq = exp2f(e), sk = exp2f(-e);
-    float xq[8], xk[8];
-    load8(q + bth * kD + part * 8, xq);
-    load8(k + bth * kD + part * 8, xk);
-    float oq[8], ok[8];
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        float c = sq, s = 0.f, ck = sk, sk2 = 0.f;
+               TcPrepParams pp, __nv_bfloat16 *__restrict__ qt, __nv_bfloat16 *__restrict__ kt,
+               int batch, int heads, int n, int chunk, long long pos0, int rotate) {
+    __shared__ float2 cs[kD / 2];
+    const int t = blockIdx.x;
+    if (threadIdx.x < kD / 2) {
+        float2 v = make_float2(1.f, 0.f);
         if (rotate) {
-            float2 cs = table[(size_t)t * (kD / 2) + part * 4 + p];
-            c = cs.x * sq; s = cs.y * sq;
-            ck = cs.x * sk; sk2 = cs.y * sk;
+            const double two_pi = 6.283185307179586476925286766559;
+            const double inv_two_pi = 0.15915494309189533576888376337251;
+            const double a = (double)(pos0 + t) * pp.theta[threadIdx.x];
+            const double red = a - two_pi * rint(a * inv_two_pi);
+            float sn, cn;
+            sincosf((float)red, &sn, &cn);
+            v = make_float2(cn, sn);
         }
-        float a = xq[2 * p], bb = xq[2 * p + 1];
-        oq[2 * p] = a * c - bb * s;
-        oq[2 * p + 1] = a * s + bb * c;
-        a = xk[2 * p]; bb = xk[2 * p + 1];
-        ok[2 * p] = a * ck - bb * sk2;
-        ok[2 * p + 1] = a * sk2 + bb * ck;
+        cs[threadIdx.x] = v;
     }
-    const size_t dst = (((size_t)b * heads + h) * n + t) * kD + part * 8;
-    store8(qt + dst, oq);
-    store8(kt + dst, ok);
+    __syncthreads();
+    const int i = t % chunk;                        // index inside the chunk
+    const int tasks = batch * heads * (kD / 8);
+    for (int task = threadIdx.x; task < tasks; task += blockDim.x) {
+        const int part = task % (kD / 8);
+        const int bhi = task / (kD / 8);
+        const int h = bhi % heads, b = bhi / heads;
+        const float e = (float)(i + 1) * pp.log2g[h];
+        const float sq = exp2f(e), sk = exp2f(-e);
+        const size_t src = (((size_t)b * n + t) * heads + h) * kD + part * 8;
+        float xq[8], xk[8], oq[8], ok[8];
+        load8(q + src, xq);
+        load8(k + src, xk);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float2 r = cs[part * 4 + p];
+            const float cq = r.x * sq, sq2 = r.y * sq, ck = r.x * sk, sk2 = r.y * sk;
+            float a = xq[2 * p], bb = xq[2 * p + 1];
+            oq[2 * p] = a * cq - bb * sq2;
+            oq[2 * p + 1] = a * sq2 + bb * cq;
+            a = xk[2 * p]; bb = xk[2 * p + 1];
+            ok[2 * p] = a * ck - bb * sk2;
+            ok[2 * p + 1] = a * sk2 + bb * ck;
+        }
+        const size_t dst = (((size_t)b * heads + h) * n + t) * kD + part * 8;
+        store8(qt + dst, oq);
+        store8(kt + dst, ok);
+    }
 }
 
 // ------------------------------------------------------------------ state pass
+// One CTA per (sequence, head, 128x128 quarter of S).  Warp 0 streams Kt and
+// V sub-tiles of 128 tokens through a 3-stage TMA ring; warp 1 accumulates
+// U_c = Kt_c^T V_c of every chunk into one of two TMEM buffers (M = d_k
+// quarter, N = d_v quarter, both operands MN-major); warps 2-5 keep the
+// running state row in registers, S <- g^L (S + U_c), hand the buffer back
+// as soon as it is read, and write S_prev of the next chunk (bf16) or the
+// final state (f32).  The tensor core never waits for the state update.
 struct TcStateSmem {
     static constexpr int kStages = 3;
     static constexpr uint32_t kStage = 4 * kBox;       // Kt 128x128 + V 128x128
     static constexpr uint32_t kBytes = kStages * kStage + 1024;
 };
+
+__device__ __forceinline__ void store_bf16_row(__nv_bfloat16 *dst, const float *v, int count) {
+    for (int i = 0; i < count; i += 8)
+        *reinterpret_cast<uint4 *>(dst + i) =
+            make_uint4(sm100::pack_bf16x2(v[i], v[i + 1]), sm100::pack_bf16x2(v[i + 2], v[i + 3]),
+                       sm100::pack_bf16x2(v[i + 4], v[i + 5]), sm100::pack_bf16x2(v[i + 6], v[i + 7]));
+}
 
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -106,7 +135,7 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     constexpr int S = TcStateSmem::kStages;
-    __shared__ uint64_t full[S], empty[S], acc_full, acc_ready;
+    __shared__ uint64_t full[S], empty[S], acc_full[2], acc_free[2];
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
@@ -121,13 +150,15 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(&acc_full, 1);
-        mbar_init(&acc_ready, 128);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&acc_full[x], 1);
+            mbar_init(&acc_free[x], 128);
+        }
         abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(&tmem_slot, 128);
+        tmem_alloc(&tmem_slot, 256);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -162,11 +193,13 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(128, 128, 1, 1);
             int it = 0;
-            for (int c = 0; c < nchunks; ++c) {
-                if (!mbar_wait(&acc_ready, c & 1, &abort_flag, err)) break;
+            bool ok = true;
+            for (int c = 0; ok && c < nchunks; ++c) {
+                const int buf = c & 1;
+                if (c >= 2 && !mbar_wait(&acc_free[buf], ((c - 2) >> 1) & 1, &abort_flag, err)) break;
                 tc_fence_after();
                 const int L = min(chunk, n - c * chunk);
-                bool ok = true;
+                uint32_t accumulate = 0;
                 for (int st = 0; st * kBlk < L; ++st, ++it) {
                     const int s = it % S;
                     if (!mbar_wait(&full[s], (it / S) & 1, &abort_flag, err)) { ok = false; break; }
@@ -177,89 +210,61 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     for (int ks = 0; ks < kBlk / 16; ++ks) {
                         // A = Kt^T (M = d_k, K = tokens), B = V (N = d_v, K = tokens):
                         // both MN-major; 16 tokens = two 8-row atoms = 2048 B.
-                        uint64_t ad = smem_desc_sw128(kb + ks * 2048, kBox, 1024);
-                        uint64_t bd = smem_desc_sw128(vb + ks * 2048, kBox, 1024);
-                        mma_bf16(tmem, ad, bd, idesc, 1u);
+                        const uint64_t ad = smem_desc_sw128(kb + ks * 2048, kBox, 1024);
+                        const uint64_t bd = smem_desc_sw128(vb + ks * 2048, kBox, 1024);
+                        mma_bf16(tmem + 128 * buf, ad, bd, idesc, accumulate);
+                        accumulate = 1;
                     }
                     mma_commit(&empty[s]);
                 }
-                if (!ok) break;
-                mma_commit(&acc_full);
+                if (ok) mma_commit(&acc_full[buf]);
             }
         }
     } else {
-        // epilogue warpgroup: warp w owns TMEM lanes 32*(w%4) .. +31
+        // state warpgroup: warp w owns TMEM lanes 32*(w%4) .. +31 = rows of the d_k half
         const int q4 = warp % 4;
-        const int row = 32 * q4 + lane;                      // row of the d_k half
+        const int row = 32 * q4 + lane;
         const int krow = 128 * mh + row;                     // row of S
-        const uint32_t taddr = tmem + ((uint32_t)(32 * q4) << 16);
+        const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
         const size_t sbase = ((size_t)bh * kD + krow) * kD + 128 * nh;
-        // initial state -> TMEM and S_prev[0]
-        {
-            __nv_bfloat16 *dst = s_prev + (((size_t)bh * nchunks + 0) * kD + krow) * kD + 128 * nh;
-#pragma unroll 1
-            for (int cb = 0; cb < 4; ++cb) {
-                uint32_t r[32];
-                if (state_in) {
-                    const float4 *src = reinterpret_cast<const float4 *>(state_in + sbase + 32 * cb);
+        float st[128];
+        if (state_in) {
+            const float4 *src = reinterpret_cast<const float4 *>(state_in + sbase);
 #pragma unroll
-                    for (int v4 = 0; v4 < 8; ++v4) {
-                        float4 f = src[v4];
-                        r[4 * v4] = __float_as_uint(f.x); r[4 * v4 + 1] = __float_as_uint(f.y);
-                        r[4 * v4 + 2] = __float_as_uint(f.z); r[4 * v4 + 3] = __float_as_uint(f.w);
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) r[e] = 0u;
-                }
-                tmem_st32(taddr + 32 * cb, r);
-                uint4 *o = reinterpret_cast<uint4 *>(dst + 32 * cb);
-#pragma unroll
-                for (int v = 0; v < 4; ++v)
-                    o[v] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * v]), __uint_as_float(r[8 * v + 1])),
-                                      pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
-                                      pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
-                                      pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
+            for (int v4 = 0; v4 < 32; ++v4) {
+                const float4 f = src[v4];
+                st[4 * v4] = f.x; st[4 * v4 + 1] = f.y; st[4 * v4 + 2] = f.z; st[4 * v4 + 3] = f.w;
             }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&acc_ready);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 128; ++e) st[e] = 0.f;
         }
+        store_bf16_row(s_prev + ((size_t)bh * nchunks * kD + krow) * kD + 128 * nh, st, 128);
         for (int c = 0; c < nchunks; ++c) {
-            if (!warp_wait(&acc_full, c & 1, &abort_flag, err)) break;
+            const int buf = c & 1;
+            if (!warp_wait(&acc_full[buf], (c >> 1) & 1, &abort_flag, err)) break;
             tc_fence_after();
             const bool last = (c == nchunks - 1);
             const float decay = last ? hp.decay_last[h] : hp.decay_chunk[h];
-#pragma unroll 1
+#pragma unroll
             for (int cb = 0; cb < 4; ++cb) {
-                uint32_t r[32];
-                tmem_ld32(taddr + 32 * cb, r);
+                uint32_t v[32];
+                tmem_ld32(tmem + 128 * buf + lane_off + 32 * cb, v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * decay);
-                if (!last) {
-                    tmem_st32(taddr + 32 * cb, r);
-                    __nv_bfloat16 *dst =
-                        s_prev + (((size_t)bh * nchunks + c + 1) * kD + krow) * kD + 128 * nh + 32 * cb;
-                    uint4 *o = reinterpret_cast<uint4 *>(dst);
-#pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        o[v] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * v]), __uint_as_float(r[8 * v + 1])),
-                                          pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
-                                          pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
-                                          pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
-                } else if (state_out) {
-                    float4 *o = reinterpret_cast<float4 *>(state_out + sbase + 32 * cb);
-#pragma unroll
-                    for (int v4 = 0; v4 < 8; ++v4)
-                        o[v4] = make_float4(__uint_as_float(r[4 * v4]), __uint_as_float(r[4 * v4 + 1]),
-                                            __uint_as_float(r[4 * v4 + 2]), __uint_as_float(r[4 * v4 + 3]));
-                }
+                for (int e = 0; e < 32; ++e)
+                    st[32 * cb + e] = decay * (st[32 * cb + e] + __uint_as_float(v[e]));
             }
+            tc_fence_before();
+            mbar_arrive(&acc_free[buf]);                     // buffer free for chunk c + 2
             if (!last) {
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&acc_ready);
+                store_bf16_row(s_prev + (((size_t)bh * nchunks + c + 1) * kD + krow) * kD + 128 * nh,
+                               st, 128);
+            } else if (state_out) {
+                float4 *o = reinterpret_cast<float4 *>(state_out + sbase);
+#pragma unroll
+                for (int v4 = 0; v4 < 32; ++v4)
+                    o[v4] = make_float4(st[4 * v4], st[4 * v4 + 1], st[4 * v4 + 2], st[4 * v4 + 3]);
             }
         }
     }
@@ -267,36 +272,54 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 128);
+        tmem_dealloc(tmem, 256);
     }
 }
 
 // ------------------------------------------------------------------ output pass
+// One CTA per (sequence, head, chunk, 128-row block), heavy blocks first.
+// TMEM (512 columns): O [0,256) f32; Qt [256,384) bf16 pairs (A operand);
+// two S/P buffers [384,448) and [448,512): S = Qt Kt^T for a 64-key tile in
+// f32; P (bf16 pairs, A operand of P V) for keys 0-31 overwrites columns
+// 0-15 and for keys 32-63 columns 32-47 of the same buffer.
+// Shared memory: a K ring (3 x 32 KB) carrying the Kt tiles with the four
+// 64-row parts of S_prev interleaved, a V ring (2 x 32 KB), and a 64 KB
+// tile buffer that holds Qt (TMA, then copied to TMEM by tcgen05.cp), then
+// the gate G, then the output rows for the TMA store.
+// Warps: 0 TMA, 1 MMA (+ TMEM allocation), 2-9 two warpgroups that split
+// the columns of every TMEM row (S/P tiles: 32 + 32; O: 128 + 128).
+// MMA order per key tile t: QK^T(t), Qt S_prev part t (t < 4), P V(t-1),
+// so the mask pass of one tile overlaps the tensor core work around it.
+constexpr int kKeyTile = 64;
+constexpr uint32_t kBox64 = 8192;                  // one 64-row x 64-col bf16 box
+constexpr int kKRing = 3, kVRing = 2;
+constexpr int kOutThreads = 320;                   // 10 warps
+constexpr int kEpiThreads = 256;
+
 struct TcOutSmem {
-    static constexpr uint32_t kQ = 0;                  // Qt  128 x 256  (4 boxes)
-    static constexpr uint32_t kK = 4 * kBox;           // Kt  128 x 256  (4 boxes)
-    static constexpr uint32_t kV = 8 * kBox;           // V   128 x 256  (4 boxes)
-    static constexpr uint32_t kS = 4 * kBox;           // S_prev 256 x 256 over K and V
-    static constexpr uint32_t kP = 12 * kBox;          // P   128 x 128  (2 boxes)
-    static constexpr uint32_t kBytes = 14 * kBox + 1024;
+    static constexpr uint32_t kStage = 4 * kBox64;     // 64 rows x 256 cols
+    static constexpr uint32_t kK = 0;
+    static constexpr uint32_t kV = kKRing * kStage;
+    static constexpr uint32_t kY = kV + kVRing * kStage;   // 128 rows x 256 cols (4 boxes)
+    static constexpr uint32_t kBytes = kY + 4 * kBox + 1024;
 };
 
 struct TcOutArgs {
-    int heads, n, chunk, nchunks, rblocks, has_state_in;
-    __nv_bfloat16 *out;
-    const __nv_bfloat16 *gate;
+    int heads, n, chunk, nchunks, rblocks, has_state_in, has_gate;
     const float *gn_weight, *gn_bias;
     float eps;
     unsigned *err;
 };
 
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(kOutThreads, 1)
 tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_s,
+                 const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_out,
                  TcOutArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    __shared__ uint64_t q_full, k_full, v_full, s_full, k_empty, v_empty, sqk_full, p_full, o_full;
+    __shared__ uint64_t kfull[kKRing], kempty[kKRing], vfull[kVRing], vempty[kVRing];
+    __shared__ uint64_t s_full[2], p_full[2], s_free[2], q_full, q_copied, o_full, g_full;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
@@ -310,14 +333,25 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int c0 = c * a.chunk;
     const int L = min(a.chunk, a.n - c0);
     if (r * kBlk >= L) return;                            // past a short last chunk
+    const int kend = min(kBlk * (r + 1), L);              // keys this row block sees
+    const int nk = (kend + kKeyTile - 1) / kKeyTile;
     const bool has_s = (c > 0) || a.has_state_in;
+    const int nsp = has_s ? 4 : 0;                        // S_prev parts in the K ring
+    const int t0row = c0 + r * kBlk;                      // first token of the block
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     unsigned *err = a.err;
+    uint8_t *ybuf = smem + TcOutSmem::kY;
 
     if (threadIdx.x == 0) {
-        mbar_init(&q_full, 1); mbar_init(&k_full, 1); mbar_init(&v_full, 1);
-        mbar_init(&s_full, 1); mbar_init(&k_empty, 1); mbar_init(&v_empty, 1);
-        mbar_init(&sqk_full, 1); mbar_init(&p_full, 128); mbar_init(&o_full, 1);
+        for (int s = 0; s < kKRing; ++s) { mbar_init(&kfull[s], 1); mbar_init(&kempty[s], 1); }
+        for (int s = 0; s < kVRing; ++s) { mbar_init(&vfull[s], 1); mbar_init(&vempty[s], 1); }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&s_full[s], 1); mbar_init(&p_full[s], kEpiThreads); mbar_init(&s_free[s], 1);
+        }
+        mbar_init(&q_full, 1);
+        mbar_init(&q_copied, 1);
+        mbar_init(&o_full, 1);
+        mbar_init(&g_full, 1);
         abort_flag = 0;
         fence_barrier_init();
     }
@@ -329,201 +363,258 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_slot;
-    const uint32_t tO = tmem;             // columns   0..255: O  (128 x 256 f32)
-    const uint32_t tS = tmem + 256;       // columns 256..383: S  (128 x 128 f32)
+    const uint32_t tO = tmem, tQ = tmem + 256;
+    auto tSP = [tmem](int t) -> uint32_t { return tmem + 384 + 64 * (t & 1); };
 
     if (warp == 0) {
         if (lane == 0) {
             tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v); tma_prefetch_desc(&tm_s);
-            const int tq = c0 + r * kBlk;
             mbar_expect_tx(&q_full, 4 * kBox);
             for (int x = 0; x < 4; ++x)
-                tma_load_3d(smem + TcOutSmem::kQ + x * kBox, &tm_q, &q_full, 64 * x, tq, bh);
-            for (int t = 0; t <= r; ++t) {
-                const int tk = c0 + t * kBlk;
-                if (t > 0 && !mbar_wait(&k_empty, (t - 1) & 1, &abort_flag, err)) break;
-                mbar_expect_tx(&k_full, 4 * kBox);
+                tma_load_3d(ybuf + x * kBox, &tm_q, &q_full, 64 * x, t0row, bh);
+            const int srow = (bh * a.nchunks + c) * kD;
+            int it = 0;
+            bool ok = true;
+            auto load_s = [&](int p) -> bool {
+                const int s = it % kKRing;
+                if (it >= kKRing && !mbar_wait(&kempty[s], ((it / kKRing) - 1) & 1, &abort_flag, err))
+                    return false;
+                uint8_t *dst = smem + TcOutSmem::kK + s * TcOutSmem::kStage;
+                mbar_expect_tx(&kfull[s], TcOutSmem::kStage);
                 for (int x = 0; x < 4; ++x)
-                    tma_load_3d(smem + TcOutSmem::kK + x * kBox, &tm_k, &k_full, 64 * x, tk, bh);
-                if (t > 0 && !mbar_wait(&v_empty, (t - 1) & 1, &abort_flag, err)) break;
-                mbar_expect_tx(&v_full, 4 * kBox);
+                    tma_load_2d(dst + x * kBox64, &tm_s, &kfull[s], 64 * x, srow + 64 * p);
+                ++it;
+                return true;
+            };
+            for (int t = 0; ok && t < nk; ++t) {
+                const int tk = c0 + t * kKeyTile;
+                const int s = it % kKRing;
+                if (it >= kKRing && !mbar_wait(&kempty[s], ((it / kKRing) - 1) & 1, &abort_flag, err)) { ok = false; break; }
+                uint8_t *kd = smem + TcOutSmem::kK + s * TcOutSmem::kStage;
+                mbar_expect_tx(&kfull[s], TcOutSmem::kStage);
                 for (int x = 0; x < 4; ++x)
-                    tma_load_4d(smem + TcOutSmem::kV + x * kBox, &tm_v, &v_full, 64 * x, h, tk, b);
+                    tma_load_3d(kd + x * kBox64, &tm_k, &kfull[s], 64 * x, tk, bh);
+                ++it;
+                if (t < nsp && !(ok = load_s(t))) break;
+                const int vs = t % kVRing;
+                if (t >= kVRing && !mbar_wait(&vempty[vs], ((t / kVRing) - 1) & 1, &abort_flag, err)) { ok = false; break; }
+                uint8_t *vd = smem + TcOutSmem::kV + vs * TcOutSmem::kStage;
+                mbar_expect_tx(&vfull[vs], TcOutSmem::kStage);
+                for (int x = 0; x < 4; ++x)
+                    tma_load_4d(vd + x * kBox64, &tm_v, &vfull[vs], 64 * x, h, tk, b);
             }
-            if (has_s && !abort_flag && mbar_wait(&k_empty, r & 1, &abort_flag, err) &&
-                mbar_wait(&v_empty, r & 1, &abort_flag, err)) {
-                mbar_expect_tx(&s_full, 8 * kBox);
-                const int srow = (bh * a.nchunks + c) * kD;
+            for (int p = nk; ok && p < nsp; ++p) ok = load_s(p);
+            // the gate tile reuses the Qt buffer once Qt sits in TMEM
+            if (ok && a.has_gate && mbar_wait(&q_copied, 0, &abort_flag, err)) {
+                tma_prefetch_desc(&tm_g);
+                mbar_expect_tx(&g_full, 4 * kBox);
                 for (int x = 0; x < 4; ++x)
-                    tma_load_2d(smem + TcOutSmem::kS + x * 2 * kBox, &tm_s, &s_full, 64 * x, srow);
+                    tma_load_4d(ybuf + x * kBox, &tm_g, &g_full, 64 * x, h, t0row, b);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t id_qk = idesc_bf16(128, 128, 0, 0);
+            const uint32_t id_qk = idesc_bf16(128, kKeyTile, 0, 0);
             const uint32_t id_pv = idesc_bf16(128, 256, 0, 1);
-            const uint32_t sQ = smem_u32(smem + TcOutSmem::kQ);
             const uint32_t sK = smem_u32(smem + TcOutSmem::kK);
             const uint32_t sV = smem_u32(smem + TcOutSmem::kV);
-            const uint32_t sP = smem_u32(smem + TcOutSmem::kP);
-            const uint32_t sS = smem_u32(smem + TcOutSmem::kS);
+            const uint32_t sY = smem_u32(ybuf);
             bool ok = mbar_wait(&q_full, 0, &abort_flag, err);
-            for (int t = 0; ok && t <= r; ++t) {
-                if (!mbar_wait(&k_full, t & 1, &abort_flag, err)) { ok = false; break; }
+            if (ok) {
                 tc_fence_after();
+                // Qt (K-major, 128-byte swizzle) -> TMEM, 16 columns of K per copy
 #pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks) {
-                    const uint32_t off = (ks / 4) * kBox + (ks % 4) * 32;
-                    mma_bf16(tS, smem_desc_sw128(sQ + off, 16, 1024),
-                             smem_desc_sw128(sK + off, 16, 1024), id_qk, ks > 0);
-                }
-                mma_commit(&sqk_full);
-                mma_commit(&k_empty);
-                if (!mbar_wait(&p_full, t & 1, &abort_flag, err)) { ok = false; break; }
-                if (!mbar_wait(&v_full, t & 1, &abort_flag, err)) { ok = false; break; }
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < kBlk / 16; ++ks) {
-                    const uint32_t offp = (ks / 4) * kBox + (ks % 4) * 32;
-                    mma_bf16(tO, smem_desc_sw128(sP + offp, 16, 1024),
-                             smem_desc_sw128(sV + ks * 2048, kBox, 1024), id_pv,
-                             (t > 0 || ks > 0) ? 1u : 0u);
-                }
-                mma_commit(&v_empty);
+                for (int ks = 0; ks < kD / 16; ++ks)
+                    tmem_cp_128x256b(tQ + 8 * ks,
+                                     smem_desc_sw128(sY + (ks / 4) * kBox + (ks % 4) * 32, 16, 1024));
+                mma_commit(&q_copied);
             }
-            if (ok && has_s) {
-                if (mbar_wait(&s_full, 0, &abort_flag, err)) {
+            bool o_written = false;
+            int it = 0;
+            auto qs_part = [&](int p) -> bool {
+                const int s = it % kKRing;
+                if (!mbar_wait(&kfull[s], (it / kKRing) & 1, &abort_flag, err)) return false;
+                tc_fence_after();
+                const uint32_t base = sK + s * TcOutSmem::kStage;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ts(tO, tQ + 8 * (4 * p + kk),
+                                smem_desc_sw128(base + kk * 2048, kBox64, 1024), id_pv,
+                                (o_written || kk > 0) ? 1u : 0u);
+                o_written = true;
+                mma_commit(&kempty[s]);
+                ++it;
+                return true;
+            };
+            for (int t = 0; ok && t <= nk; ++t) {
+                if (t < nk) {
+                    const int s = it % kKRing;
+                    if (!mbar_wait(&kfull[s], (it / kKRing) & 1, &abort_flag, err)) { ok = false; break; }
+                    if (t >= 2 && !mbar_wait(&s_free[t & 1], ((t - 2) >> 1) & 1, &abort_flag, err)) { ok = false; break; }
                     tc_fence_after();
+                    const uint32_t base = sK + s * TcOutSmem::kStage;
 #pragma unroll
-                    for (int ks = 0; ks < kD / 16; ++ks) {
-                        const uint32_t off = (ks / 4) * kBox + (ks % 4) * 32;
-                        mma_bf16(tO, smem_desc_sw128(sQ + off, 16, 1024),
-                                 smem_desc_sw128(sS + ks * 2048, 2 * kBox, 1024), id_pv, 1u);
-                    }
+                    for (int ks = 0; ks < kD / 16; ++ks)
+                        mma_bf16_ts(tSP(t), tQ + 8 * ks,
+                                    smem_desc_sw128(base + (ks / 4) * kBox64 + (ks % 4) * 32, 16, 1024),
+                                    id_qk, ks > 0 ? 1u : 0u);
+                    mma_commit(&kempty[s]);
+                    mma_commit(&s_full[t & 1]);
+                    ++it;
+                    if (t < nsp && !(ok = qs_part(t))) break;
+                }
+                if (t >= 1) {
+                    const int u = t - 1;
+                    if (!mbar_wait(&p_full[u & 1], (u >> 1) & 1, &abort_flag, err)) { ok = false; break; }
+                    if (!mbar_wait(&vfull[u % kVRing], (u / kVRing) & 1, &abort_flag, err)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t base = sV + (u % kVRing) * TcOutSmem::kStage;
+#pragma unroll
+                    for (int kk = 0; kk < kKeyTile / 16; ++kk)   // P halves at columns 0 and 32
+                        mma_bf16_ts(tO, tSP(u) + 8 * kk + (kk >= 2 ? 16 : 0),
+                                    smem_desc_sw128(base + kk * 2048, kBox64, 1024), id_pv,
+                                    (o_written || kk > 0) ? 1u : 0u);
+                    o_written = true;
+                    mma_commit(&vempty[u % kVRing]);
+                    mma_commit(&s_free[u & 1]);
                 }
             }
+            for (int p = nk; ok && p < nsp; ++p) ok = qs_part(p);
             mma_commit(&o_full);
         }
     } else {
+        // two warpgroups: wg 0 owns S columns [0,32) and O columns [0,128),
+        // wg 1 owns S columns [32,64) and O columns [128,256)
+        const int wg = (warp - 2) / 4;
         const int q4 = warp % 4;
         const int row = 32 * q4 + lane;                         // row of the 128-row block
         const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
-        uint8_t *prow = smem + TcOutSmem::kP + row * 128;
+        const int lrow = r * kBlk + row;                        // row within the chunk
+        const int t_row = t0row + row;
         bool ok = true;
-        for (int t = 0; t <= r; ++t) {
-            if (!warp_wait(&sqk_full, t & 1, &abort_flag, err)) { ok = false; break; }
-            if (t > 0 && !warp_wait(&v_empty, (t - 1) & 1, &abort_flag, err)) { ok = false; break; }
+        for (int t = 0; t < nk; ++t) {
+            if (!warp_wait(&s_full[t & 1], (t >> 1) & 1, &abort_flag, err)) { ok = false; break; }
             tc_fence_after();
-            const bool diag = (t == r);
-#pragma unroll 1
-            for (int cb = 0; cb < 4; ++cb) {
-                uint32_t v[32];
-                tmem_ld32(tS + lane_off + 32 * cb, v);
-                tmem_wait_ld();
+            uint32_t v[32];
+            tmem_ld32(tSP(t) + lane_off + 32 * wg, v);
+            tmem_wait_ld();
+            const int j0 = t * kKeyTile + 32 * wg;              // first key of this half tile
+            uint32_t w[16];
+            if (j0 + 31 <= lrow) {                              // every key at or before the row
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {          // 16-byte chunks of 8 columns
-                    uint32_t w[4];
+                for (int e = 0; e < 16; ++e)
+                    w[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+            } else {
 #pragma unroll
-                    for (int e2 = 0; e2 < 4; ++e2) {
-                        const int j0 = 32 * cb + 8 * ch + 2 * e2;
-                        float lo = __uint_as_float(v[8 * ch + 2 * e2]);
-                        float hi = __uint_as_float(v[8 * ch + 2 * e2 + 1]);
-                        if (diag) {
-                            lo = (row >= j0) ? lo : 0.f;
-                            hi = (row >= j0 + 1) ? hi : 0.f;
-                        }
-                        w[e2] = pack_bf16x2(lo, hi);
-                    }
-                    const int col = 32 * cb + 8 * ch;             // first column of the chunk
-                    const int box = col / 64;
-                    const int c16 = (col % 64) / 8;
-                    uint4 *dst = reinterpret_cast<uint4 *>(prow + box * kBox +
-                                                           ((c16 ^ (row & 7)) * 16));
-                    *dst = make_uint4(w[0], w[1], w[2], w[3]);
+                for (int e = 0; e < 16; ++e) {
+                    const float x0 = (lrow >= j0 + 2 * e) ? __uint_as_float(v[2 * e]) : 0.f;
+                    const float x1 = (lrow >= j0 + 2 * e + 1) ? __uint_as_float(v[2 * e + 1]) : 0.f;
+                    w[e] = pack_bf16x2(x0, x1);
                 }
             }
-            fence_async_shared();
+            // P (bf16 pairs) goes to the first 16 columns of this warpgroup's own
+            // 32 S columns, so it never overwrites S the other warpgroup still reads.
+            tmem_st16(tSP(t) + lane_off + 32 * wg, w);
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&p_full);
+            mbar_arrive(&p_full[t & 1]);
         }
-        if (ok && warp_wait(&o_full, 0, &abort_flag, err)) {
-            tc_fence_after();
-            // Every lane runs the TMEM loads (they are warp-collective); only
-            // rows inside the sequence store.
-            const int t = c0 + r * kBlk + row;
-            const bool valid = t < a.n;
-            __nv_bfloat16 *orow = a.out + (((size_t)b * a.n + (valid ? t : 0)) * a.heads + h) * kD;
-            if (!a.gate) {
+        const bool go = ok && warp_wait(&o_full, 0, &abort_flag, err) &&
+                        (!a.has_gate || warp_wait(&g_full, 0, &abort_flag, err));
+        // The K ring is idle once O is complete: its first bytes hold the
+        // two warpgroups' partial row sums.
+        float (*red)[kBlk] = reinterpret_cast<float (*)[kBlk]>(smem + TcOutSmem::kK);
+        float mean = 0.f, rstd = 1.f;
+        if (go) tc_fence_after();
+        if (a.has_gate) {
+            // GroupNorm statistics over the row's 256 channels; each
+            // warpgroup sums its half and the halves meet in shared memory.
+            float sum = 0.f;
+            if (go) {
 #pragma unroll 1
-                for (int cb = 0; cb < 8; ++cb) {
+                for (int cb = 0; cb < 4; ++cb) {
                     uint32_t v[32];
-                    tmem_ld32(tO + lane_off + 32 * cb, v);
-                    tmem_wait_ld();
-                    if (valid) {
-                        uint4 *o = reinterpret_cast<uint4 *>(orow + 32 * cb);
-#pragma unroll
-                        for (int q8 = 0; q8 < 4; ++q8)
-                            o[q8] = make_uint4(
-                                pack_bf16x2(__uint_as_float(v[8 * q8]), __uint_as_float(v[8 * q8 + 1])),
-                                pack_bf16x2(__uint_as_float(v[8 * q8 + 2]), __uint_as_float(v[8 * q8 + 3])),
-                                pack_bf16x2(__uint_as_float(v[8 * q8 + 4]), __uint_as_float(v[8 * q8 + 5])),
-                                pack_bf16x2(__uint_as_float(v[8 * q8 + 6]), __uint_as_float(v[8 * q8 + 7])));
-                    }
-                }
-            } else {
-                // GroupNorm over this row's 256 channels, then the swish gate
-                float sum = 0.f;
-#pragma unroll 1
-                for (int cb = 0; cb < 8; ++cb) {
-                    uint32_t v[32];
-                    tmem_ld32(tO + lane_off + 32 * cb, v);
+                    tmem_ld32(tO + lane_off + 128 * wg + 32 * cb, v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) sum += __uint_as_float(v[e]);
                 }
-                const float mean = sum * (1.f / kD);
-                float sq = 0.f;
+            }
+            red[wg][row] = sum;
+            named_barrier(1, kEpiThreads);
+            mean = (red[0][row] + red[1][row]) * (1.f / kD);
+            named_barrier(1, kEpiThreads);
+            float sq = 0.f;
+            if (go) {
 #pragma unroll 1
-                for (int cb = 0; cb < 8; ++cb) {
+                for (int cb = 0; cb < 4; ++cb) {
                     uint32_t v[32];
-                    tmem_ld32(tO + lane_off + 32 * cb, v);
+                    tmem_ld32(tO + lane_off + 128 * wg + 32 * cb, v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
-                        float d = __uint_as_float(v[e]) - mean;
+                        const float d = __uint_as_float(v[e]) - mean;
                         sq = fmaf(d, d, sq);
                     }
                 }
-                const float rstd = rsqrtf(sq * (1.f / kD) + a.eps);
-                const __nv_bfloat16 *grow =
-                    a.gate + (((size_t)b * a.n + (valid ? t : 0)) * a.heads + h) * kD;
-                const float *wv = a.gn_weight ? a.gn_weight + h * kD : nullptr;
-                const float *bv = a.gn_bias ? a.gn_bias + h * kD : nullptr;
+            }
+            red[wg][row] = sq;
+            named_barrier(1, kEpiThreads);
+            rstd = rsqrtf((red[0][row] + red[1][row]) * (1.f / kD) + a.eps);
+        }
+        if (go) {
+            // This row's slot in the 128-byte-swizzled output/gate tile.
+            uint8_t *yrow = ybuf + row * 128;
+            const int sw = row & 7;
+            const float *wv = a.gn_weight ? a.gn_weight + h * kD : nullptr;
+            const float *bv = a.gn_bias ? a.gn_bias + h * kD : nullptr;
 #pragma unroll 1
-                for (int cb = 0; cb < 8; ++cb) {
-                    uint32_t v[32];
-                    tmem_ld32(tO + lane_off + 32 * cb, v);
-                    tmem_wait_ld();
-                    if (valid) {
+            for (int k4 = 0; k4 < 4; ++k4) {
+                const int cb = 4 * wg + k4;                       // 32-column block
+                uint32_t v[32];
+                tmem_ld32(tO + lane_off + 32 * cb, v);
+                tmem_wait_ld();
+                uint8_t *box = yrow + (cb >> 1) * kBox;
 #pragma unroll
-                        for (int q8 = 0; q8 < 4; ++q8) {
-                            float gv[8], y[8];
-                            load8(grow + 32 * cb + 8 * q8, gv);
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    uint4 *slot = reinterpret_cast<uint4 *>(box + ((((cb & 1) * 4 + q8) ^ sw) * 16));
+                    float y[8];
+                    if (a.has_gate) {
+                        uint4 graw = *slot;
+                        const __nv_bfloat162 *g2 = reinterpret_cast<const __nv_bfloat162 *>(&graw);
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) {
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            const float2 gg = __bfloat1622float2(g2[e2]);
+#pragma unroll
+                            for (int hh = 0; hh < 2; ++hh) {
+                                const int e = 2 * e2 + hh;
                                 const int ch = 32 * cb + 8 * q8 + e;
                                 float yh = (__uint_as_float(v[8 * q8 + e]) - mean) * rstd;
                                 if (wv) yh *= wv[ch];
                                 if (bv) yh += bv[ch];
-                                y[e] = gv[e] / (1.f + __expf(-gv[e])) * yh;
+                                const float g = hh ? gg.y : gg.x;
+                                y[e] = __fdividef(g, 1.f + __expf(-g)) * yh;
                             }
-                            store8(orow + 32 * cb + 8 * q8, y);
                         }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) y[e] = __uint_as_float(v[8 * q8 + e]);
                     }
+                    *slot = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
+                                       pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
                 }
             }
+            fence_async_shared();
         }
+        // Both epilogue warpgroups reach this barrier on every path.
+        named_barrier(1, kEpiThreads);
+        if (wg == 0 && row == 0 && !abort_flag) {
+            for (int x = 0; x < 4; ++x) tma_store_4d(&tm_out, ybuf + x * kBox, 64 * x, h, t0row, b);
+            tma_store_commit();
+            tma_store_wait_read();
+        }
+        (void)t_row;
     }
     tc_fence_before();
     __syncthreads();
@@ -576,7 +667,7 @@ static TcLayout tc_layout(int batch, int heads, int n, int chunk) {
     const size_t bh = (size_t)batch * heads;
     const size_t nchunks = ((size_t)n + chunk - 1) / chunk;
     l.table = 0;
-    l.qt = align1k((size_t)n * (kD / 2) * sizeof(float2));
+    l.qt = 0;
     l.kt = l.qt + align1k(bh * n * kD * 2);
     l.sprev = l.kt + align1k(bh * n * kD * 2);
     l.total = l.sprev + align1k(bh * nchunks * kD * kD * 2);
@@ -619,7 +710,6 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
     const int last_len = n - (nchunks - 1) * C;
     const TcLayout lay = tc_layout(B, H, n, C);
     char *ws = (char *)a.workspace;
-    float2 *table = (float2 *)(ws + lay.table);
     __nv_bfloat16 *qt = (__nv_bfloat16 *)(ws + lay.qt);
     __nv_bfloat16 *kt = (__nv_bfloat16 *)(ws + lay.kt);
     __nv_bfloat16 *sp = (__nv_bfloat16 *)(ws + lay.sprev);
@@ -635,40 +725,53 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
         hp.decay_last[h] = (float)std::pow(g, (double)last_len);
     }
 
-    // tensor maps
-    CUtensorMap tm_q, tm_k, tm_v, tm_s;
+    // tensor maps: 128-row boxes for the state pass, 64-row boxes for the output pass
+    CUtensorMap tm_q128, tm_k128, tm_v128, tm_k64, tm_v64, tm_s64;
     {
         cuuint64_t dims[3] = {kD, (cuuint64_t)n, (cuuint64_t)BH};
         cuuint64_t str[2] = {kD * 2, (cuuint64_t)n * kD * 2};
-        cuuint32_t box[3] = {64, kBlk, 1};
-        if (!make_map(&tm_q, qt, 3, dims, str, box) || !make_map(&tm_k, kt, 3, dims, str, box))
+        cuuint32_t box128[3] = {64, kBlk, 1};
+        cuuint32_t box64[3] = {64, kKeyTile, 1};
+        if (!make_map(&tm_k128, kt, 3, dims, str, box128) ||
+            !make_map(&tm_k64, kt, 3, dims, str, box64) ||
+            !make_map(&tm_q128, qt, 3, dims, str, box128))
             return cudaErrorInvalidValue;
     }
     {
         cuuint64_t dims[4] = {kD, (cuuint64_t)H, (cuuint64_t)n, (cuuint64_t)B};
         cuuint64_t str[3] = {kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)n * H * kD * 2};
-        cuuint32_t box[4] = {64, 1, kBlk, 1};
-        if (!make_map(&tm_v, a.v, 4, dims, str, box)) return cudaErrorInvalidValue;
+        cuuint32_t box128[4] = {64, 1, kBlk, 1};
+        cuuint32_t box64[4] = {64, 1, kKeyTile, 1};
+        if (!make_map(&tm_v128, a.v, 4, dims, str, box128) ||
+            !make_map(&tm_v64, a.v, 4, dims, str, box64))
+            return cudaErrorInvalidValue;
     }
     {
         cuuint64_t dims[2] = {kD, (cuuint64_t)BH * nchunks * kD};
         cuuint64_t str[1] = {kD * 2};
-        cuuint32_t box[2] = {64, 256};
-        if (!make_map(&tm_s, sp, 2, dims, str, box)) return cudaErrorInvalidValue;
+        cuuint32_t box[2] = {64, 64};
+        if (!make_map(&tm_s64, sp, 2, dims, str, box)) return cudaErrorInvalidValue;
+    }
+    // output and gate tiles: 128 tokens x 64 channels of one head
+    CUtensorMap tm_out, tm_g;
+    {
+        cuuint64_t dims[4] = {kD, (cuuint64_t)H, (cuuint64_t)n, (cuuint64_t)B};
+        cuuint64_t str[3] = {kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)n * H * kD * 2};
+        cuuint32_t box[4] = {64, 1, kBlk, 1};
+        if (!make_map(&tm_out, a.out, 4, dims, str, box)) return cudaErrorInvalidValue;
+        if (!make_map(&tm_g, a.gate ? a.gate->g : a.out, 4, dims, str, box))
+            return cudaErrorInvalidValue;
     }
 
     cudaError_t e;
-    if (a.rotate) {
-        e = launch_rotation_table(table, n, kD, a.pos0, stream);
-        if (e != cudaSuccess) return e;
-    }
     {
-        const long long total = (long long)B * n * H * (kD / 8);
-        const unsigned blocks = (unsigned)((total + 255) / 256);
+        TcPrepParams pp;
+        for (int j = 0; j < kD / 2; ++j) pp.theta[j] = std::pow(10000.0, -2.0 * j / kD);
+        for (int h = 0; h < kMaxHeads; ++h) pp.log2g[h] = hp.log2g[h];
         KernelTimer timer("tc_prep", stream);
-        tc_prep_kernel<<<blocks, 256, 0, stream>>>((const __nv_bfloat16 *)a.q,
-                                                   (const __nv_bfloat16 *)a.k, table, hp, qt, kt,
-                                                   B, H, n, C, a.rotate);
+        tc_prep_kernel<<<n, 256, 0, stream>>>((const __nv_bfloat16 *)a.q,
+                                             (const __nv_bfloat16 *)a.k, pp, qt, kt, B, H, n, C,
+                                             a.pos0, a.rotate);
         count_launch();
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
@@ -677,7 +780,7 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
         e = cudaFuncSetAttribute(tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         KernelTimer timer("tc_state", stream);
-        tc_state_kernel<<<BH * 4, kTcThreads, smem, stream>>>(tm_k, tm_v, hp, a.state_in,
+        tc_state_kernel<<<BH * 4, kTcThreads, smem, stream>>>(tm_k128, tm_v128, hp, a.state_in,
                                                              a.state_out, sp, H, n, C, nchunks,
                                                              err);
         count_launch();
@@ -687,8 +790,7 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
         TcOutArgs oa;
         oa.heads = H; oa.n = n; oa.chunk = C; oa.nchunks = nchunks; oa.rblocks = C / kBlk;
         oa.has_state_in = a.state_in != nullptr;
-        oa.out = (__nv_bfloat16 *)a.out;
-        oa.gate = a.gate ? (const __nv_bfloat16 *)a.gate->g : nullptr;
+        oa.has_gate = a.gate != nullptr;
         oa.gn_weight = a.gate ? a.gate->weight : nullptr;
         oa.gn_bias = a.gate ? a.gate->bias : nullptr;
         oa.eps = a.gate ? a.gate->eps : 0.f;
@@ -699,7 +801,8 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
         if (e != cudaSuccess) return e;
         const unsigned grid = (unsigned)(BH * nchunks * oa.rblocks);
         KernelTimer timer("tc_output", stream);
-        tc_output_kernel<<<grid, kTcThreads, smem, stream>>>(tm_q, tm_k, tm_v, tm_s, oa);
+        tc_output_kernel<<<grid, kOutThreads, smem, stream>>>(tm_q128, tm_k64, tm_v64, tm_s64, tm_g,
+                                                             tm_out, oa);
         count_launch();
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
