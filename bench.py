@@ -331,28 +331,67 @@ def run_ours(args, w, chunk):
     value = world * tokens_per_step * args.steps / (ms / 1e3)
 
     # ---- end to end through the public API with host buffers
+    # Every step copies its inputs from pinned host memory, runs the hot path
+    # and copies y and the decode output back.  Copies run on their own
+    # streams, double-buffered, so step i's upload overlaps step i-1's
+    # compute and download (PCIe is full duplex).
     h2d = sum(x.numel() * x.element_size() for x in host if x is not None)
     d2h = y.numel() * y.element_size() + o.numel() * o.element_size()
-    y_host = torch.empty_like(y, device="cpu").pin_memory()
-    o_host = torch.empty_like(o, device="cpu").pin_memory()
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    dsets = [[None if x is None else torch.empty_like(x, device=dev) for x in host]
+             for _ in range(2)]
+    ys = [torch.empty_like(y) for _ in range(2)]
+    os_ = [torch.empty_like(o) for _ in range(2)]
+    yh = [torch.empty_like(y, device="cpu").pin_memory() for _ in range(2)]
+    oh = [torch.empty_like(o, device="cpu").pin_memory() for _ in range(2)]
+    st2 = [torch.empty_like(state) for _ in range(2)]
+    ws2 = [torch.empty_like(ws) for _ in range(2)]
 
-    def e2e_step():
-        s = [None if x is None else x.to(dev, non_blocking=True) for x in host]
-        step(s)
-        y_host.copy_(y, non_blocking=True)
-        o_host.copy_(o, non_blocking=True)
+    def run_e2e(nsteps):
+        in_ready = [torch.cuda.Event() for _ in range(nsteps)]
+        done = [torch.cuda.Event() for _ in range(nsteps)]
+        out_done = [torch.cuda.Event() for _ in range(nsteps)]
+        for i in range(nsteps):
+            j = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(done[i - 2])
+                for dst, src in zip(dsets[j], host):
+                    if src is not None:
+                        dst.copy_(src, non_blocking=True)
+                in_ready[i].record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(in_ready[i])
+                if i >= 2:
+                    s_cmp.wait_event(out_done[i - 2])
+                qq, kk, vv, gg, q1, k1, v1 = dsets[j]
+                rn.retnet_retention_chunkwise(qq, kk, vv, gam, chunk, state_out=st2[j], gate=gg,
+                                              out=ys[j], workspace=ws2[j], algo=args.algo)
+                rn.retnet_retention_step(q1, k1, v1, gam, st2[j], n, out=os_[j])
+                done[i].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done[i])
+                yh[j].copy_(ys[j], non_blocking=True)
+                oh[j].copy_(os_[j], non_blocking=True)
+                out_done[i].record(s_out)
+        return out_done[-1]
 
-    e2e_step()
+    run_e2e(2)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ev0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    ev1.record(stream)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    s_cmp.wait_stream(s_in)
+    s_out.wait_stream(s_in)
+    last = run_e2e(e2e_steps)
+    s_in.wait_event(last)
+    s_in.wait_stream(s_cmp)
+    e1.record(s_in)
     torch.cuda.synchronize()
-    e2e_ms = ev0.elapsed_time(ev1)
+    e2e_ms = e0.elapsed_time(e1)
     if world > 1:
         t = torch.tensor([e2e_ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)

@@ -27,6 +27,7 @@
 // issues tcgen05.mma, warps 2-5 move data between TMEM, registers and
 // memory.  Every mbarrier wait is bounded (about 2 s); on timeout the CTA
 // records kDevErrTimeout and unwinds.
+#include <algorithm>
 #include <cmath>
 
 #include "kernels.h"
@@ -79,30 +80,51 @@ tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
     __syncthreads();
     const int i = t % chunk;                        // index inside the chunk
     const int tasks = batch * heads * (kD / 8);
-    for (int task = threadIdx.x; task < tasks; task += blockDim.x) {
-        const int part = task % (kD / 8);
-        const int bhi = task / (kD / 8);
-        const int h = bhi % heads, b = bhi / heads;
-        const float e = (float)(i + 1) * pp.log2g[h];
-        const float sq = exp2f(e), sk = exp2f(-e);
-        const size_t src = (((size_t)b * n + t) * heads + h) * kD + part * 8;
-        float xq[8], xk[8], oq[8], ok[8];
-        load8(q + src, xq);
-        load8(k + src, xk);
+    // Up to kPrepBatch tasks per thread with every load issued before any
+    // arithmetic, so each thread keeps 2 * kPrepBatch 16-byte loads in flight.
+    constexpr int kPrepBatch = 4;
+    for (int base = threadIdx.x; base < tasks; base += kPrepBatch * blockDim.x) {
+        uint4 rq[kPrepBatch], rk[kPrepBatch];
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            const float2 r = cs[part * 4 + p];
-            const float cq = r.x * sq, sq2 = r.y * sq, ck = r.x * sk, sk2 = r.y * sk;
-            float a = xq[2 * p], bb = xq[2 * p + 1];
-            oq[2 * p] = a * cq - bb * sq2;
-            oq[2 * p + 1] = a * sq2 + bb * cq;
-            a = xk[2 * p]; bb = xk[2 * p + 1];
-            ok[2 * p] = a * ck - bb * sk2;
-            ok[2 * p + 1] = a * sk2 + bb * ck;
+        for (int u = 0; u < kPrepBatch; ++u) {
+            const int task = base + u * blockDim.x;
+            if (task < tasks) {
+                const int part = task % (kD / 8);
+                const int bhi = task / (kD / 8);
+                const int h = bhi % heads, b = bhi / heads;
+                const size_t src = (((size_t)b * n + t) * heads + h) * kD + part * 8;
+                rq[u] = *reinterpret_cast<const uint4 *>(q + src);
+                rk[u] = *reinterpret_cast<const uint4 *>(k + src);
+            }
         }
-        const size_t dst = (((size_t)b * heads + h) * n + t) * kD + part * 8;
-        store8(qt + dst, oq);
-        store8(kt + dst, ok);
+#pragma unroll
+        for (int u = 0; u < kPrepBatch; ++u) {
+            const int task = base + u * blockDim.x;
+            if (task < tasks) {
+            const int part = task % (kD / 8);
+            const int bhi = task / (kD / 8);
+            const int h = bhi % heads, b = bhi / heads;
+            const float e = (float)(i + 1) * pp.log2g[h];
+            const float sq = exp2f(e), sk = exp2f(-e);
+            const __nv_bfloat162 *hq = reinterpret_cast<const __nv_bfloat162 *>(&rq[u]);
+            const __nv_bfloat162 *hk = reinterpret_cast<const __nv_bfloat162 *>(&rk[u]);
+            float oq[8], ok[8];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                const float2 r = cs[part * 4 + p];
+                const float cq = r.x * sq, sq2 = r.y * sq, ck = r.x * sk, sk2 = r.y * sk;
+                const float2 xq = __bfloat1622float2(hq[p]);
+                const float2 xk = __bfloat1622float2(hk[p]);
+                oq[2 * p] = xq.x * cq - xq.y * sq2;
+                oq[2 * p + 1] = xq.x * sq2 + xq.y * cq;
+                ok[2 * p] = xk.x * ck - xk.y * sk2;
+                ok[2 * p + 1] = xk.x * sk2 + xk.y * ck;
+            }
+            const size_t dst = (((size_t)b * heads + h) * n + t) * kD + part * 8;
+            store8(qt + dst, oq);
+            store8(kt + dst, ok);
+            }
+        }
     }
 }
 
@@ -277,39 +299,69 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 }
 
 // ------------------------------------------------------------------ output pass
-// One CTA per (sequence, head, chunk, 128-row block), heavy blocks first.
-// TMEM (512 columns): O [0,256) f32; Qt [256,384) bf16 pairs (A operand);
-// two S/P buffers [384,448) and [448,512): S = Qt Kt^T for a 64-key tile in
-// f32; P (bf16 pairs, A operand of P V) for keys 0-31 overwrites columns
-// 0-15 and for keys 32-63 columns 32-47 of the same buffer.
-// Shared memory: a K ring (3 x 32 KB) carrying the Kt tiles with the four
-// 64-row parts of S_prev interleaved, a V ring (2 x 32 KB), and a 64 KB
-// tile buffer that holds Qt (TMA, then copied to TMEM by tcgen05.cp), then
-// the gate G, then the output rows for the TMA store.
-// Warps: 0 TMA, 1 MMA (+ TMEM allocation), 2-9 two warpgroups that split
-// the columns of every TMEM row (S/P tiles: 32 + 32; O: 128 + 128).
-// MMA order per key tile t: QK^T(t), Qt S_prev part t (t < 4), P V(t-1),
-// so the mask pass of one tile overlaps the tensor core work around it.
-constexpr int kKeyTile = 64;
-constexpr uint32_t kBox64 = 8192;                  // one 64-row x 64-col bf16 box
-constexpr int kKRing = 3, kVRing = 2;
+// Persistent: one CTA per SM walks work items (sequence, head, chunk,
+// 128-row block), heavy row blocks first, so the loads and the first
+// QK^T of the next item overlap the epilogue of the current one.
+// TMEM (512 columns, allocated once): O [0,256) f32; Qt [256,384) bf16 pairs
+// (A operand); S [384,512): S = Qt Kt^T for a 128-key tile in f32 (N = 128
+// keeps tcgen05.mma at its full rate).  The mask pass reads S, releases the
+// buffer at once (so QK^T of the next tile overlaps the rest of the pass and
+// P V) and writes P (bf16) to a 32 KB shared-memory tile, the A operand of P V.
+//
+// Shared memory: a ring of three 64 KB slots carrying every tile in the
+// order it is consumed; per item
+//     Qt, Kt(0), then for t = 0..nk-1: Kt(t+1), S_prev half t (t < 2), V(t),
+//     the remaining S_prev half, and the gate/output tile.
+// Qt is moved into TMEM by tcgen05.cp; the gate/output tile receives G by
+// TMA (or is merely reserved), is overwritten in place by the output rows,
+// leaves by TMA store and is released by the storing thread.
+// Warps: 0 TMA, 1 MMA (+ TMEM allocation), 2-9 two warpgroups: for each
+// tile wg w masks and converts S columns [64w, 64w+64); in the epilogue wg w
+// owns O columns [128w, 128w+128).
+// MMA order per item: copy Qt, QK^T(0), then for each tile t: QK^T(t+1),
+// Qt S_prev half t (t < 2), P V(t).
+constexpr int kKeyTile = 128;
+constexpr int kSlots = 3;
+constexpr uint32_t kSlot = 4 * kBox;               // 64 KB: 128 rows x 256 cols
 constexpr int kOutThreads = 320;                   // 10 warps
 constexpr int kEpiThreads = 256;
 
 struct TcOutSmem {
-    static constexpr uint32_t kStage = 4 * kBox64;     // 64 rows x 256 cols
-    static constexpr uint32_t kK = 0;
-    static constexpr uint32_t kV = kKRing * kStage;
-    static constexpr uint32_t kY = kV + kVRing * kStage;   // 128 rows x 256 cols (4 boxes)
-    static constexpr uint32_t kBytes = kY + 4 * kBox + 1024;
+    static constexpr uint32_t kP = kSlots * kSlot;     // P tile; the epilogue's row sums
+    static constexpr uint32_t kBytes = kP + 2 * kBox + 1024;
 };
 
 struct TcOutArgs {
-    int heads, n, chunk, nchunks, rblocks, has_state_in, has_gate;
+    int heads, n, chunk, nchunks, rblocks, has_state_in, has_gate, items;
     const float *gn_weight, *gn_bias;
     float eps;
     unsigned *err;
 };
+
+struct TcItem {
+    int r, c, bh, b, h, c0, nk, nsp, t0row;
+    bool valid;
+};
+
+// Work item w, heavy row blocks first: w -> (r from the last block down, bh, c).
+__device__ __forceinline__ TcItem tc_item(const TcOutArgs &a, int w) {
+    TcItem it;
+    const int per_r = a.items / a.rblocks;
+    it.r = a.rblocks - 1 - w / per_r;
+    const int rest = w % per_r;
+    it.c = rest % a.nchunks;
+    it.bh = rest / a.nchunks;
+    it.b = it.bh / a.heads;
+    it.h = it.bh % a.heads;
+    it.c0 = it.c * a.chunk;
+    const int L = min(a.chunk, a.n - it.c0);
+    it.valid = it.r * kBlk < L;                        // false past a short last chunk
+    const int kend = min(kBlk * (it.r + 1), L);        // keys this row block sees
+    it.nk = (kend + kKeyTile - 1) / kKeyTile;
+    it.nsp = (it.c > 0 || a.has_state_in) ? 2 : 0;     // S_prev halves (128 d_k rows each)
+    it.t0row = it.c0 + it.r * kBlk;
+    return it;
+}
 
 __global__ void __launch_bounds__(kOutThreads, 1)
 tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -318,40 +370,24 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                  TcOutArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    __shared__ uint64_t kfull[kKRing], kempty[kKRing], vfull[kVRing], vempty[kVRing];
-    __shared__ uint64_t s_full[2], p_full[2], s_free[2], q_full, q_copied, o_full, g_full;
+    __shared__ uint64_t rfull[kSlots], rempty[kSlots];
+    __shared__ uint64_t s_full, s_read, p_full, p_free, o_full, o_free;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
-    // heavy row blocks first: blockIdx.x -> (r from the last block down, bh, c)
-    const int per_r = gridDim.x / a.rblocks;
-    const int r = a.rblocks - 1 - (int)(blockIdx.x / per_r);
-    const int rest = blockIdx.x % per_r;
-    const int c = rest % a.nchunks;
-    const int bh = rest / a.nchunks;
-    const int b = bh / a.heads, h = bh % a.heads;
-    const int c0 = c * a.chunk;
-    const int L = min(a.chunk, a.n - c0);
-    if (r * kBlk >= L) return;                            // past a short last chunk
-    const int kend = min(kBlk * (r + 1), L);              // keys this row block sees
-    const int nk = (kend + kKeyTile - 1) / kKeyTile;
-    const bool has_s = (c > 0) || a.has_state_in;
-    const int nsp = has_s ? 4 : 0;                        // S_prev parts in the K ring
-    const int t0row = c0 + r * kBlk;                      // first token of the block
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     unsigned *err = a.err;
-    uint8_t *ybuf = smem + TcOutSmem::kY;
+    auto slot_ptr = [smem](int it) -> uint8_t * { return smem + (it % kSlots) * kSlot; };
+    uint8_t *pbuf = smem + TcOutSmem::kP;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kKRing; ++s) { mbar_init(&kfull[s], 1); mbar_init(&kempty[s], 1); }
-        for (int s = 0; s < kVRing; ++s) { mbar_init(&vfull[s], 1); mbar_init(&vempty[s], 1); }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&s_full[s], 1); mbar_init(&p_full[s], kEpiThreads); mbar_init(&s_free[s], 1);
-        }
-        mbar_init(&q_full, 1);
-        mbar_init(&q_copied, 1);
+        for (int s = 0; s < kSlots; ++s) { mbar_init(&rfull[s], 1); mbar_init(&rempty[s], 1); }
+        mbar_init(&s_full, 1);
+        mbar_init(&s_read, kEpiThreads);
+        mbar_init(&p_full, kEpiThreads);
+        mbar_init(&p_free, 1);
         mbar_init(&o_full, 1);
-        mbar_init(&g_full, 1);
+        mbar_init(&o_free, kEpiThreads);
         abort_flag = 0;
         fence_barrier_init();
     }
@@ -363,258 +399,311 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_slot;
-    const uint32_t tO = tmem, tQ = tmem + 256;
-    auto tSP = [tmem](int t) -> uint32_t { return tmem + 384 + 64 * (t & 1); };
+    const uint32_t tO = tmem, tQ = tmem + 256, tS = tmem + 384;
 
     if (warp == 0) {
         if (lane == 0) {
             tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v); tma_prefetch_desc(&tm_s);
-            mbar_expect_tx(&q_full, 4 * kBox);
-            for (int x = 0; x < 4; ++x)
-                tma_load_3d(ybuf + x * kBox, &tm_q, &q_full, 64 * x, t0row, bh);
-            const int srow = (bh * a.nchunks + c) * kD;
+            if (a.has_gate) tma_prefetch_desc(&tm_g);
             int it = 0;
             bool ok = true;
-            auto load_s = [&](int p) -> bool {
-                const int s = it % kKRing;
-                if (it >= kKRing && !mbar_wait(&kempty[s], ((it / kKRing) - 1) & 1, &abort_flag, err))
-                    return false;
-                uint8_t *dst = smem + TcOutSmem::kK + s * TcOutSmem::kStage;
-                mbar_expect_tx(&kfull[s], TcOutSmem::kStage);
-                for (int x = 0; x < 4; ++x)
-                    tma_load_2d(dst + x * kBox64, &tm_s, &kfull[s], 64 * x, srow + 64 * p);
-                ++it;
-                return true;
+            auto acquire = [&]() -> bool {
+                if (it < kSlots) return true;
+                return mbar_wait(&rempty[it % kSlots], ((it / kSlots) - 1) & 1, &abort_flag, err);
             };
-            for (int t = 0; ok && t < nk; ++t) {
-                const int tk = c0 + t * kKeyTile;
-                const int s = it % kKRing;
-                if (it >= kKRing && !mbar_wait(&kempty[s], ((it / kKRing) - 1) & 1, &abort_flag, err)) { ok = false; break; }
-                uint8_t *kd = smem + TcOutSmem::kK + s * TcOutSmem::kStage;
-                mbar_expect_tx(&kfull[s], TcOutSmem::kStage);
-                for (int x = 0; x < 4; ++x)
-                    tma_load_3d(kd + x * kBox64, &tm_k, &kfull[s], 64 * x, tk, bh);
+            auto issue = [&](const CUtensorMap *map, int rank, int c1, int c2, int c3) {
+                uint8_t *d = slot_ptr(it);
+                uint64_t *bar = &rfull[it % kSlots];
+                mbar_expect_tx(bar, kSlot);
+                for (int x = 0; x < 4; ++x) {
+                    if (rank == 2) tma_load_2d(d + x * kBox, map, bar, 64 * x, c1);
+                    else if (rank == 3) tma_load_3d(d + x * kBox, map, bar, 64 * x, c1, c2);
+                    else tma_load_4d(d + x * kBox, map, bar, 64 * x, c1, c2, c3);
+                }
                 ++it;
-                if (t < nsp && !(ok = load_s(t))) break;
-                const int vs = t % kVRing;
-                if (t >= kVRing && !mbar_wait(&vempty[vs], ((t / kVRing) - 1) & 1, &abort_flag, err)) { ok = false; break; }
-                uint8_t *vd = smem + TcOutSmem::kV + vs * TcOutSmem::kStage;
-                mbar_expect_tx(&vfull[vs], TcOutSmem::kStage);
-                for (int x = 0; x < 4; ++x)
-                    tma_load_4d(vd + x * kBox64, &tm_v, &vfull[vs], 64 * x, h, tk, b);
-            }
-            for (int p = nk; ok && p < nsp; ++p) ok = load_s(p);
-            // the gate tile reuses the Qt buffer once Qt sits in TMEM
-            if (ok && a.has_gate && mbar_wait(&q_copied, 0, &abort_flag, err)) {
-                tma_prefetch_desc(&tm_g);
-                mbar_expect_tx(&g_full, 4 * kBox);
-                for (int x = 0; x < 4; ++x)
-                    tma_load_4d(ybuf + x * kBox, &tm_g, &g_full, 64 * x, h, t0row, b);
+            };
+            for (int w = blockIdx.x; ok && w < a.items; w += gridDim.x) {
+                const TcItem m = tc_item(a, w);
+                if (!m.valid) continue;
+                const int srow = (m.bh * a.nchunks + m.c) * kD;
+                if (!(ok = acquire())) break;
+                issue(&tm_q, 3, m.t0row, m.bh, 0);
+                if (!(ok = acquire())) break;
+                issue(&tm_k, 3, m.c0, m.bh, 0);
+                for (int t = 0; ok && t < m.nk; ++t) {
+                    if (t + 1 < m.nk) {
+                        if (!(ok = acquire())) break;
+                        issue(&tm_k, 3, m.c0 + (t + 1) * kKeyTile, m.bh, 0);
+                    }
+                    if (t < m.nsp) {
+                        if (!(ok = acquire())) break;
+                        issue(&tm_s, 2, srow + kBlk * t, 0, 0);
+                    }
+                    if (!(ok = acquire())) break;
+                    issue(&tm_v, 4, m.h, m.c0 + t * kKeyTile, m.b);
+                }
+                for (int p = m.nk; ok && p < m.nsp; ++p) {
+                    if (!(ok = acquire())) break;
+                    issue(&tm_s, 2, srow + kBlk * p, 0, 0);
+                }
+                if (ok && (ok = acquire())) {                // the gate/output tile
+                    if (a.has_gate) {
+                        issue(&tm_g, 4, m.h, m.t0row, m.b);
+                    } else {
+                        mbar_arrive(&rfull[it % kSlots]);     // reserved for the output rows
+                        ++it;
+                    }
+                }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t id_qk = idesc_bf16(128, kKeyTile, 0, 0);
             const uint32_t id_pv = idesc_bf16(128, 256, 0, 1);
-            const uint32_t sK = smem_u32(smem + TcOutSmem::kK);
-            const uint32_t sV = smem_u32(smem + TcOutSmem::kV);
-            const uint32_t sY = smem_u32(ybuf);
-            bool ok = mbar_wait(&q_full, 0, &abort_flag, err);
-            if (ok) {
+            const uint32_t sbase = smem_u32(smem);
+            const uint32_t sP = sbase + TcOutSmem::kP;
+            int it = 0, nqk = 0, npv = 0, li = 0;
+            bool ok = true;
+            auto take = [&]() -> bool {
+                if (!mbar_wait(&rfull[it % kSlots], (it / kSlots) & 1, &abort_flag, err)) return false;
                 tc_fence_after();
-                // Qt (K-major, 128-byte swizzle) -> TMEM, 16 columns of K per copy
-#pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks)
-                    tmem_cp_128x256b(tQ + 8 * ks,
-                                     smem_desc_sw128(sY + (ks / 4) * kBox + (ks % 4) * 32, 16, 1024));
-                mma_commit(&q_copied);
-            }
-            bool o_written = false;
-            int it = 0;
-            auto qs_part = [&](int p) -> bool {
-                const int s = it % kKRing;
-                if (!mbar_wait(&kfull[s], (it / kKRing) & 1, &abort_flag, err)) return false;
-                tc_fence_after();
-                const uint32_t base = sK + s * TcOutSmem::kStage;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16_ts(tO, tQ + 8 * (4 * p + kk),
-                                smem_desc_sw128(base + kk * 2048, kBox64, 1024), id_pv,
-                                (o_written || kk > 0) ? 1u : 0u);
-                o_written = true;
-                mma_commit(&kempty[s]);
-                ++it;
                 return true;
             };
-            for (int t = 0; ok && t <= nk; ++t) {
-                if (t < nk) {
-                    const int s = it % kKRing;
-                    if (!mbar_wait(&kfull[s], (it / kKRing) & 1, &abort_flag, err)) { ok = false; break; }
-                    if (t >= 2 && !mbar_wait(&s_free[t & 1], ((t - 2) >> 1) & 1, &abort_flag, err)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t base = sK + s * TcOutSmem::kStage;
+            for (int w = blockIdx.x; ok && w < a.items; w += gridDim.x, ++li) {
+                const TcItem m = tc_item(a, w);
+                if (!m.valid) { --li; continue; }
+                bool o_written = false;
+                // O is free once the previous item's epilogue has read it
+                auto claim_o = [&]() -> bool {
+                    if (o_written || li == 0) return true;
+                    return mbar_wait(&o_free, (li - 1) & 1, &abort_flag, err);
+                };
+                // Qt (K-major, 128-byte swizzle) -> TMEM, 16 columns of K per copy;
+                // ordered after the previous item's MMAs that read Qt.
+                if (!(ok = take())) break;
+                {
+                    const uint32_t base = sbase + (it % kSlots) * kSlot;
 #pragma unroll
                     for (int ks = 0; ks < kD / 16; ++ks)
-                        mma_bf16_ts(tSP(t), tQ + 8 * ks,
-                                    smem_desc_sw128(base + (ks / 4) * kBox64 + (ks % 4) * 32, 16, 1024),
-                                    id_qk, ks > 0 ? 1u : 0u);
-                    mma_commit(&kempty[s]);
-                    mma_commit(&s_full[t & 1]);
+                        tmem_cp_128x256b(tQ + 8 * ks,
+                                         smem_desc_sw128(base + (ks / 4) * kBox + (ks % 4) * 32, 16, 1024));
+                    mma_commit(&rempty[it % kSlots]);
                     ++it;
-                    if (t < nsp && !(ok = qs_part(t))) break;
                 }
-                if (t >= 1) {
-                    const int u = t - 1;
-                    if (!mbar_wait(&p_full[u & 1], (u >> 1) & 1, &abort_flag, err)) { ok = false; break; }
-                    if (!mbar_wait(&vfull[u % kVRing], (u / kVRing) & 1, &abort_flag, err)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t base = sV + (u % kVRing) * TcOutSmem::kStage;
+                auto qk = [&](int t) -> bool {
+                    if (nqk >= 1 && !mbar_wait(&s_read, (nqk - 1) & 1, &abort_flag, err)) return false;
+                    if (!take()) return false;
+                    const uint32_t base = sbase + (it % kSlots) * kSlot;
 #pragma unroll
-                    for (int kk = 0; kk < kKeyTile / 16; ++kk)   // P halves at columns 0 and 32
-                        mma_bf16_ts(tO, tSP(u) + 8 * kk + (kk >= 2 ? 16 : 0),
-                                    smem_desc_sw128(base + kk * 2048, kBox64, 1024), id_pv,
+                    for (int ks = 0; ks < kD / 16; ++ks)
+                        mma_bf16_ts(tS, tQ + 8 * ks,
+                                    smem_desc_sw128(base + (ks / 4) * kBox + (ks % 4) * 32, 16, 1024),
+                                    id_qk, ks > 0 ? 1u : 0u);
+                    mma_commit(&rempty[it % kSlots]);
+                    mma_commit(&s_full);
+                    ++it;
+                    ++nqk;
+                    (void)t;
+                    return true;
+                };
+                // O += Qt[:, 128p .. 128p+128) S_prev[128p .. 128p+128, :]
+                auto qs_half = [&](int p) -> bool {
+                    if (!take() || !claim_o()) return false;
+                    const uint32_t base = sbase + (it % kSlots) * kSlot;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ts(tO, tQ + 8 * (8 * p + kk),
+                                    smem_desc_sw128(base + kk * 2048, kBox, 1024), id_pv,
                                     (o_written || kk > 0) ? 1u : 0u);
                     o_written = true;
-                    mma_commit(&vempty[u % kVRing]);
-                    mma_commit(&s_free[u & 1]);
+                    mma_commit(&rempty[it % kSlots]);
+                    ++it;
+                    return true;
+                };
+                ok = qk(0);
+                for (int t = 0; ok && t < m.nk; ++t) {
+                    if (t + 1 < m.nk && !(ok = qk(t + 1))) break;
+                    if (t < m.nsp && !(ok = qs_half(t))) break;
+                    if (!mbar_wait(&p_full, npv & 1, &abort_flag, err)) { ok = false; break; }
+                    if (!(ok = take() && claim_o())) break;
+                    const uint32_t base = sbase + (it % kSlots) * kSlot;
+#pragma unroll
+                    for (int kk = 0; kk < kKeyTile / 16; ++kk)
+                        mma_bf16(tO, smem_desc_sw128(sP + (kk / 4) * kBox + (kk % 4) * 32, 16, 1024),
+                                 smem_desc_sw128(base + kk * 2048, kBox, 1024), id_pv,
+                                 (o_written || kk > 0) ? 1u : 0u);
+                    o_written = true;
+                    mma_commit(&rempty[it % kSlots]);
+                    mma_commit(&p_free);
+                    ++it;
+                    ++npv;
                 }
+                for (int p = m.nk; ok && p < m.nsp; ++p) ok = qs_half(p);
+                mma_commit(&o_full);
+                ++it;                                          // skip the gate/output item
             }
-            for (int p = nk; ok && p < nsp; ++p) ok = qs_part(p);
-            mma_commit(&o_full);
         }
     } else {
-        // two warpgroups: wg 0 owns S columns [0,32) and O columns [0,128),
-        // wg 1 owns S columns [32,64) and O columns [128,256)
+        // two warpgroups: for every tile wg w masks and converts S columns
+        // [64w, 64w+64); in the epilogue wg w owns O columns [128w, 128w+128)
         const int wg = (warp - 2) / 4;
         const int q4 = warp % 4;
         const int row = 32 * q4 + lane;                         // row of the 128-row block
         const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
-        const int lrow = r * kBlk + row;                        // row within the chunk
-        const int t_row = t0row + row;
+        uint8_t *prow = pbuf + wg * kBox + row * 128;           // this row in P box wg
+        int it_base = 0, ntile = 0, li = 0;
         bool ok = true;
-        for (int t = 0; t < nk; ++t) {
-            if (!warp_wait(&s_full[t & 1], (t >> 1) & 1, &abort_flag, err)) { ok = false; break; }
-            tc_fence_after();
-            uint32_t v[32];
-            tmem_ld32(tSP(t) + lane_off + 32 * wg, v);
-            tmem_wait_ld();
-            const int j0 = t * kKeyTile + 32 * wg;              // first key of this half tile
-            uint32_t w[16];
-            if (j0 + 31 <= lrow) {                              // every key at or before the row
-#pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    w[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
-            } else {
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float x0 = (lrow >= j0 + 2 * e) ? __uint_as_float(v[2 * e]) : 0.f;
-                    const float x1 = (lrow >= j0 + 2 * e + 1) ? __uint_as_float(v[2 * e + 1]) : 0.f;
-                    w[e] = pack_bf16x2(x0, x1);
-                }
-            }
-            // P (bf16 pairs) goes to the first 16 columns of this warpgroup's own
-            // 32 S columns, so it never overwrites S the other warpgroup still reads.
-            tmem_st16(tSP(t) + lane_off + 32 * wg, w);
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&p_full[t & 1]);
-        }
-        const bool go = ok && warp_wait(&o_full, 0, &abort_flag, err) &&
-                        (!a.has_gate || warp_wait(&g_full, 0, &abort_flag, err));
-        // The K ring is idle once O is complete: its first bytes hold the
-        // two warpgroups' partial row sums.
-        float (*red)[kBlk] = reinterpret_cast<float (*)[kBlk]>(smem + TcOutSmem::kK);
-        float mean = 0.f, rstd = 1.f;
-        if (go) tc_fence_after();
-        if (a.has_gate) {
-            // GroupNorm statistics over the row's 256 channels; each
-            // warpgroup sums its half and the halves meet in shared memory.
-            float sum = 0.f;
-            if (go) {
-#pragma unroll 1
-                for (int cb = 0; cb < 4; ++cb) {
-                    uint32_t v[32];
-                    tmem_ld32(tO + lane_off + 128 * wg + 32 * cb, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) sum += __uint_as_float(v[e]);
-                }
-            }
-            red[wg][row] = sum;
-            named_barrier(1, kEpiThreads);
-            mean = (red[0][row] + red[1][row]) * (1.f / kD);
-            named_barrier(1, kEpiThreads);
-            float sq = 0.f;
-            if (go) {
-#pragma unroll 1
-                for (int cb = 0; cb < 4; ++cb) {
-                    uint32_t v[32];
-                    tmem_ld32(tO + lane_off + 128 * wg + 32 * cb, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float d = __uint_as_float(v[e]) - mean;
-                        sq = fmaf(d, d, sq);
-                    }
-                }
-            }
-            red[wg][row] = sq;
-            named_barrier(1, kEpiThreads);
-            rstd = rsqrtf((red[0][row] + red[1][row]) * (1.f / kD) + a.eps);
-        }
-        if (go) {
-            // This row's slot in the 128-byte-swizzled output/gate tile.
-            uint8_t *yrow = ybuf + row * 128;
-            const int sw = row & 7;
-            const float *wv = a.gn_weight ? a.gn_weight + h * kD : nullptr;
-            const float *bv = a.gn_bias ? a.gn_bias + h * kD : nullptr;
-#pragma unroll 1
-            for (int k4 = 0; k4 < 4; ++k4) {
-                const int cb = 4 * wg + k4;                       // 32-column block
-                uint32_t v[32];
-                tmem_ld32(tO + lane_off + 32 * cb, v);
+        for (int w = blockIdx.x; ok && w < a.items; w += gridDim.x, ++li) {
+            const TcItem m = tc_item(a, w);
+            if (!m.valid) { --li; continue; }
+            const int lrow = m.r * kBlk + row;                  // row within the chunk
+            for (int t = 0; t < m.nk; ++t, ++ntile) {
+                if (!warp_wait(&s_full, ntile & 1, &abort_flag, err)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t v0[32], v1[32];
+                const uint32_t col = tS + lane_off + 64 * wg;
+                tmem_ld32(col, v0);
+                tmem_ld32(col + 32, v1);
                 tmem_wait_ld();
-                uint8_t *box = yrow + (cb >> 1) * kBox;
+                tc_fence_before();
+                mbar_arrive(&s_read);                           // S may be overwritten now
+                const int j0 = t * kKeyTile + 64 * wg;          // first key of this half tile
+                uint32_t wv[32];
+                if (j0 + 63 <= lrow) {                          // every key at or before the row
 #pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    uint4 *slot = reinterpret_cast<uint4 *>(box + ((((cb & 1) * 4 + q8) ^ sw) * 16));
-                    float y[8];
-                    if (a.has_gate) {
-                        uint4 graw = *slot;
-                        const __nv_bfloat162 *g2 = reinterpret_cast<const __nv_bfloat162 *>(&graw);
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            const float2 gg = __bfloat1622float2(g2[e2]);
-#pragma unroll
-                            for (int hh = 0; hh < 2; ++hh) {
-                                const int e = 2 * e2 + hh;
-                                const int ch = 32 * cb + 8 * q8 + e;
-                                float yh = (__uint_as_float(v[8 * q8 + e]) - mean) * rstd;
-                                if (wv) yh *= wv[ch];
-                                if (bv) yh += bv[ch];
-                                const float g = hh ? gg.y : gg.x;
-                                y[e] = __fdividef(g, 1.f + __expf(-g)) * yh;
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) y[e] = __uint_as_float(v[8 * q8 + e]);
+                    for (int e = 0; e < 16; ++e) {
+                        wv[e] = pack_bf16x2(__uint_as_float(v0[2 * e]), __uint_as_float(v0[2 * e + 1]));
+                        wv[16 + e] = pack_bf16x2(__uint_as_float(v1[2 * e]), __uint_as_float(v1[2 * e + 1]));
                     }
-                    *slot = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
-                                       pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int j = j0 + 2 * e;
+                        const float x0 = (lrow >= j) ? __uint_as_float(v0[2 * e]) : 0.f;
+                        const float x1 = (lrow >= j + 1) ? __uint_as_float(v0[2 * e + 1]) : 0.f;
+                        const float y0 = (lrow >= j + 32) ? __uint_as_float(v1[2 * e]) : 0.f;
+                        const float y1 = (lrow >= j + 33) ? __uint_as_float(v1[2 * e + 1]) : 0.f;
+                        wv[e] = pack_bf16x2(x0, x1);
+                        wv[16 + e] = pack_bf16x2(y0, y1);
+                    }
                 }
+                // the previous tile's P must have been consumed by its P V
+                if (ntile >= 1 && !warp_wait(&p_free, (ntile - 1) & 1, &abort_flag, err)) { ok = false; break; }
+                // 64 keys of this row = eight 16-byte chunks of the 128-byte-swizzled box
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    *reinterpret_cast<uint4 *>(prow + ((ch ^ (row & 7)) * 16)) =
+                        make_uint4(wv[4 * ch], wv[4 * ch + 1], wv[4 * ch + 2], wv[4 * ch + 3]);
+                fence_async_shared();
+                tc_fence_before();
+                mbar_arrive(&p_full);
             }
-            fence_async_shared();
+            // ring items of this work item: Qt, nk Kt tiles, nsp S_prev halves,
+            // nk V tiles, then the gate/output tile
+            const int ig = it_base + 1 + 2 * m.nk + m.nsp;
+            it_base = ig + 1;
+            uint8_t *ybuf = slot_ptr(ig);
+            const bool go = ok && warp_wait(&o_full, li & 1, &abort_flag, err) &&
+                            warp_wait(&rfull[ig % kSlots], (ig / kSlots) & 1, &abort_flag, err);
+            // the P tile is idle between items: it holds the partial row sums
+            float (*red)[kBlk] = reinterpret_cast<float (*)[kBlk]>(pbuf);   // [4][128]
+            float mean = 0.f, rstd = 1.f;
+            if (go) tc_fence_after();
+            if (a.has_gate) {
+                // GroupNorm statistics over the row's 256 channels: each
+                // warpgroup sums its half (values and squares, shifted by the
+                // row's first value for accuracy); the halves meet in shared memory.
+                float sum = 0.f, sq = 0.f, shift = 0.f;
+                if (go) {
+                    uint32_t v0[32];
+                    tmem_ld32(tO + lane_off, v0);           // column 0 of the row: the shift
+                    tmem_wait_ld();
+                    shift = __uint_as_float(v0[0]);
+#pragma unroll 1
+                    for (int cb = 0; cb < 4; ++cb) {
+                        uint32_t v[32];
+                        tmem_ld32(tO + lane_off + 128 * wg + 32 * cb, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const float d = __uint_as_float(v[e]) - shift;
+                            sum += d;
+                            sq = fmaf(d, d, sq);
+                        }
+                    }
+                }
+                red[2 * wg][row] = sum;
+                red[2 * wg + 1][row] = sq;
+                named_barrier(1, kEpiThreads);
+                const float ms = (red[0][row] + red[2][row]) * (1.f / kD);  // mean of x - shift
+                const float m2 = (red[1][row] + red[3][row]) * (1.f / kD);
+                mean = shift + ms;
+                rstd = rsqrtf(fmaxf(m2 - ms * ms, 0.f) + a.eps);
+                named_barrier(1, kEpiThreads);              // red is reused as P next
+            }
+            if (go) {
+                // This row's slot in the 128-byte-swizzled gate/output tile.
+                uint8_t *yrow = ybuf + row * 128;
+                const int sw = row & 7;
+                const float *gw = a.gn_weight ? a.gn_weight + m.h * kD : nullptr;
+                const float *gb = a.gn_bias ? a.gn_bias + m.h * kD : nullptr;
+#pragma unroll 1
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const int cb = 4 * wg + k4;                   // 32-column block of O
+                    uint32_t v[32];
+                    tmem_ld32(tO + lane_off + 32 * cb, v);
+                    tmem_wait_ld();
+                    if (k4 == 3) {                                // O fully read: free it
+                        tc_fence_before();
+                        mbar_arrive(&o_free);
+                    }
+                    uint8_t *box = yrow + (cb >> 1) * kBox;
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8) {
+                        uint4 *slot = reinterpret_cast<uint4 *>(box + ((((cb & 1) * 4 + q8) ^ sw) * 16));
+                        float y[8];
+                        if (a.has_gate) {
+                            uint4 graw = *slot;
+                            const __nv_bfloat162 *g2 = reinterpret_cast<const __nv_bfloat162 *>(&graw);
+#pragma unroll
+                            for (int e2 = 0; e2 < 4; ++e2) {
+                                const float2 gg = __bfloat1622float2(g2[e2]);
+#pragma unroll
+                                for (int hh = 0; hh < 2; ++hh) {
+                                    const int e = 2 * e2 + hh;
+                                    const int ch = 32 * cb + 8 * q8 + e;
+                                    float yh = (__uint_as_float(v[8 * q8 + e]) - mean) * rstd;
+                                    if (gw) yh *= gw[ch];
+                                    if (gb) yh += gb[ch];
+                                    y[e] = swish_fast(hh ? gg.y : gg.x) * yh;
+                                }
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) y[e] = __uint_as_float(v[8 * q8 + e]);
+                        }
+                        *slot = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
+                                           pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
+                    }
+                }
+                fence_async_shared();
+            } else {
+                mbar_arrive(&o_free);
+            }
+            // Both epilogue warpgroups reach this barrier on every path.
+            named_barrier(1, kEpiThreads);
+            if (wg == 0 && row == 0) {
+                if (!abort_flag) {
+                    for (int x = 0; x < 4; ++x)
+                        tma_store_4d(&tm_out, ybuf + x * kBox, 64 * x, m.h, m.t0row, m.b);
+                    tma_store_commit();
+                    tma_store_wait_read();
+                }
+                mbar_arrive(&rempty[ig % kSlots]);             // the tile may be refilled
+            }
+            if (!go) ok = false;
         }
-        // Both epilogue warpgroups reach this barrier on every path.
-        named_barrier(1, kEpiThreads);
-        if (wg == 0 && row == 0 && !abort_flag) {
-            for (int x = 0; x < 4; ++x) tma_store_4d(&tm_out, ybuf + x * kBox, 64 * x, h, t0row, b);
-            tma_store_commit();
-            tma_store_wait_read();
-        }
-        (void)t_row;
     }
     tc_fence_before();
     __syncthreads();
@@ -725,32 +814,27 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
         hp.decay_last[h] = (float)std::pow(g, (double)last_len);
     }
 
-    // tensor maps: 128-row boxes for the state pass, 64-row boxes for the output pass
-    CUtensorMap tm_q128, tm_k128, tm_v128, tm_k64, tm_v64, tm_s64;
+    // tensor maps: every tile is 128 rows (tokens, or d_k rows of S_prev) by
+    // 64 channels, 128-byte swizzled
+    CUtensorMap tm_q, tm_k, tm_v, tm_s;
     {
         cuuint64_t dims[3] = {kD, (cuuint64_t)n, (cuuint64_t)BH};
         cuuint64_t str[2] = {kD * 2, (cuuint64_t)n * kD * 2};
-        cuuint32_t box128[3] = {64, kBlk, 1};
-        cuuint32_t box64[3] = {64, kKeyTile, 1};
-        if (!make_map(&tm_k128, kt, 3, dims, str, box128) ||
-            !make_map(&tm_k64, kt, 3, dims, str, box64) ||
-            !make_map(&tm_q128, qt, 3, dims, str, box128))
+        cuuint32_t box[3] = {64, kBlk, 1};
+        if (!make_map(&tm_k, kt, 3, dims, str, box) || !make_map(&tm_q, qt, 3, dims, str, box))
             return cudaErrorInvalidValue;
     }
     {
         cuuint64_t dims[4] = {kD, (cuuint64_t)H, (cuuint64_t)n, (cuuint64_t)B};
         cuuint64_t str[3] = {kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)n * H * kD * 2};
-        cuuint32_t box128[4] = {64, 1, kBlk, 1};
-        cuuint32_t box64[4] = {64, 1, kKeyTile, 1};
-        if (!make_map(&tm_v128, a.v, 4, dims, str, box128) ||
-            !make_map(&tm_v64, a.v, 4, dims, str, box64))
-            return cudaErrorInvalidValue;
+        cuuint32_t box[4] = {64, 1, kBlk, 1};
+        if (!make_map(&tm_v, a.v, 4, dims, str, box)) return cudaErrorInvalidValue;
     }
     {
         cuuint64_t dims[2] = {kD, (cuuint64_t)BH * nchunks * kD};
         cuuint64_t str[1] = {kD * 2};
-        cuuint32_t box[2] = {64, 64};
-        if (!make_map(&tm_s64, sp, 2, dims, str, box)) return cudaErrorInvalidValue;
+        cuuint32_t box[2] = {64, kBlk};
+        if (!make_map(&tm_s, sp, 2, dims, str, box)) return cudaErrorInvalidValue;
     }
     // output and gate tiles: 128 tokens x 64 channels of one head
     CUtensorMap tm_out, tm_g;
@@ -780,7 +864,7 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
         e = cudaFuncSetAttribute(tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         KernelTimer timer("tc_state", stream);
-        tc_state_kernel<<<BH * 4, kTcThreads, smem, stream>>>(tm_k128, tm_v128, hp, a.state_in,
+        tc_state_kernel<<<BH * 4, kTcThreads, smem, stream>>>(tm_k, tm_v, hp, a.state_in,
                                                              a.state_out, sp, H, n, C, nchunks,
                                                              err);
         count_launch();
@@ -795,14 +879,18 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
         oa.gn_bias = a.gate ? a.gate->bias : nullptr;
         oa.eps = a.gate ? a.gate->eps : 0.f;
         oa.err = err;
+        oa.items = BH * nchunks * oa.rblocks;
         const int smem = (int)TcOutSmem::kBytes;
         e = cudaFuncSetAttribute(tc_output_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  smem);
         if (e != cudaSuccess) return e;
-        const unsigned grid = (unsigned)(BH * nchunks * oa.rblocks);
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess)
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const unsigned grid = (unsigned)std::min(oa.items, sms);
         KernelTimer timer("tc_output", stream);
-        tc_output_kernel<<<grid, kOutThreads, smem, stream>>>(tm_q128, tm_k64, tm_v64, tm_s64, tm_g,
-                                                             tm_out, oa);
+        tc_output_kernel<<<grid, kOutThreads, smem, stream>>>(tm_q, tm_k, tm_v, tm_s, tm_g, tm_out,
+                                                             oa);
         count_launch();
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
