@@ -64,6 +64,28 @@ tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
                int batch, int heads, int n, int chunk, long long pos0, int rotate) {
     __shared__ float2 cs[kD / 2];
     const int t = blockIdx.x;
+    const int i = t % chunk;                        // index inside the chunk
+    const int tasks = batch * heads * (kD / 8);
+    // Up to kPrepBatch 8-element tasks per thread per round; the first
+    // round's loads are issued before the (cos, sin) prologue so its latency
+    // overlaps the memory traffic.
+    constexpr int kPrepBatch = 4;
+    uint4 rq[kPrepBatch], rk[kPrepBatch];
+    auto load_round = [&](int base) {
+#pragma unroll
+        for (int u = 0; u < kPrepBatch; ++u) {
+            const int task = base + u * blockDim.x;
+            if (task < tasks) {
+                const int part = task % (kD / 8);
+                const int bhi = task / (kD / 8);
+                const int h = bhi % heads, b = bhi / heads;
+                const size_t src = (((size_t)b * n + t) * heads + h) * kD + part * 8;
+                rq[u] = *reinterpret_cast<const uint4 *>(q + src);
+                rk[u] = *reinterpret_cast<const uint4 *>(k + src);
+            }
+        }
+    };
+    load_round(threadIdx.x);
     if (threadIdx.x < kD / 2) {
         float2 v = make_float2(1.f, 0.f);
         if (rotate) {
@@ -78,13 +100,8 @@ tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
         cs[threadIdx.x] = v;
     }
     __syncthreads();
-    const int i = t % chunk;                        // index inside the chunk
-    const int tasks = batch * heads * (kD / 8);
-    // Up to kPrepBatch tasks per thread with every load issued before any
-    // arithmetic, so each thread keeps 2 * kPrepBatch 16-byte loads in flight.
-    constexpr int kPrepBatch = 4;
     for (int base = threadIdx.x; base < tasks; base += kPrepBatch * blockDim.x) {
-        uint4 rq[kPrepBatch], rk[kPrepBatch];
+        if (base != (int)threadIdx.x) load_round(base);
 #pragma unroll
         for (int u = 0; u < kPrepBatch; ++u) {
             const int task = base + u * blockDim.x;
@@ -92,37 +109,25 @@ tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
                 const int part = task % (kD / 8);
                 const int bhi = task / (kD / 8);
                 const int h = bhi % heads, b = bhi / heads;
-                const size_t src = (((size_t)b * n + t) * heads + h) * kD + part * 8;
-                rq[u] = *reinterpret_cast<const uint4 *>(q + src);
-                rk[u] = *reinterpret_cast<const uint4 *>(k + src);
-            }
-        }
+                const float e = (float)(i + 1) * pp.log2g[h];
+                const float sq = exp2f(e), sk = exp2f(-e);
+                const __nv_bfloat162 *hq = reinterpret_cast<const __nv_bfloat162 *>(&rq[u]);
+                const __nv_bfloat162 *hk = reinterpret_cast<const __nv_bfloat162 *>(&rk[u]);
+                float oq[8], ok[8];
 #pragma unroll
-        for (int u = 0; u < kPrepBatch; ++u) {
-            const int task = base + u * blockDim.x;
-            if (task < tasks) {
-            const int part = task % (kD / 8);
-            const int bhi = task / (kD / 8);
-            const int h = bhi % heads, b = bhi / heads;
-            const float e = (float)(i + 1) * pp.log2g[h];
-            const float sq = exp2f(e), sk = exp2f(-e);
-            const __nv_bfloat162 *hq = reinterpret_cast<const __nv_bfloat162 *>(&rq[u]);
-            const __nv_bfloat162 *hk = reinterpret_cast<const __nv_bfloat162 *>(&rk[u]);
-            float oq[8], ok[8];
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                const float2 r = cs[part * 4 + p];
-                const float cq = r.x * sq, sq2 = r.y * sq, ck = r.x * sk, sk2 = r.y * sk;
-                const float2 xq = __bfloat1622float2(hq[p]);
-                const float2 xk = __bfloat1622float2(hk[p]);
-                oq[2 * p] = xq.x * cq - xq.y * sq2;
-                oq[2 * p + 1] = xq.x * sq2 + xq.y * cq;
-                ok[2 * p] = xk.x * ck - xk.y * sk2;
-                ok[2 * p + 1] = xk.x * sk2 + xk.y * ck;
-            }
-            const size_t dst = (((size_t)b * heads + h) * n + t) * kD + part * 8;
-            store8(qt + dst, oq);
-            store8(kt + dst, ok);
+                for (int p = 0; p < 4; ++p) {
+                    const float2 r = cs[part * 4 + p];
+                    const float cq = r.x * sq, sq2 = r.y * sq, ck = r.x * sk, sk2 = r.y * sk;
+                    const float2 xq = __bfloat1622float2(hq[p]);
+                    const float2 xk = __bfloat1622float2(hk[p]);
+                    oq[2 * p] = xq.x * cq - xq.y * sq2;
+                    oq[2 * p + 1] = xq.x * sq2 + xq.y * cq;
+                    ok[2 * p] = xk.x * ck - xk.y * sk2;
+                    ok[2 * p + 1] = xk.x * sk2 + xk.y * ck;
+                }
+                const size_t dst = (((size_t)b * heads + h) * n + t) * kD + part * 8;
+                store8(qt + dst, oq);
+                store8(kt + dst, ok);
             }
         }
     }
@@ -300,7 +305,7 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
 // ------------------------------------------------------------------ output pass
 // Persistent: one CTA per SM walks work items (sequence, head, chunk,
-// 128-row block), heavy row blocks first, so the loads and the first
+// 128-row block), so the loads and the first
 // QK^T of the next item overlap the epilogue of the current one.
 // TMEM (512 columns, allocated once): O [0,256) f32; Qt [256,384) bf16 pairs
 // (A operand); S [384,512): S = Qt Kt^T for a 128-key tile in f32 (N = 128
@@ -343,14 +348,17 @@ struct TcItem {
     bool valid;
 };
 
-// Work item w, heavy row blocks first: w -> (r from the last block down, bh, c).
+// Work item w: group g = w / rblocks is one (sequence, head, chunk); its
+// row blocks sit at consecutive w, so CTAs working side by side share that
+// chunk's Kt, V and S_prev tiles through L2.  The row block is rotated by
+// the group index, r = (w + g) mod rblocks, so a CTA striding by the grid
+// size still meets a mix of heavy and light blocks.
 __device__ __forceinline__ TcItem tc_item(const TcOutArgs &a, int w) {
     TcItem it;
-    const int per_r = a.items / a.rblocks;
-    it.r = a.rblocks - 1 - w / per_r;
-    const int rest = w % per_r;
-    it.c = rest % a.nchunks;
-    it.bh = rest / a.nchunks;
+    const int g = w / a.rblocks;
+    it.r = (w + g) % a.rblocks;
+    it.c = g % a.nchunks;
+    it.bh = g / a.nchunks;
     it.b = it.bh / a.heads;
     it.h = it.bh % a.heads;
     it.c0 = it.c * a.chunk;

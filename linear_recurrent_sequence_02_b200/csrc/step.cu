@@ -6,23 +6,20 @@
 // [dk, dv] is read and written once, so the step is an HBM stream:
 // 8 * dk * dv bytes per head-step against ~5 dk dv flops.
 //
-// Layout of the work: a thread-block cluster owns one (sequence, head).
-// Each CTA of the cluster owns a slab of 32 state rows; each thread owns a
-// float4 of columns and walks a few rows, so o's partial sums need no
-// shuffles.  Partials are reduced across the row lanes in shared memory and
-// across the cluster through distributed shared memory, by cluster rank 0.
-#include <cooperative_groups.h>
-
+// Layout of the work: CTA (sequence, head, 32-column slab of S) owns every
+// row of its slab, so its 32 outputs are complete inside the CTA.  Each
+// thread owns a float4 of columns for dk/32 rows, issues all of its state
+// loads first, updates S in place and accumulates o; the 32 row lanes are
+// reduced in shared memory.
 #include <cmath>
 
 #include "kernels.h"
 
-namespace cg = cooperative_groups;
-
 namespace retnet {
 
 constexpr int kStepThreads = 256;
-constexpr int kStepRows = 32;       // state rows per CTA
+constexpr int kStepCols = 32;       // state columns per CTA
+constexpr int kStepLanes = kStepThreads / (kStepCols / 4);   // 32 row lanes
 
 // (cos, sin) of pos * theta_j for the pairs of this step, formed on the host
 // in float64 (the position is a host scalar), j < dk / 2 <= 128.
@@ -45,43 +42,38 @@ __device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16 *p, flo
     o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y;
 }
 
-template <typename T, int DV>
+template <typename T, int DK>
 __global__ void __launch_bounds__(kStepThreads)
 retention_step_kernel(const T *__restrict__ q, const T *__restrict__ k,
                       const T *__restrict__ v, HeadGammas gam, StepRotation rot,
-                      float *__restrict__ state, T *__restrict__ out, int heads, int dk,
+                      float *__restrict__ state, T *__restrict__ out, int heads, int dv,
                       int rotate) {
-    constexpr int NCG = DV / 4;                      // float4 column groups
-    constexpr int NRL = kStepThreads / NCG;          // row lanes
-    constexpr int RPL = kStepRows / NRL;             // rows per lane: 2, 4 or 8
-    cg::cluster_group cluster = cg::this_cluster();
+    constexpr int RPL = DK / kStepLanes;             // rows per thread: 2, 4 or 8
     const int bh = blockIdx.x;                       // sequence * heads + head
     const int h = bh % heads;
-    const int row0 = blockIdx.y * kStepRows;         // blockIdx.y == cluster rank
+    const int col0 = blockIdx.y * kStepCols;
     const float g = gam.g[h];
-    const int cgi = threadIdx.x % NCG;
-    const int rl = threadIdx.x / NCG;
+    const int cgi = threadIdx.x % (kStepCols / 4);   // float4 column group in the slab
+    const int rl = threadIdx.x / (kStepCols / 4);    // row lane
 
-    __shared__ float qs[kStepRows], ks[kStepRows];
-    __shared__ float4 red[kStepThreads];
-    __shared__ float4 partial[NCG];
+    __shared__ float qs[DK], ks[DK];
+    __shared__ float4 red[kStepLanes][kStepCols / 4];
 
     // Issue this thread's state loads first: they do not depend on q, k, v.
-    float *S = state + (size_t)bh * dk * DV;
+    float *S = state + (size_t)bh * DK * dv + col0 + cgi * 4;
     float4 s[RPL];
 #pragma unroll
-    for (int i = 0; i < RPL; ++i)
-        s[i] = reinterpret_cast<const float4 *>(S + (size_t)(row0 + rl + i * NRL) * DV)[cgi];
+    for (int i = 0; i < RPL; ++i) s[i] = *reinterpret_cast<const float4 *>(S + (size_t)(rl + i * kStepLanes) * dv);
 
-    // Rotated q, k entries of this CTA's rows (pairs never straddle CTAs).
-    if (threadIdx.x < kStepRows / 2) {
-        const int r = row0 + 2 * threadIdx.x;
-        const T *qh = q + (size_t)bh * dk + r;
-        const T *kh = k + (size_t)bh * dk + r;
+    // Rotated q and k of the whole head (every row of the slab is used).
+    if (threadIdx.x < DK / 2) {
+        const int r = 2 * threadIdx.x;
+        const T *qh = q + (size_t)bh * DK + r;
+        const T *kh = k + (size_t)bh * DK + r;
         float q0 = to_f32(qh[0]), q1 = to_f32(qh[1]);
         float k0 = to_f32(kh[0]), k1 = to_f32(kh[1]);
         if (rotate) {
-            const float2 cs = rot.cs[r / 2];
+            const float2 cs = rot.cs[threadIdx.x];
             float a = q0;
             q0 = a * cs.x - q1 * cs.y;
             q1 = a * cs.y + q1 * cs.x;
@@ -89,78 +81,44 @@ retention_step_kernel(const T *__restrict__ q, const T *__restrict__ k,
             k0 = a * cs.x - k1 * cs.y;
             k1 = a * cs.y + k1 * cs.x;
         }
-        qs[2 * threadIdx.x] = q0; qs[2 * threadIdx.x + 1] = q1;
-        ks[2 * threadIdx.x] = k0; ks[2 * threadIdx.x + 1] = k1;
+        qs[r] = q0; qs[r + 1] = q1;
+        ks[r] = k0; ks[r + 1] = k1;
     }
     float vv[4];
-    load4<T>(v + (size_t)bh * DV + cgi * 4, vv);
+    load4<T>(v + (size_t)bh * dv + col0 + cgi * 4, vv);
     __syncthreads();
 
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < RPL; ++i) {
-        const int rr = rl + i * NRL;
+        const int rr = rl + i * kStepLanes;
         const float kr = ks[rr], qr = qs[rr];
         float4 t = s[i];
         t.x = fmaf(g, t.x, kr * vv[0]);
         t.y = fmaf(g, t.y, kr * vv[1]);
         t.z = fmaf(g, t.z, kr * vv[2]);
         t.w = fmaf(g, t.w, kr * vv[3]);
-        reinterpret_cast<float4 *>(S + (size_t)(row0 + rr) * DV)[cgi] = t;
+        *reinterpret_cast<float4 *>(S + (size_t)rr * dv) = t;
         acc.x = fmaf(qr, t.x, acc.x);
         acc.y = fmaf(qr, t.y, acc.y);
         acc.z = fmaf(qr, t.z, acc.z);
         acc.w = fmaf(qr, t.w, acc.w);
     }
-    red[threadIdx.x] = acc;
+    red[rl][cgi] = acc;
     __syncthreads();
-    if (threadIdx.x < NCG) {
-        float4 t = red[threadIdx.x];
+    if (threadIdx.x < kStepCols / 4) {
+        float4 t = red[0][threadIdx.x];
 #pragma unroll
-        for (int l = 1; l < NRL; ++l) {
-            float4 u = red[l * NCG + threadIdx.x];
+        for (int l = 1; l < kStepLanes; ++l) {
+            const float4 u = red[l][threadIdx.x];
             t.x += u.x; t.y += u.y; t.z += u.z; t.w += u.w;
         }
-        partial[threadIdx.x] = t;
-    }
-    cluster.sync();
-    if (cluster.block_rank() == 0 && threadIdx.x < NCG) {
-        float4 t = partial[threadIdx.x];
-        const unsigned nblk = cluster.num_blocks();
-        for (unsigned r = 1; r < nblk; ++r) {
-            const float4 *rp = cluster.map_shared_rank(partial, r);
-            float4 u = rp[threadIdx.x];
-            t.x += u.x; t.y += u.y; t.z += u.z; t.w += u.w;
-        }
-        T *oh = out + (size_t)bh * DV + threadIdx.x * 4;
+        T *oh = out + (size_t)bh * dv + col0 + threadIdx.x * 4;
         oh[0] = from_f32<T>(t.x);
         oh[1] = from_f32<T>(t.y);
         oh[2] = from_f32<T>(t.z);
         oh[3] = from_f32<T>(t.w);
     }
-    cluster.sync();       // keep every CTA's shared memory alive until rank 0 has read it
-}
-
-template <typename T, int DV>
-static cudaError_t launch_step_typed(const void *q, const void *k, const void *v,
-                                     const HeadGammas &gam, const StepRotation &rot,
-                                     float *state, void *out, int batch, int heads, int dk,
-                                     int rotate, cudaStream_t stream) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(batch * heads), (unsigned)(dk / kStepRows), 1);
-    cfg.blockDim = dim3(kStepThreads, 1, 1);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = (unsigned)(dk / kStepRows);
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    KernelTimer timer("retention_step", stream);
-    return cudaLaunchKernelEx(&cfg, retention_step_kernel<T, DV>, (const T *)q, (const T *)k,
-                              (const T *)v, gam, rot, state, (T *)out, heads, dk, rotate);
 }
 
 template <typename T>
@@ -168,12 +126,25 @@ static cudaError_t launch_step_t(const void *q, const void *k, const void *v,
                                  const HeadGammas &gam, const StepRotation &rot, float *state,
                                  void *out, int batch, int heads, int dk, int dv, int rotate,
                                  cudaStream_t stream) {
-    switch (dv) {
-        case 64: return launch_step_typed<T, 64>(q, k, v, gam, rot, state, out, batch, heads, dk, rotate, stream);
-        case 128: return launch_step_typed<T, 128>(q, k, v, gam, rot, state, out, batch, heads, dk, rotate, stream);
-        case 256: return launch_step_typed<T, 256>(q, k, v, gam, rot, state, out, batch, heads, dk, rotate, stream);
+    const dim3 grid((unsigned)(batch * heads), (unsigned)(dv / kStepCols));
+    KernelTimer timer("retention_step", stream);
+    switch (dk) {
+        case 64:
+            retention_step_kernel<T, 64><<<grid, kStepThreads, 0, stream>>>(
+                (const T *)q, (const T *)k, (const T *)v, gam, rot, state, (T *)out, heads, dv, rotate);
+            break;
+        case 128:
+            retention_step_kernel<T, 128><<<grid, kStepThreads, 0, stream>>>(
+                (const T *)q, (const T *)k, (const T *)v, gam, rot, state, (T *)out, heads, dv, rotate);
+            break;
+        case 256:
+            retention_step_kernel<T, 256><<<grid, kStepThreads, 0, stream>>>(
+                (const T *)q, (const T *)k, (const T *)v, gam, rot, state, (T *)out, heads, dv, rotate);
+            break;
+        default:
+            return cudaErrorInvalidValue;
     }
-    return cudaErrorInvalidValue;
+    return cudaGetLastError();
 }
 
 cudaError_t launch_retention_step(const void *q, const void *k, const void *v,
