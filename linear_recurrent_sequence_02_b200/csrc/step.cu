@@ -11,6 +11,7 @@
 // thread owns a float4 of columns for dk/32 rows, issues all of its state
 // loads first, updates S in place and accumulates o; the 32 row lanes are
 // reduced in shared memory.
+#include <algorithm>
 #include <cmath>
 
 #include "kernels.h"
@@ -46,12 +47,12 @@ template <typename T, int DK>
 __global__ void __launch_bounds__(kStepThreads)
 retention_step_kernel(const T *__restrict__ q, const T *__restrict__ k,
                       const T *__restrict__ v, HeadGammas gam, StepRotation rot,
-                      float *__restrict__ state, T *__restrict__ out, int heads, int dv,
-                      int rotate) {
+                      float *__restrict__ state, T *__restrict__ out, int bh0, int heads,
+                      int dv, int rotate) {
     constexpr int RPL = DK / kStepLanes;             // rows per thread: 2, 4 or 8
-    const int bh = blockIdx.x;                       // sequence * heads + head
+    const int bh = bh0 + blockIdx.y;                 // sequence * heads + head
     const int h = bh % heads;
-    const int col0 = blockIdx.y * kStepCols;
+    const int col0 = blockIdx.x * kStepCols;         // a head's slabs run side by side
     const float g = gam.g[h];
     const int cgi = threadIdx.x % (kStepCols / 4);   // float4 column group in the slab
     const int rl = threadIdx.x / (kStepCols / 4);    // row lane
@@ -126,25 +127,35 @@ static cudaError_t launch_step_t(const void *q, const void *k, const void *v,
                                  const HeadGammas &gam, const StepRotation &rot, float *state,
                                  void *out, int batch, int heads, int dk, int dv, int rotate,
                                  cudaStream_t stream) {
-    const dim3 grid((unsigned)(batch * heads), (unsigned)(dv / kStepCols));
+    const long long bh_total = (long long)batch * heads;
     KernelTimer timer("retention_step", stream);
-    switch (dk) {
-        case 64:
-            retention_step_kernel<T, 64><<<grid, kStepThreads, 0, stream>>>(
-                (const T *)q, (const T *)k, (const T *)v, gam, rot, state, (T *)out, heads, dv, rotate);
-            break;
-        case 128:
-            retention_step_kernel<T, 128><<<grid, kStepThreads, 0, stream>>>(
-                (const T *)q, (const T *)k, (const T *)v, gam, rot, state, (T *)out, heads, dv, rotate);
-            break;
-        case 256:
-            retention_step_kernel<T, 256><<<grid, kStepThreads, 0, stream>>>(
-                (const T *)q, (const T *)k, (const T *)v, gam, rot, state, (T *)out, heads, dv, rotate);
-            break;
-        default:
-            return cudaErrorInvalidValue;
+    // grid.y holds (sequence, head) rows; more than 65535 of them take several launches
+    for (long long bh0 = 0; bh0 < bh_total; bh0 += 65535) {
+        const dim3 grid((unsigned)(dv / kStepCols), (unsigned)std::min(65535LL, bh_total - bh0));
+        switch (dk) {
+            case 64:
+                retention_step_kernel<T, 64><<<grid, kStepThreads, 0, stream>>>(
+                    (const T *)q, (const T *)k, (const T *)v, gam, rot, state, (T *)out, (int)bh0,
+                    heads, dv, rotate);
+                break;
+            case 128:
+                retention_step_kernel<T, 128><<<grid, kStepThreads, 0, stream>>>(
+                    (const T *)q, (const T *)k, (const T *)v, gam, rot, state, (T *)out, (int)bh0,
+                    heads, dv, rotate);
+                break;
+            case 256:
+                retention_step_kernel<T, 256><<<grid, kStepThreads, 0, stream>>>(
+                    (const T *)q, (const T *)k, (const T *)v, gam, rot, state, (T *)out, (int)bh0,
+                    heads, dv, rotate);
+                break;
+            default:
+                return cudaErrorInvalidValue;
+        }
+        count_launch();
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
     }
-    return cudaGetLastError();
+    return cudaSuccess;
 }
 
 cudaError_t launch_retention_step(const void *q, const void *k, const void *v,
@@ -168,7 +179,6 @@ cudaError_t launch_retention_step(const void *q, const void *k, const void *v,
                                                          heads, dk, dv, rotate, stream)
                           : launch_step_t<float>(q, k, v, gam, rot, state, out, batch, heads,
                                                  dk, dv, rotate, stream);
-    count_launch();
     return err;
 }
 

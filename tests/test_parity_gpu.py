@@ -97,6 +97,28 @@ def test_decode_steps(rn, dtype, d, batch):
     assert serr < 1e-5, serr
 
 
+def test_decode_more_rows_than_one_grid(rn):
+    # 4097 sequences x 16 heads = 65552 (sequence, head) rows: more than one
+    # launch's grid holds; rows on both sides of the split are checked.
+    B, H, d, pos = 4097, 16, 64, 7
+    g = torch.Generator(device="cuda")
+    g.manual_seed(11)
+    q, k, v = ((torch.randn(B, H, d, generator=g, device="cuda") / 8).to(torch.bfloat16)
+               for _ in range(3))
+    S = torch.randn(B, H, d, d, generator=g, device="cuda") * 0.1
+    picks = [0, 2048, 4095, 4096]
+    S0 = S[picks].cpu().numpy().astype(np.float64)
+    gam = rn.retnet_default_gammas(H)
+    o = rn.retnet_retention_step(q, k, v, gam, S, pos)
+    torch.cuda.synchronize()
+    qs, ks, vs = (host(x[picks]) for x in (q, k, v))
+    qr = oracle.xpos_rotate(qs[:, None], pos)[:, 0]
+    kr = oracle.xpos_rotate(ks[:, None], pos)[:, 0]
+    o_ref, S_ref = oracle.retention_step(qr, kr, vs, np.float32(gam), S0)
+    assert slice_rel_err(host(o[picks])[:, None], o_ref[:, None]) < TOL["bf16"]
+    assert slice_rel_err(S[picks].cpu().numpy(), S_ref, head_axis=1) < 1e-5
+
+
 def test_decode_without_rotation(rn):
     B, H, d = 2, 2, 64
     rng = np.random.default_rng(4)

@@ -89,6 +89,18 @@ def test_state_in_gate_affine_no_rotation(rn):
     assert slice_rel_err(st, ws, head_axis=1) < TOL
 
 
+def test_more_work_items_than_sms(rn):
+    # 3 x 4 (sequence, head) x 8 chunks x 2 row blocks = 192 output work items:
+    # more than one per SM, so each persistent CTA walks several items.
+    B, n, H = 3, 2048, 4
+    q, k, v, g = inputs(B, n, H, 61, gate_width=256)
+    gam = rn.retnet_default_gammas(H)
+    want, ws = oracle.retention_prefill(q, k, v, np.float32(gam), 256, pos0=3, gate=g)
+    got, st = run(rn, q, k, v, gam, 256, pos0=3, gate=g)
+    assert slice_rel_err(got, want) < TOL
+    assert slice_rel_err(st, ws, head_axis=1) < TOL
+
+
 def test_tensor_matches_simt_path(rn):
     B, n, H = 1, 1024, 4
     q, k, v, g = inputs(B, n, H, 31, gate_width=256)
