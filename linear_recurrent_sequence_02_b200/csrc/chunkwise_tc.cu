@@ -58,7 +58,7 @@ struct TcPrepParams {
     float log2g[kMaxHeads];        // log2(gamma_h)
 };
 
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                TcPrepParams pp, __nv_bfloat16 *__restrict__ qt, __nv_bfloat16 *__restrict__ kt,
                int batch, int heads, int n, int chunk, long long pos0, int rotate) {
