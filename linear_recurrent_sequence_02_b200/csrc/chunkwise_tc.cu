@@ -134,16 +134,21 @@ tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
 }
 
 // ------------------------------------------------------------------ state pass
-// One CTA per (sequence, head, 128x128 quarter of S).  Warp 0 streams Kt and
-// V sub-tiles of 128 tokens through a 3-stage TMA ring; warp 1 accumulates
+// One CTA per (sequence, head, 128 x DVC block of S): the d_k half mh and
+// d_v columns [DVC nv, DVC nv + DVC).  DVC = 128 (four CTAs per
+// sequence-head) by default; DVC = 64 (eight) when there are few
+// sequence-heads, so that more SMs stream.  Warp 0 streams Kt and V
+// sub-tiles of 128 tokens through a TMA ring; warp 1 accumulates
 // U_c = Kt_c^T V_c of every chunk into one of two TMEM buffers (M = d_k
-// quarter, N = d_v quarter, both operands MN-major); warps 2-5 keep the
-// running state row in registers, S <- g^L (S + U_c), hand the buffer back
-// as soon as it is read, and write S_prev of the next chunk (bf16) or the
-// final state (f32).  The tensor core never waits for the state update.
+// half, N = DVC, both operands MN-major); warps 2-5 keep the running state
+// row in registers, S <- g^L (S + U_c), hand the buffer back as soon as it
+// is read, and write S_prev of the next chunk (bf16) or the final state
+// (f32).  The tensor core never waits for the state update.
+template <int DVC>
 struct TcStateSmem {
-    static constexpr int kStages = 3;
-    static constexpr uint32_t kStage = 4 * kBox;       // Kt 128x128 + V 128x128
+    static constexpr int kVBoxes = DVC / 64;
+    static constexpr uint32_t kStage = (2 + kVBoxes) * kBox;   // Kt 128 x 128 + V 128 x DVC
+    static constexpr int kStages = DVC == 128 ? 3 : 4;
     static constexpr uint32_t kBytes = kStages * kStage + 1024;
 };
 
@@ -154,22 +159,25 @@ __device__ __forceinline__ void store_bf16_row(__nv_bfloat16 *dst, const float *
                        sm100::pack_bf16x2(v[i + 4], v[i + 5]), sm100::pack_bf16x2(v[i + 6], v[i + 7]));
 }
 
+template <int DVC>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 TcHeadParams hp, const float *__restrict__ state_in, float *__restrict__ state_out,
                 __nv_bfloat16 *__restrict__ s_prev, int heads, int n, int chunk, int nchunks,
                 unsigned *err) {
+    using Smem = TcStateSmem<DVC>;
+    constexpr int S = Smem::kStages;
+    constexpr int kParts = 2 * (kD / DVC);             // CTAs per sequence-head
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    constexpr int S = TcStateSmem::kStages;
     __shared__ uint64_t full[S], empty[S], acc_full[2], acc_free[2];
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int bh = blockIdx.x / 4;
-    const int quarter = blockIdx.x % 4;
-    const int mh = quarter / 2, nh = quarter % 2;      // d_k half, d_v half
+    const int bh = blockIdx.x / kParts;
+    const int part = blockIdx.x % kParts;
+    const int mh = part / (kD / DVC), nv = part % (kD / DVC);   // d_k half, d_v block
     const int b = bh / heads, h = bh % heads;
 
     if (threadIdx.x == 0) {
@@ -205,20 +213,20 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     const int s = it % S;
                     if (it >= S && !mbar_wait(&empty[s], ((it / S) - 1) & 1, &abort_flag, err))
                         break;
-                    uint8_t *kb = smem + s * TcStateSmem::kStage;
+                    uint8_t *kb = smem + s * Smem::kStage;
                     uint8_t *vb = kb + 2 * kBox;
-                    mbar_expect_tx(&full[s], TcStateSmem::kStage);
+                    mbar_expect_tx(&full[s], Smem::kStage);
                     const int t0 = c0 + st * kBlk;
-                    for (int x = 0; x < 2; ++x) {
+                    for (int x = 0; x < 2; ++x)
                         tma_load_3d(kb + x * kBox, &tm_k, &full[s], 128 * mh + 64 * x, t0, bh);
-                        tma_load_4d(vb + x * kBox, &tm_v, &full[s], 128 * nh + 64 * x, h, t0, b);
-                    }
+                    for (int x = 0; x < Smem::kVBoxes; ++x)
+                        tma_load_4d(vb + x * kBox, &tm_v, &full[s], DVC * nv + 64 * x, h, t0, b);
                 }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16(128, 128, 1, 1);
+            const uint32_t idesc = idesc_bf16(128, DVC, 1, 1);
             int it = 0;
             bool ok = true;
             for (int c = 0; ok && c < nchunks; ++c) {
@@ -231,7 +239,7 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     const int s = it % S;
                     if (!mbar_wait(&full[s], (it / S) & 1, &abort_flag, err)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t kb = smem_u32(smem + s * TcStateSmem::kStage);
+                    const uint32_t kb = smem_u32(smem + s * Smem::kStage);
                     const uint32_t vb = kb + 2 * kBox;
 #pragma unroll
                     for (int ks = 0; ks < kBlk / 16; ++ks) {
@@ -253,20 +261,20 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const int row = 32 * q4 + lane;
         const int krow = 128 * mh + row;                     // row of S
         const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
-        const size_t sbase = ((size_t)bh * kD + krow) * kD + 128 * nh;
-        float st[128];
+        const size_t sbase = ((size_t)bh * kD + krow) * kD + DVC * nv;
+        float st[DVC];
         if (state_in) {
             const float4 *src = reinterpret_cast<const float4 *>(state_in + sbase);
 #pragma unroll
-            for (int v4 = 0; v4 < 32; ++v4) {
+            for (int v4 = 0; v4 < DVC / 4; ++v4) {
                 const float4 f = src[v4];
                 st[4 * v4] = f.x; st[4 * v4 + 1] = f.y; st[4 * v4 + 2] = f.z; st[4 * v4 + 3] = f.w;
             }
         } else {
 #pragma unroll
-            for (int e = 0; e < 128; ++e) st[e] = 0.f;
+            for (int e = 0; e < DVC; ++e) st[e] = 0.f;
         }
-        store_bf16_row(s_prev + ((size_t)bh * nchunks * kD + krow) * kD + 128 * nh, st, 128);
+        store_bf16_row(s_prev + ((size_t)bh * nchunks * kD + krow) * kD + DVC * nv, st, DVC);
         for (int c = 0; c < nchunks; ++c) {
             const int buf = c & 1;
             if (!warp_wait(&acc_full[buf], (c >> 1) & 1, &abort_flag, err)) break;
@@ -274,7 +282,7 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const bool last = (c == nchunks - 1);
             const float decay = last ? hp.decay_last[h] : hp.decay_chunk[h];
 #pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {
+            for (int cb = 0; cb < DVC / 32; ++cb) {
                 uint32_t v[32];
                 tmem_ld32(tmem + 128 * buf + lane_off + 32 * cb, v);
                 tmem_wait_ld();
@@ -285,12 +293,12 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             tc_fence_before();
             mbar_arrive(&acc_free[buf]);                     // buffer free for chunk c + 2
             if (!last) {
-                store_bf16_row(s_prev + (((size_t)bh * nchunks + c + 1) * kD + krow) * kD + 128 * nh,
-                               st, 128);
+                store_bf16_row(s_prev + (((size_t)bh * nchunks + c + 1) * kD + krow) * kD + DVC * nv,
+                               st, DVC);
             } else if (state_out) {
                 float4 *o = reinterpret_cast<float4 *>(state_out + sbase);
 #pragma unroll
-                for (int v4 = 0; v4 < 32; ++v4)
+                for (int v4 = 0; v4 < DVC / 4; ++v4)
                     o[v4] = make_float4(st[4 * v4], st[4 * v4 + 1], st[4 * v4 + 2], st[4 * v4 + 3]);
             }
         }
@@ -379,7 +387,7 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     __shared__ uint64_t rfull[kSlots], rempty[kSlots];
-    __shared__ uint64_t s_full, s_read, p_full, p_free, o_full, o_free;
+    __shared__ uint64_t s_full, s_read, p_full[2], p_free[2], o_full, o_free;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
@@ -392,8 +400,10 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int s = 0; s < kSlots; ++s) { mbar_init(&rfull[s], 1); mbar_init(&rempty[s], 1); }
         mbar_init(&s_full, 1);
         mbar_init(&s_read, kEpiThreads);
-        mbar_init(&p_full, kEpiThreads);
-        mbar_init(&p_free, 1);
+        for (int x = 0; x < 2; ++x) {                    // one P half per warpgroup
+            mbar_init(&p_full[x], kEpiThreads / 2);
+            mbar_init(&p_free[x], 1);
+        }
         mbar_init(&o_full, 1);
         mbar_init(&o_free, kEpiThreads);
         abort_flag = 0;
@@ -533,17 +543,25 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 for (int t = 0; ok && t < m.nk; ++t) {
                     if (t + 1 < m.nk && !(ok = qk(t + 1))) break;
                     if (t < m.nsp && !(ok = qs_half(t))) break;
-                    if (!mbar_wait(&p_full, npv & 1, &abort_flag, err)) { ok = false; break; }
+                    // P V in two halves of 64 keys, each issued as soon as its
+                    // warpgroup has written that half of P
                     if (!(ok = take() && claim_o())) break;
                     const uint32_t base = sbase + (it % kSlots) * kSlot;
+                    for (int hx = 0; ok && hx < 2; ++hx) {
+                        if (!mbar_wait(&p_full[hx], npv & 1, &abort_flag, err)) { ok = false; break; }
+                        tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < kKeyTile / 16; ++kk)
-                        mma_bf16(tO, smem_desc_sw128(sP + (kk / 4) * kBox + (kk % 4) * 32, 16, 1024),
-                                 smem_desc_sw128(base + kk * 2048, kBox, 1024), id_pv,
-                                 (o_written || kk > 0) ? 1u : 0u);
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            const int kk = 4 * hx + k4;
+                            mma_bf16(tO, smem_desc_sw128(sP + hx * kBox + k4 * 32, 16, 1024),
+                                     smem_desc_sw128(base + kk * 2048, kBox, 1024), id_pv,
+                                     (o_written || kk > 0) ? 1u : 0u);
+                        }
+                        mma_commit(&p_free[hx]);
+                    }
+                    if (!ok) break;
                     o_written = true;
                     mma_commit(&rempty[it % kSlots]);
-                    mma_commit(&p_free);
                     ++it;
                     ++npv;
                 }
@@ -597,7 +615,7 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     }
                 }
                 // the previous tile's P must have been consumed by its P V
-                if (ntile >= 1 && !warp_wait(&p_free, (ntile - 1) & 1, &abort_flag, err)) { ok = false; break; }
+                if (ntile >= 1 && !warp_wait(&p_free[wg], (ntile - 1) & 1, &abort_flag, err)) { ok = false; break; }
                 // 64 keys of this row = eight 16-byte chunks of the 128-byte-swizzled box
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch)
@@ -605,7 +623,7 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         make_uint4(wv[4 * ch], wv[4 * ch + 1], wv[4 * ch + 2], wv[4 * ch + 3]);
                 fence_async_shared();
                 tc_fence_before();
-                mbar_arrive(&p_full);
+                mbar_arrive(&p_full[wg]);
             }
             // ring items of this work item: Qt, nk Kt tiles, nsp S_prev halves,
             // nk V tiles, then the gate/output tile
@@ -868,13 +886,28 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     {
-        const int smem = (int)TcStateSmem::kBytes;
-        e = cudaFuncSetAttribute(tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
+        // d_v columns per state CTA: 128 (four CTAs per sequence-head) unless
+        // eight CTAs per sequence-head still fit in one wave
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess)
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const bool narrow = BH * 8 <= sms;
         KernelTimer timer("tc_state", stream);
-        tc_state_kernel<<<BH * 4, kTcThreads, smem, stream>>>(tm_k, tm_v, hp, a.state_in,
-                                                             a.state_out, sp, H, n, C, nchunks,
-                                                             err);
+        if (narrow) {
+            const int smem = (int)TcStateSmem<64>::kBytes;
+            e = cudaFuncSetAttribute(tc_state_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     smem);
+            if (e != cudaSuccess) return e;
+            tc_state_kernel<64><<<BH * 8, kTcThreads, smem, stream>>>(
+                tm_k, tm_v, hp, a.state_in, a.state_out, sp, H, n, C, nchunks, err);
+        } else {
+            const int smem = (int)TcStateSmem<128>::kBytes;
+            e = cudaFuncSetAttribute(tc_state_kernel<128>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (e != cudaSuccess) return e;
+            tc_state_kernel<128><<<BH * 4, kTcThreads, smem, stream>>>(
+                tm_k, tm_v, hp, a.state_in, a.state_out, sp, H, n, C, nchunks, err);
+        }
         count_launch();
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
