@@ -10,7 +10,7 @@
 // row of its slab, so its 32 outputs are complete inside the CTA.  Each
 // thread owns a float4 of columns for dk/32 rows, issues all of its state
 // loads first, updates S in place and accumulates o; the 32 row lanes are
-// reduced in shared memory.
+// reduced by warp shuffles and then across the eight warps in shared memory.
 #include <algorithm>
 #include <cmath>
 
@@ -58,7 +58,7 @@ retention_step_kernel(const T *__restrict__ q, const T *__restrict__ k,
     const int rl = threadIdx.x / (kStepCols / 4);    // row lane
 
     __shared__ float qs[DK], ks[DK];
-    __shared__ float4 red[kStepLanes][kStepCols / 4];
+    __shared__ float4 red[kStepThreads / 32][kStepCols / 4];
 
     // Issue this thread's state loads first: they do not depend on q, k, v.
     float *S = state + (size_t)bh * DK * dv + col0 + cgi * 4;
@@ -105,13 +105,23 @@ retention_step_kernel(const T *__restrict__ q, const T *__restrict__ k,
         acc.z = fmaf(qr, t.z, acc.z);
         acc.w = fmaf(qr, t.w, acc.w);
     }
-    red[rl][cgi] = acc;
+    // Row lanes of one column group: four per warp (lanes cgi, cgi+8,
+    // cgi+16, cgi+24) meet by shuffles, then the eight warps in shared memory.
+#pragma unroll
+    for (int m = 8; m < 32; m <<= 1) {
+        acc.x += __shfl_xor_sync(0xffffffffu, acc.x, m);
+        acc.y += __shfl_xor_sync(0xffffffffu, acc.y, m);
+        acc.z += __shfl_xor_sync(0xffffffffu, acc.z, m);
+        acc.w += __shfl_xor_sync(0xffffffffu, acc.w, m);
+    }
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (lane < kStepCols / 4) red[warp][lane] = acc;
     __syncthreads();
     if (threadIdx.x < kStepCols / 4) {
         float4 t = red[0][threadIdx.x];
 #pragma unroll
-        for (int l = 1; l < kStepLanes; ++l) {
-            const float4 u = red[l][threadIdx.x];
+        for (int w = 1; w < kStepThreads / 32; ++w) {
+            const float4 u = red[w][threadIdx.x];
             t.x += u.x; t.y += u.y; t.z += u.z; t.w += u.w;
         }
         T *oh = out + (size_t)bh * dv + col0 + threadIdx.x * 4;
