@@ -220,9 +220,17 @@ RETNET_API retnet_status retnet_check_device_errors(retnet_stream_t stream);
 /* ---- Kernel timer (diagnostics; off by default) ----------------------
  * While enabled, every kernel this library launches is bracketed by CUDA
  * events on its own stream, and per-kernel totals accumulate until reset.
- * Adds a few microseconds of host work per launch; do not enable it while
- * capturing a CUDA graph. */
+ * Adds a few microseconds of host work per launch.  Launches made while the
+ * stream is being captured into a CUDA graph get event-record nodes in the
+ * graph: the next read or reset after the graph has run reports the times
+ * of its most recent replay.  Those events stay allocated (one pair per
+ * captured launch) for as long as the graph may run. */
 RETNET_API retnet_status retnet_profiler_enable(int on);
+/* Restricts the timer to the kernel named `name` (a NUL-terminated string
+ * the library copies; one of the names retnet_profiler_read reports), or
+ * lifts the restriction when `name` is NULL.  Timing one kernel keeps the
+ * events' own cost out of the other kernels' boundaries. */
+RETNET_API retnet_status retnet_profiler_select(const char *name);
 /* Drops accumulated totals (waits for pending events first). */
 RETNET_API retnet_status retnet_profiler_reset(void);
 /* Totals of the index-th kernel name (0-based, sorted by name): copies the

@@ -22,7 +22,8 @@ __all__ = [
     "RetnetError", "load_library", "retnet_status_string", "retnet_kernel_launch_count",
     "retnet_default_gammas", "retnet_xpos_rotate", "retnet_chunkwise_workspace_size",
     "retnet_retention_chunkwise", "retnet_retention_step", "retnet_groupnorm_swish",
-    "retnet_check_device_errors", "retnet_profiler_enable", "retnet_profiler_reset",
+    "retnet_check_device_errors", "retnet_profiler_enable", "retnet_profiler_select",
+    "retnet_profiler_reset",
     "retnet_profiler_read", "ALGO_AUTO", "ALGO_SIMT", "ALGO_TENSOR", "LIB_PATH",
 ]
 
@@ -76,6 +77,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "retnet_groupnorm_swish": (i, [vp, vp, vp, vp, f, ll, i, i, i, vp, vp]),
         "retnet_check_device_errors": (i, [vp]),
         "retnet_profiler_enable": (i, [i]),
+        "retnet_profiler_select": (i, [ctypes.c_char_p]),
         "retnet_profiler_reset": (i, []),
         "retnet_profiler_read": (i, [i, ctypes.c_char_p, sz, ctypes.POINTER(ctypes.c_double),
                                      ctypes.POINTER(ctypes.c_ulonglong)]),
@@ -277,6 +279,12 @@ def retnet_check_device_errors(device=None) -> None:
 def retnet_profiler_enable(on: bool = True) -> None:
     """Start/stop bracketing every library kernel launch with CUDA events."""
     _check("retnet_profiler_enable", load_library().retnet_profiler_enable(int(bool(on))))
+
+
+def retnet_profiler_select(name: Optional[str] = None) -> None:
+    """Times only the kernel `name` (None: every kernel)."""
+    _check("retnet_profiler_select",
+           load_library().retnet_profiler_select(None if name is None else name.encode()))
 
 
 def retnet_profiler_reset() -> None:

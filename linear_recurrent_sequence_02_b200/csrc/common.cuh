@@ -40,6 +40,7 @@ class KernelTimer {
     const char *name_ = nullptr;
     void *start_ = nullptr;
     void *stop_ = nullptr;
+    bool captured_ = false;
 };
 
 // ---------------------------------------------------------------- element IO

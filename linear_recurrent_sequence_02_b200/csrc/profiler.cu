@@ -15,6 +15,7 @@ namespace {
 struct Pending {
     std::string name;
     cudaEvent_t start, stop;
+    bool captured;       // recorded by a graph node: never handed out again
 };
 struct Totals {
     double ms = 0.0;
@@ -22,6 +23,7 @@ struct Totals {
 };
 std::mutex g_mu;
 bool g_enabled = false;
+std::string g_only;          // time only this kernel when not empty
 std::vector<cudaEvent_t> g_pool;
 std::vector<Pending> g_pending;
 std::map<std::string, Totals> g_totals;
@@ -51,29 +53,55 @@ cudaError_t resolve_pending() {
         } else if (first == cudaSuccess) {
             first = e;
         }
-        g_pool.push_back(p.start);
-        g_pool.push_back(p.stop);
+        if (!p.captured) {
+            g_pool.push_back(p.start);
+            g_pool.push_back(p.stop);
+        }
     }
     g_pending.clear();
     return first;
 }
 }  // namespace
 
+namespace {
+bool capturing(cudaStream_t s) {
+    cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+    return cudaStreamIsCapturing(s, &st) == cudaSuccess && st == cudaStreamCaptureStatusActive;
+}
+// Inside a capture an ordinary record only marks a dependency; an external
+// record becomes a node that takes a timestamp whenever the graph runs.
+void record(cudaEvent_t e, cudaStream_t s, bool captured) {
+    if (captured)
+        cudaEventRecordWithFlags(e, s, cudaEventRecordExternal);
+    else
+        cudaEventRecord(e, s);
+}
+}  // namespace
+
 KernelTimer::KernelTimer(const char *name, cudaStream_t stream) : stream_(stream) {
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_enabled) return;
-    start_ = take_event();
-    stop_ = take_event();
-    if (!start_ || !stop_) return;
+    if (!g_enabled || (!g_only.empty() && g_only != name)) return;
+    captured_ = capturing(stream_);
+    if (captured_) {                       // fresh events: the graph keeps using them
+        cudaEvent_t a = nullptr, b = nullptr;
+        if (cudaEventCreate(&a) != cudaSuccess) return;
+        if (cudaEventCreate(&b) != cudaSuccess) { cudaEventDestroy(a); return; }
+        start_ = a;
+        stop_ = b;
+    } else {
+        start_ = take_event();
+        stop_ = take_event();
+        if (!start_ || !stop_) return;
+    }
     name_ = name;
-    cudaEventRecord((cudaEvent_t)start_, stream_);
+    record((cudaEvent_t)start_, stream_, captured_);
 }
 
 KernelTimer::~KernelTimer() {
     if (!name_) return;
     std::lock_guard<std::mutex> lk(g_mu);
-    cudaEventRecord((cudaEvent_t)stop_, stream_);
-    g_pending.push_back({name_, (cudaEvent_t)start_, (cudaEvent_t)stop_});
+    record((cudaEvent_t)stop_, stream_, captured_);
+    g_pending.push_back({name_, (cudaEvent_t)start_, (cudaEvent_t)stop_, captured_});
 }
 
 }  // namespace retnet
@@ -85,6 +113,12 @@ extern "C" {
 retnet_status retnet_profiler_enable(int on) {
     std::lock_guard<std::mutex> lk(g_mu);
     g_enabled = on != 0;
+    return RETNET_OK;
+}
+
+retnet_status retnet_profiler_select(const char *name) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_only = name ? std::string(name) : std::string();
     return RETNET_OK;
 }
 
