@@ -614,7 +614,9 @@ def run_decode(args, w):
                   "kernel_event_us": eager_avg_s * 1e6, "clocks": clock_info,
                   "gpu_launches": launches_eager},
         "tokens_per_s": B * args.steps / (ms / 1e3),
-        "roofline": {"kernel": "retention_step", "bound": "hbm", "achieved": bytes_step / avg_s / 1e9,
+        "roofline": {"kernel": "retention_step", "bound": "hbm",
+                     "state_l2_resident": bytes_step <= 126e6,
+                     "achieved": bytes_step / avg_s / 1e9,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": bytes_step / avg_s / 1e9 / peaks["hbm_gbs"], "traffic": None,
                      "peak_source": src, "work_per_launch": bytes_step},
