@@ -55,13 +55,17 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
-def workload_config(w: wl.Workload, chunk: int) -> dict:
+def workload_config(w: wl.Workload, chunk: int, form: str = "chunkwise") -> dict:
+    if form == "parallel":
+        what = "parallel form over the whole sequence" + \
+            (" + GroupNorm/swish gate" if w.hidden else "") + " (prefill only, no state)"
+    else:
+        what = f"chunk {chunk}" + (" + GroupNorm/swish gate" if w.hidden else "") + \
+            " + 1 decode step"
     return {
-        "workload": f"{w.name}: B={w.batch} H={w.heads} n={w.seqlen} d={w.d} {w.dtype} "
-                    f"chunk {chunk}" + (" + GroupNorm/swish gate" if w.hidden else "") +
-                    " + 1 decode step",
+        "workload": f"{w.name}: B={w.batch} H={w.heads} n={w.seqlen} d={w.d} {w.dtype} " + what,
         "batch": w.batch, "heads": w.heads, "seqlen": w.seqlen, "dk": w.d, "dv": w.d,
-        "chunk": chunk, "gate": bool(w.hidden),
+        "chunk": chunk if form == "chunkwise" else None, "form": form, "gate": bool(w.hidden),
         "l2": "3 rotating input sets, each beyond 1/3 of the 126 MB L2",
     }
 
@@ -71,8 +75,8 @@ def workload_config(w: wl.Workload, chunk: int) -> dict:
 # source file at capture time; reported only while the source is unchanged.
 NCU_TRAFFIC = {
     "tc_output": {"source": "chunkwise_tc.cu",
-                  "sha256": "0a8c8dc8ace82e0f41ef1c1aeb552671cdf3ce694edbf6aa70602ad1bf4c33fb",
-                  "bytes": 160.73e6},
+                  "sha256": "e3333684a93e5d795a472e19407c04562ca5d6c6dbfb80a38e6d422e90ecbbf8",
+                  "bytes": 160.64e6},
 }
 
 
@@ -102,6 +106,11 @@ def output_kernel_flops_per_token_head(d: int, chunk: int) -> int:
 
 def state_kernel_flops_per_token_head(d: int) -> int:
     return 2 * d * d
+
+
+def parallel_flops_per_token_head(d: int, n: int) -> int:
+    # causal Q K^T and P V over the whole sequence: 2 d (n + 1) on average
+    return 2 * d * (n + 1)
 
 
 class ClockSampler:
@@ -288,14 +297,24 @@ def run_ours(args, w, chunk):
     y = torch.empty(B, n, H, d, dtype=tdt, device=dev)
     o = torch.empty(B, H, d, dtype=tdt, device=dev)
     state = torch.empty(B, H, d, d, dtype=torch.float32, device=dev)
-    wsb = rn.retnet_chunkwise_workspace_size(B, H, n, d, d, tdt, chunk, args.algo)
-    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device=dev)
+    par = args.form == "parallel"
+    wsb = rn.retnet_parallel_workspace_size(B, H, n, d, d, tdt) if par else \
+        rn.retnet_chunkwise_workspace_size(B, H, n, d, d, tdt, chunk, args.algo)
+
+    def prefill(qq, kk, vv, gg, st, out, wsp):
+        if par:
+            rn.retnet_retention_parallel(qq, kk, vv, gam, gate=gg, out=out, workspace=wsp)
+        else:
+            rn.retnet_retention_chunkwise(qq, kk, vv, gam, chunk, state_out=st, gate=gg, out=out,
+                                          workspace=wsp, algo=args.algo)
+
+    ws = rn.retnet_workspace(wsb, dev)
 
     def step(s):
         qq, kk, vv, gg, q1, k1, v1 = s
-        rn.retnet_retention_chunkwise(qq, kk, vv, gam, chunk, state_out=state, gate=gg, out=y,
-                                      workspace=ws, algo=args.algo)
-        rn.retnet_retention_step(q1, k1, v1, gam, state, n, out=o)
+        prefill(qq, kk, vv, gg, state, y, ws)
+        if not par:     # the parallel form leaves no state to decode from
+            rn.retnet_retention_step(q1, k1, v1, gam, state, n, out=o)
 
     torch.cuda.synchronize()
     for i in range(args.warmup):
@@ -367,7 +386,7 @@ def run_ours(args, w, chunk):
         ms = float(t.item())
     rn.retnet_check_device_errors(dev)
 
-    tokens_per_step = B * n + B
+    tokens_per_step = B * n + (0 if par else B)
     value = world * tokens_per_step * args.steps / (ms / 1e3)
 
     # ---- end to end through the public API with host buffers
@@ -375,8 +394,8 @@ def run_ours(args, w, chunk):
     # and copies y and the decode output back.  Copies run on their own
     # streams, double-buffered, so step i's upload overlaps step i-1's
     # compute and download (PCIe is full duplex).
-    h2d = sum(x.numel() * x.element_size() for x in host if x is not None)
-    d2h = y.numel() * y.element_size() + o.numel() * o.element_size()
+    h2d = sum(x.numel() * x.element_size() for x in host[:4 if par else 7] if x is not None)
+    d2h = y.numel() * y.element_size() + (0 if par else o.numel() * o.element_size())
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
     s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
     dsets = [[None if x is None else torch.empty_like(x, device=dev) for x in host]
@@ -386,7 +405,8 @@ def run_ours(args, w, chunk):
     yh = [torch.empty_like(y, device="cpu").pin_memory() for _ in range(2)]
     oh = [torch.empty_like(o, device="cpu").pin_memory() for _ in range(2)]
     st2 = [torch.empty_like(state) for _ in range(2)]
-    ws2 = [torch.empty_like(ws) for _ in range(2)]
+    ws2 = [rn.retnet_workspace(wsb, dev) for _ in range(2)]
+    nin = 4 if par else 7                 # the parallel form uploads no decode inputs
 
     def run_e2e(nsteps):
         in_ready = [torch.cuda.Event() for _ in range(nsteps)]
@@ -397,7 +417,7 @@ def run_ours(args, w, chunk):
             with torch.cuda.stream(s_in):
                 if i >= 2:
                     s_in.wait_event(done[i - 2])
-                for dst, src in zip(dsets[j], host):
+                for dst, src in zip(dsets[j][:nin], host[:nin]):
                     if src is not None:
                         dst.copy_(src, non_blocking=True)
                 in_ready[i].record(s_in)
@@ -406,14 +426,15 @@ def run_ours(args, w, chunk):
                 if i >= 2:
                     s_cmp.wait_event(out_done[i - 2])
                 qq, kk, vv, gg, q1, k1, v1 = dsets[j]
-                rn.retnet_retention_chunkwise(qq, kk, vv, gam, chunk, state_out=st2[j], gate=gg,
-                                              out=ys[j], workspace=ws2[j], algo=args.algo)
-                rn.retnet_retention_step(q1, k1, v1, gam, st2[j], n, out=os_[j])
+                prefill(qq, kk, vv, gg, st2[j], ys[j], ws2[j])
+                if not par:
+                    rn.retnet_retention_step(q1, k1, v1, gam, st2[j], n, out=os_[j])
                 done[i].record(s_cmp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(done[i])
                 yh[j].copy_(ys[j], non_blocking=True)
-                oh[j].copy_(os_[j], non_blocking=True)
+                if not par:
+                    oh[j].copy_(os_[j], non_blocking=True)
                 out_done[i].record(s_out)
         return out_done[-1]
 
@@ -450,7 +471,8 @@ def run_ours(args, w, chunk):
         avg_s = tot / cnt / 1e3
         th = B * n * H
         if dom in ("tc_output", "simt_output"):
-            flops = output_kernel_flops_per_token_head(d, chunk) * th
+            flops = (parallel_flops_per_token_head(d, n) if par else
+                     output_kernel_flops_per_token_head(d, chunk)) * th
             achieved = flops / avg_s / 1e12
             bound = "tensor" if dom.startswith("tc") else "alu"
             if bound == "tensor":
@@ -459,7 +481,7 @@ def run_ours(args, w, chunk):
                 peak = 148 * 128 * 2 * (peaks.get("sm_max_mhz", 1965.0) * 1e6) / 1e12
             roof = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak,
                     "unit": "TFLOP/s", "frac": achieved / peak,
-                    "traffic": measured_traffic(dom, w.name),
+                    "traffic": None if par else measured_traffic(dom, w.name),
                     "peak_source": peak_src, "work_per_launch": flops}
         elif dom in ("tc_state", "simt_state"):
             flops = state_kernel_flops_per_token_head(d) * th
@@ -481,7 +503,8 @@ def run_ours(args, w, chunk):
     pre_ms = ms / max(args.steps, 1) - dec_ms
     prefill = None
     if pre_ms > 0:
-        alg = algorithmic_flops_per_token_head(d, chunk) * B * n * H
+        alg = (parallel_flops_per_token_head(d, n) if par else
+               algorithmic_flops_per_token_head(d, chunk)) * B * n * H
         prefill = {"tokens_per_s": B * n / (pre_ms / 1e3),
                    "ms": pre_ms,
                    "tflops_algorithmic": alg / (pre_ms / 1e3) / 1e12,
@@ -497,7 +520,7 @@ def run_ours(args, w, chunk):
                   peaks["hbm_gbs"], "note": "state just written by the prefill (L2-warm)"}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not par:
         cpu = cpu_baseline(w, chunk)
 
     if rank == 0:
@@ -505,8 +528,8 @@ def run_ours(args, w, chunk):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": w.dtype, "data": "synthetic", "config": workload_config(w, chunk),
-            "algo": args.algo, "roofline": roof, "prefill": prefill, "decode": decode,
+            "dtype": w.dtype, "data": "synthetic", "config": workload_config(w, chunk, args.form),
+            "algo": "tensor" if par else args.algo, "roofline": roof, "prefill": prefill, "decode": decode,
             "kernels": kernels_json, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
@@ -639,6 +662,8 @@ def main():
     ap.add_argument("--algo", choices=["auto", "simt", "tensor"], default="auto")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--form", choices=["chunkwise", "parallel"], default="chunkwise",
+                    help="prefill form; 'parallel' times the parallel form alone (no decode)")
     args = ap.parse_args()
     w = wl.WORKLOADS[args.workload]
     chunk = args.chunk or w.chunk

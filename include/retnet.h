@@ -157,6 +157,25 @@ RETNET_API retnet_status retnet_retention_chunkwise(const void *q, const void *k
                                          void *workspace, size_t workspace_bytes,
                                          retnet_stream_t stream);
 
+/* ---- Parallel form ------------------------------------------------------
+ * The parallel (training) form over the whole sequence ("Summary": the
+ * parallel representation computes all tokens at once):
+ *   out[b, t, h, :] = sum_{m <= t} gamma_h^(t-m) (R q_t . R k_m) v_m,
+ * then swish(G) (.) GroupNorm when `gate` is given, with R the rotation of
+ * retnet_retention_chunkwise.  O(n^2) work per sequence-head; the initial
+ * state is zero and no state is returned.  Tensor-core kernels only: bf16,
+ * dk = dv = 256, and every decay must satisfy 128 * log2(1/gamma) <= 100
+ * (gamma >= 0.58); other requests return UNSUPPORTED.  Arguments as for
+ * retnet_retention_chunkwise; workspace: retnet_parallel_workspace_size()
+ * bytes, 1024-byte aligned.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+RETNET_API retnet_status retnet_parallel_workspace_size(const retnet_shape *shape, size_t *bytes);
+RETNET_API retnet_status retnet_retention_parallel(const void *q, const void *k, const void *v,
+                                        const float *gammas, void *out,
+                                        const retnet_shape *shape, long long pos0, int rotate,
+                                        const retnet_gate *gate, void *workspace,
+                                        size_t workspace_bytes, retnet_stream_t stream);
+
 /* ---- Prefill without any allocation ---------------------------------
  * No counterpart on the pages: an addition for callers that cannot
  * allocate device memory at run time -- for example a plugin inside a

@@ -21,7 +21,9 @@ import torch
 __all__ = [
     "RetnetError", "load_library", "retnet_status_string", "retnet_kernel_launch_count",
     "retnet_default_gammas", "retnet_xpos_rotate", "retnet_chunkwise_workspace_size",
-    "retnet_retention_chunkwise", "retnet_retention_step", "retnet_groupnorm_swish",
+    "retnet_retention_chunkwise", "retnet_parallel_workspace_size", "retnet_retention_parallel",
+    "retnet_workspace",
+    "retnet_retention_step", "retnet_groupnorm_swish",
     "retnet_check_device_errors", "retnet_profiler_enable", "retnet_profiler_select",
     "retnet_profiler_reset",
     "retnet_profiler_read", "ALGO_AUTO", "ALGO_SIMT", "ALGO_TENSOR", "LIB_PATH",
@@ -73,6 +75,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "retnet_chunkwise_workspace_size": (i, [ctypes.POINTER(_Shape), i, i, ctypes.POINTER(sz)]),
         "retnet_retention_chunkwise": (i, [vp, vp, vp, vp, i, vp, ctypes.POINTER(_Shape), ll, i,
                                            vp, vp, ctypes.POINTER(_Gate), i, vp, sz, vp]),
+        "retnet_parallel_workspace_size": (i, [ctypes.POINTER(_Shape), ctypes.POINTER(sz)]),
+        "retnet_retention_parallel": (i, [vp, vp, vp, vp, vp, ctypes.POINTER(_Shape), ll, i,
+                                          ctypes.POINTER(_Gate), vp, sz, vp]),
         "retnet_retention_step": (i, [vp, vp, vp, vp, vp, vp, i, i, i, i, i, ll, i, vp]),
         "retnet_groupnorm_swish": (i, [vp, vp, vp, vp, f, ll, i, i, i, vp, vp]),
         "retnet_check_device_errors": (i, [vp]),
@@ -164,6 +169,19 @@ def retnet_xpos_rotate(x: torch.Tensor, pos0: int = 0, out: Optional[torch.Tenso
     return out
 
 
+WORKSPACE_ALIGN = 1024
+
+
+def retnet_workspace(nbytes: int, device) -> torch.Tensor:
+    """A uint8 device buffer of at least `nbytes` whose first byte is
+    1024-byte aligned, as the tensor-core path requires.  The caching
+    allocator only guarantees 512-byte alignment for sub-allocations, so
+    this over-allocates by one alignment unit and returns an aligned view."""
+    buf = torch.empty(max(int(nbytes), 1) + WORKSPACE_ALIGN, dtype=torch.uint8, device=device)
+    off = (-buf.data_ptr()) % WORKSPACE_ALIGN
+    return buf[off:off + max(int(nbytes), 1)]
+
+
 def retnet_chunkwise_workspace_size(batch: int, heads: int, seqlen: int, dk: int, dv: int,
                                     dtype: torch.dtype, chunk: int, algo="auto") -> int:
     shape = _Shape(batch, heads, seqlen, dk, dv, BF16 if dtype == torch.bfloat16 else F32)
@@ -207,7 +225,7 @@ def retnet_retention_chunkwise(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor
     a = _ALGOS[algo]
     need = retnet_chunkwise_workspace_size(B, H, n, dk, dv, q.dtype, chunk, a)
     if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+        workspace = retnet_workspace(need, q.device)
     else:
         _dev(workspace, "workspace", torch.uint8)
     shape = _Shape(B, H, n, dk, dv, _dtype_code(q))
@@ -222,6 +240,55 @@ def retnet_retention_chunkwise(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor
             None if g is None else ctypes.byref(g), a, _ptr(workspace),
             workspace.numel(), _stream(q))
     _check("retnet_retention_chunkwise", st)
+    return out
+
+
+def retnet_parallel_workspace_size(batch: int, heads: int, seqlen: int, dk: int, dv: int,
+                                   dtype: torch.dtype) -> int:
+    shape = _Shape(batch, heads, seqlen, dk, dv, BF16 if dtype == torch.bfloat16 else F32)
+    n = ctypes.c_size_t(0)
+    _check("retnet_parallel_workspace_size",
+           load_library().retnet_parallel_workspace_size(ctypes.byref(shape), ctypes.byref(n)))
+    return int(n.value)
+
+
+def retnet_retention_parallel(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                              gammas: Sequence[float], *, pos0: int = 0, rotate: bool = True,
+                              gate: Optional[torch.Tensor] = None,
+                              weight: Optional[torch.Tensor] = None,
+                              bias: Optional[torch.Tensor] = None, eps: float = 1e-5,
+                              out: Optional[torch.Tensor] = None,
+                              workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Parallel form over the whole sequence (zero initial state).  Returns
+    out: O, or swish(gate) * GroupNorm(O) if gate is given."""
+    _dev(q, "q")
+    if q.dim() != 4:
+        raise ValueError("q must be [batch, seqlen, heads, dk]")
+    B, n, H, dk = q.shape
+    dv = v.shape[-1]
+    _dev(k, "k", q.dtype, (B, n, H, dk))
+    _dev(v, "v", q.dtype, (B, n, H, dv))
+    _dev(gate, "gate", q.dtype, (B, n, H, dv))
+    _dev(weight, "weight", torch.float32, (H * dv,))
+    _dev(bias, "bias", torch.float32, (H * dv,))
+    out = torch.empty((B, n, H, dv), dtype=q.dtype, device=q.device) if out is None else \
+        _dev(out, "out", q.dtype, (B, n, H, dv))
+    need = retnet_parallel_workspace_size(B, H, n, dk, dv, q.dtype)
+    if workspace is None:
+        workspace = retnet_workspace(need, q.device)
+    else:
+        _dev(workspace, "workspace", torch.uint8)
+    shape = _Shape(B, H, n, dk, dv, _dtype_code(q))
+    g = None
+    if gate is not None:
+        g = _Gate(gate.data_ptr(), None if weight is None else weight.data_ptr(),
+                  None if bias is None else bias.data_ptr(), float(eps))
+    with torch.cuda.device(q.device):
+        st = load_library().retnet_retention_parallel(
+            _ptr(q), _ptr(k), _ptr(v), _gammas(gammas, H), _ptr(out), ctypes.byref(shape),
+            int(pos0), int(bool(rotate)), None if g is None else ctypes.byref(g), _ptr(workspace),
+            workspace.numel(), _stream(q))
+    _check("retnet_retention_parallel", st)
     return out
 
 

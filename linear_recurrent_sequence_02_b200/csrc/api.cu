@@ -21,6 +21,8 @@ unsigned *device_error_word() {
 }
 
 static bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+// Block length of the parallel form's decay fold (one 128-row tile).
+constexpr int kParallelFoldBlock = 128;
 static bool head_dim_ok(int d) { return d == 64 || d == 128 || d == 256; }
 static bool dtype_ok(retnet_dtype t) { return t == RETNET_F32 || t == RETNET_BF16; }
 static size_t elem_size(retnet_dtype t) { return t == RETNET_BF16 ? 2 : 4; }
@@ -169,6 +171,54 @@ retnet_status retnet_retention_chunkwise(const void *q, const void *k, const voi
     } else {
         RETNET_CUDA_TRY(launch_chunkwise_simt(a, (cudaStream_t)stream));
     }
+    return RETNET_OK;
+}
+
+retnet_status retnet_parallel_workspace_size(const retnet_shape *shape, size_t *bytes) {
+    if (!bytes) return RETNET_ERR_INVALID_ARG;
+    retnet_status st = check_shape(shape, kParallelFoldBlock);
+    if (st != RETNET_OK) return st;
+    if (!tc_shape_ok(shape->dk, shape->dv, shape->dtype, kParallelFoldBlock))
+        return RETNET_ERR_UNSUPPORTED;
+    *bytes = tc_parallel_workspace_bytes(shape->batch, shape->heads, shape->seqlen);
+    return RETNET_OK;
+}
+
+retnet_status retnet_retention_parallel(const void *q, const void *k, const void *v,
+                                        const float *gammas, void *out,
+                                        const retnet_shape *shape, long long pos0, int rotate,
+                                        const retnet_gate *gate, void *workspace,
+                                        size_t workspace_bytes, retnet_stream_t stream) {
+    retnet_status st = check_shape(shape, kParallelFoldBlock);
+    if (st != RETNET_OK) return st;
+    if (pos0 < 0 || (rotate != 0 && rotate != 1)) return RETNET_ERR_INVALID_ARG;
+    ChunkwiseArgs a;
+    st = load_gammas(gammas, shape->heads, &a.gam);
+    if (st != RETNET_OK) return st;
+    const long long tokens = (long long)shape->batch * shape->seqlen;
+    if (tokens > 0) {
+        if (!q || !k || !v || !out) return RETNET_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+            return RETNET_ERR_INVALID_ARG;
+    }
+    if (gate) {
+        if (tokens > 0 && (!gate->g || !aligned16(gate->g))) return RETNET_ERR_INVALID_ARG;
+        if (!(gate->eps >= 0.f)) return RETNET_ERR_INVALID_ARG;
+    }
+    if (!tc_shape_ok(shape->dk, shape->dv, shape->dtype, kParallelFoldBlock) ||
+        !tc_gammas_ok(kParallelFoldBlock, gammas, shape->heads))
+        return RETNET_ERR_UNSUPPORTED;
+    const size_t need = tc_parallel_workspace_bytes(shape->batch, shape->heads, shape->seqlen);
+    if (need > 0 && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 1023u)))
+        return RETNET_ERR_WORKSPACE;
+    if (tokens == 0) return RETNET_OK;
+    a.q = q; a.k = k; a.v = v; a.out = out;
+    a.state_in = nullptr; a.state_out = nullptr; a.gate = gate;
+    a.batch = shape->batch; a.heads = shape->heads; a.seqlen = shape->seqlen;
+    a.dk = shape->dk; a.dv = shape->dv; a.chunk = kParallelFoldBlock; a.dtype = shape->dtype;
+    a.pos0 = pos0; a.rotate = rotate; a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
+    RETNET_CUDA_TRY(launch_chunkwise_tc(a, gammas, (cudaStream_t)stream, true));
     return RETNET_OK;
 }
 

@@ -349,6 +349,11 @@ struct TcOutArgs {
     const float *gn_weight, *gn_bias;
     float eps;
     unsigned *err;
+    // Parallel form: the whole sequence is one "chunk" with Qt, Kt folded per
+    // 128-token block, so key tile t of row block r still needs the factor
+    // g^(128 (r - t)), applied in the mask pass.
+    int parallel;
+    float log2g[kMaxHeads];
 };
 
 struct TcItem {
@@ -596,7 +601,14 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 mbar_arrive(&s_read);                           // S may be overwritten now
                 const int j0 = t * kKeyTile + 64 * wg;          // first key of this half tile
                 uint32_t wv[32];
-                if (j0 + 63 <= lrow) {                          // every key at or before the row
+                if (a.parallel && t < m.r) {                    // a whole earlier block
+                    const float tf = exp2f((float)(kKeyTile * (m.r - t)) * a.log2g[m.h]);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        wv[e] = pack_bf16x2(tf * __uint_as_float(v0[2 * e]), tf * __uint_as_float(v0[2 * e + 1]));
+                        wv[16 + e] = pack_bf16x2(tf * __uint_as_float(v1[2 * e]), tf * __uint_as_float(v1[2 * e + 1]));
+                    }
+                } else if (j0 + 63 <= lrow) {                   // every key at or before the row
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         wv[e] = pack_bf16x2(__uint_as_float(v0[2 * e]), __uint_as_float(v0[2 * e + 1]));
@@ -807,10 +819,22 @@ size_t tc_workspace_bytes(int batch, int heads, int seqlen, int chunk) {
     return tc_layout(batch, heads, seqlen, chunk).total;
 }
 
-cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cudaStream_t stream) {
-    const int n = a.seqlen, H = a.heads, B = a.batch, C = a.chunk;
+// The parallel form runs the output pass over the whole sequence as one
+// block of whole 128-row tiles.
+static int parallel_span(int n) { return (n + kBlk - 1) / kBlk * kBlk; }
+
+size_t tc_parallel_workspace_bytes(int batch, int heads, int seqlen) {
+    return seqlen > 0 ? tc_layout(batch, heads, seqlen, parallel_span(seqlen)).total : 0;
+}
+
+cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cudaStream_t stream,
+                                bool parallel) {
+    const int n = a.seqlen, H = a.heads, B = a.batch;
+    // parallel form: one chunk spanning the sequence, decay folded per 128-row block
+    const int C = parallel ? parallel_span(n) : a.chunk;
+    const int fold = parallel ? kBlk : a.chunk;
     const int BH = B * H;
-    if (BH == 0) return cudaSuccess;
+    if (BH == 0 || (parallel && n == 0)) return cudaSuccess;
     if (n == 0) {                                   // nothing to scan: state passes through
         if (!a.state_out) return cudaSuccess;
         size_t bytes = (size_t)BH * kD * kD * sizeof(float);
@@ -880,12 +904,12 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
         for (int h = 0; h < kMaxHeads; ++h) pp.log2g[h] = hp.log2g[h];
         KernelTimer timer("tc_prep", stream);
         tc_prep_kernel<<<n, 256, 0, stream>>>((const __nv_bfloat16 *)a.q,
-                                             (const __nv_bfloat16 *)a.k, pp, qt, kt, B, H, n, C,
+                                             (const __nv_bfloat16 *)a.k, pp, qt, kt, B, H, n, fold,
                                              a.pos0, a.rotate);
         count_launch();
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    {
+    if (!parallel) {
         // d_v columns per state CTA: 128 (four CTAs per sequence-head) unless
         // eight CTAs per sequence-head still fit in one wave
         int dev = 0, sms = 148;
@@ -921,6 +945,8 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
         oa.eps = a.gate ? a.gate->eps : 0.f;
         oa.err = err;
         oa.items = BH * nchunks * oa.rblocks;
+        oa.parallel = parallel ? 1 : 0;
+        for (int h = 0; h < kMaxHeads; ++h) oa.log2g[h] = hp.log2g[h];
         const int smem = (int)TcOutSmem::kBytes;
         e = cudaFuncSetAttribute(tc_output_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  smem);

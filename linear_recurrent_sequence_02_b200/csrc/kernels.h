@@ -48,6 +48,10 @@ bool tc_shape_ok(int dk, int dv, retnet_dtype dtype, int chunk);
 // Every head's decay admits the decay fold: gamma > 0 and chunk*log2(1/gamma) <= 100.
 bool tc_gammas_ok(int chunk, const float *gammas, int heads);
 size_t tc_workspace_bytes(int batch, int heads, int seqlen, int chunk);
-cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cudaStream_t stream);
+// parallel: the parallel form over the whole sequence (a.chunk, state_in and
+// state_out unused; decays must pass tc_gammas_ok at chunk 128).
+cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cudaStream_t stream,
+                                bool parallel = false);
+size_t tc_parallel_workspace_bytes(int batch, int heads, int seqlen);
 
 }  // namespace retnet

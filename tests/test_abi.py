@@ -138,3 +138,35 @@ def test_binding_refuses_cpu_tensors(lib):
     x = torch.zeros(1, 4, 2, 8)
     with pytest.raises(ValueError):
         rn.retnet_xpos_rotate(x)
+
+
+def _parallel(lib, q=1024, k=1024, v=1024, out=1024, gam=(0.9,) * 4, shape=None, pos0=0,
+              rotate=1, ws=1024, wsb=1 << 40):
+    s = shape or _shape(dk=256, dv=256, dt=1)
+    g = None if gam is None else (ctypes.c_float * len(gam))(*gam)
+    P = ctypes.c_void_p
+    return lib.retnet_retention_parallel(P(q), P(k), P(v), g, P(out), ctypes.byref(s), pos0,
+                                         rotate, None, P(ws), wsb, None)
+
+
+def test_parallel_form_rejects_before_launch(lib):
+    n = ctypes.c_size_t(0)
+    s = _shape(dk=256, dv=256, dt=1)
+    assert lib.retnet_parallel_workspace_size(ctypes.byref(s), ctypes.byref(n)) == 0
+    assert n.value > 0
+    f32 = _shape(dk=256, dv=256, dt=0)
+    assert lib.retnet_parallel_workspace_size(ctypes.byref(f32), ctypes.byref(n)) == 2
+    assert lib.retnet_parallel_workspace_size(None, ctypes.byref(n)) == 1
+    # fake, aligned, never-dereferenced addresses: every case fails validation
+    assert _parallel(lib, q=None) == 1
+    assert _parallel(lib, gam=None) == 1
+    assert _parallel(lib, gam=(0.9, 0.9, 0.9, 1.5)) == 1
+    assert _parallel(lib, pos0=-1) == 1
+    assert _parallel(lib, rotate=3) == 1
+    assert _parallel(lib, shape=_shape(dk=64, dv=64, dt=1)) == 2   # tensor path only: d = 256
+    assert _parallel(lib, gam=(0.5, 0.9, 0.9, 0.9)) == 2           # decay too fast to fold
+    assert _parallel(lib, ws=None) == 5
+    assert _parallel(lib, wsb=16) == 5
+    assert _parallel(lib, ws=1024 + 256) == 5                      # not 1024-byte aligned
+    assert _parallel(lib, q=None, k=None, v=None, out=None, shape=_shape(B=0, dk=256, dv=256,
+                                                                         dt=1)) == 0

@@ -34,7 +34,7 @@ def test_captured_prefill_and_step_replay_bit_exact(rn):
     qd, kd, vd = (torch.from_numpy(rng.standard_normal((B, H, d)).astype(np.float32) / 16)
                   .to(torch.bfloat16).cuda() for _ in range(3))
     wsb = rn.retnet_chunkwise_workspace_size(B, H, n, d, d, torch.bfloat16, 256, "auto")
-    ws = torch.empty(max(wsb, 1), dtype=torch.uint8, device="cuda")
+    ws = rn.retnet_workspace(wsb, "cuda")
 
     def run(y, st, o):
         rn.retnet_retention_chunkwise(q, k, v, gam, 256, state_out=st, gate=g, out=y,
