@@ -104,6 +104,16 @@ RETNET_API const char *retnet_status_string(retnet_status status);
  * devices, all threads).  Used to count launches inside a timed region. */
 RETNET_API unsigned long long retnet_kernel_launch_count(void);
 
+/* Launch overlap (process-wide, on by default).  When enabled, the
+ * tensor-core prefill kernels and the decode step are launched with
+ * programmatic stream serialisation: each is launched as the CTAs of the
+ * kernel before it on the stream exit, so its launch and set-up (barriers,
+ * tensor memory, descriptor prefetch) overlap that kernel's tail, and it
+ * waits for that kernel to complete before touching global memory.
+ * Results are identical either way; only the gaps between kernels change.
+ * enable: 0 or 1, else INVALID_ARG. */
+RETNET_API retnet_status retnet_set_launch_overlap(int enable);
+
 /* Per-head decay constants gamma_h = 1 - 2^(-5-h), h = 0..heads-1, written
  * to the HOST array gammas[heads] ("Key points": gamma = 1 - 2^(-5-i)).
  * Errors: INVALID_ARG if gammas is NULL or heads is outside 1..256. */

@@ -20,6 +20,7 @@ import torch
 
 __all__ = [
     "RetnetError", "load_library", "retnet_status_string", "retnet_kernel_launch_count",
+    "retnet_set_launch_overlap",
     "retnet_default_gammas", "retnet_xpos_rotate", "retnet_chunkwise_workspace_size",
     "retnet_retention_chunkwise", "retnet_parallel_workspace_size", "retnet_retention_parallel",
     "retnet_workspace",
@@ -70,6 +71,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     sigs = {
         "retnet_status_string": (ctypes.c_char_p, [i]),
         "retnet_kernel_launch_count": (ctypes.c_ulonglong, []),
+        "retnet_set_launch_overlap": (i, [i]),
         "retnet_default_gammas": (i, [i, vp]),
         "retnet_xpos_rotate": (i, [vp, vp, i, i, i, i, i, ll, vp]),
         "retnet_chunkwise_workspace_size": (i, [ctypes.POINTER(_Shape), i, i, ctypes.POINTER(sz)]),
@@ -106,6 +108,11 @@ def retnet_status_string(status: int) -> str:
 
 def retnet_kernel_launch_count() -> int:
     return int(load_library().retnet_kernel_launch_count())
+
+
+def retnet_set_launch_overlap(enable: bool) -> None:
+    """Programmatic launch overlap of the hot kernels (on by default)."""
+    _check("retnet_set_launch_overlap", load_library().retnet_set_launch_overlap(int(bool(enable))))
 
 
 def retnet_default_gammas(heads: int) -> list:

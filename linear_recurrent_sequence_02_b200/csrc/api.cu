@@ -12,6 +12,9 @@ namespace retnet {
 static std::atomic<unsigned long long> g_launches{0};
 void count_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
+static std::atomic<bool> g_overlap{true};
+bool launch_overlap_enabled() { return g_overlap.load(std::memory_order_relaxed); }
+
 __device__ unsigned g_device_error = 0u;
 
 unsigned *device_error_word() {
@@ -83,6 +86,12 @@ const char *retnet_status_string(retnet_status status) {
 
 unsigned long long retnet_kernel_launch_count(void) {
     return g_launches.load(std::memory_order_relaxed);
+}
+
+retnet_status retnet_set_launch_overlap(int enable) {
+    if (enable != 0 && enable != 1) return RETNET_ERR_INVALID_ARG;
+    g_overlap.store(enable == 1, std::memory_order_relaxed);
+    return RETNET_OK;
 }
 
 retnet_status retnet_default_gammas(int heads, float *gammas) {

@@ -85,6 +85,7 @@ tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
             }
         }
     };
+    grid_dependency_wait();                         // q, k may come from the kernel before
     load_round(threadIdx.x);
     if (threadIdx.x < kD / 2) {
         float2 v = make_float2(1.f, 0.f);
@@ -196,15 +197,18 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         tmem_alloc(&tmem_slot, 256);
         tmem_relinquish();
     }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_slot;
+    grid_dependency_wait();                             // Kt from the prep kernel
 
     if (warp == 0) {
         if (lane == 0) {
-            tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
             int it = 0;
             for (int c = 0; c < nchunks && !abort_flag; ++c) {
                 const int c0 = c * chunk;
@@ -418,17 +422,20 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tmem_alloc(&tmem_slot, 512);
         tmem_relinquish();
     }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v); tma_prefetch_desc(&tm_s);
+        if (a.has_gate) tma_prefetch_desc(&tm_g);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_slot;
     const uint32_t tO = tmem, tQ = tmem + 256, tS = tmem + 384;
+    grid_dependency_wait();                             // Qt, Kt, S_prev from the kernels before
 
     if (warp == 0) {
         if (lane == 0) {
-            tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v); tma_prefetch_desc(&tm_s);
-            if (a.has_gate) tma_prefetch_desc(&tm_g);
             int it = 0;
             bool ok = true;
             auto acquire = [&]() -> bool {
@@ -903,11 +910,11 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
         for (int j = 0; j < kD / 2; ++j) pp.theta[j] = std::pow(10000.0, -2.0 * j / kD);
         for (int h = 0; h < kMaxHeads; ++h) pp.log2g[h] = hp.log2g[h];
         KernelTimer timer("tc_prep", stream);
-        tc_prep_kernel<<<n, 256, 0, stream>>>((const __nv_bfloat16 *)a.q,
-                                             (const __nv_bfloat16 *)a.k, pp, qt, kt, B, H, n, fold,
-                                             a.pos0, a.rotate);
+        e = launch_overlapped(tc_prep_kernel, dim3(n), dim3(256), 0, stream,
+                              (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, pp, qt, kt,
+                              B, H, n, fold, a.pos0, a.rotate);
         count_launch();
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (e != cudaSuccess) return e;
     }
     if (!parallel) {
         // d_v columns per state CTA: 128 (four CTAs per sequence-head) unless
@@ -922,18 +929,20 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
             e = cudaFuncSetAttribute(tc_state_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      smem);
             if (e != cudaSuccess) return e;
-            tc_state_kernel<64><<<BH * 8, kTcThreads, smem, stream>>>(
-                tm_k, tm_v, hp, a.state_in, a.state_out, sp, H, n, C, nchunks, err);
+            e = launch_overlapped(tc_state_kernel<64>, dim3(BH * 8), dim3(kTcThreads), smem, stream,
+                                  tm_k, tm_v, hp, a.state_in, a.state_out, sp, H, n, C, nchunks,
+                                  err);
         } else {
             const int smem = (int)TcStateSmem<128>::kBytes;
             e = cudaFuncSetAttribute(tc_state_kernel<128>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
             if (e != cudaSuccess) return e;
-            tc_state_kernel<128><<<BH * 4, kTcThreads, smem, stream>>>(
-                tm_k, tm_v, hp, a.state_in, a.state_out, sp, H, n, C, nchunks, err);
+            e = launch_overlapped(tc_state_kernel<128>, dim3(BH * 4), dim3(kTcThreads), smem,
+                                  stream, tm_k, tm_v, hp, a.state_in, a.state_out, sp, H, n, C,
+                                  nchunks, err);
         }
         count_launch();
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (e != cudaSuccess) return e;
     }
     {
         TcOutArgs oa;
@@ -956,10 +965,10 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         const unsigned grid = (unsigned)std::min(oa.items, sms);
         KernelTimer timer("tc_output", stream);
-        tc_output_kernel<<<grid, kOutThreads, smem, stream>>>(tm_q, tm_k, tm_v, tm_s, tm_g, tm_out,
-                                                             oa);
+        e = launch_overlapped(tc_output_kernel, dim3(grid), dim3(kOutThreads), smem, stream, tm_q,
+                              tm_k, tm_v, tm_s, tm_g, tm_out, oa);
         count_launch();
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
 }

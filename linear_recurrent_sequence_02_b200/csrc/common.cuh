@@ -43,6 +43,43 @@ class KernelTimer {
     bool captured_ = false;
 };
 
+// ------------------------------------------------------ programmatic launch
+// The kernels of one call, and of consecutive calls, follow each other on a
+// stream.  Launched with programmatic stream serialisation, a kernel is
+// launched as its predecessor's CTAs exit rather than after the whole grid
+// has drained, so the launch gap and its set-up (barriers, TMEM allocation,
+// descriptor prefetch) overlap the predecessor's tail.  Each such kernel
+// calls grid_dependency_wait() before its first global-memory access: it
+// returns once the predecessor grid has completed and its writes are
+// visible (at once when the kernel was launched normally).  No kernel
+// triggers its successor early (griddepcontrol.launch_dependents): waiting
+// CTAs of the successor then sit on SMs that the rest of this grid needs,
+// which measured slower.  Since every CTA passes its wait before it exits,
+// a kernel never starts before its predecessors' predecessors completed.
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Host: whether launches carry the programmatic-serialisation attribute
+// (retnet_set_launch_overlap; on by default).
+bool launch_overlap_enabled();
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_overlapped(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = launch_overlap_enabled() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ---------------------------------------------------------------- element IO
 template <typename T> __device__ __forceinline__ float to_f32(T x);
 template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }

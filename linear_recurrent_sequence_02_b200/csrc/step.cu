@@ -60,6 +60,7 @@ retention_step_kernel(const T *__restrict__ q, const T *__restrict__ k,
     __shared__ float qs[DK], ks[DK];
     __shared__ float4 red[kStepThreads / 32][kStepCols / 4];
 
+    grid_dependency_wait();          // the state may come from the kernel before
     // Issue this thread's state loads first: they do not depend on q, k, v.
     float *S = state + (size_t)bh * DK * dv + col0 + cgi * 4;
     float4 s[RPL];
@@ -142,27 +143,27 @@ static cudaError_t launch_step_t(const void *q, const void *k, const void *v,
     // grid.y holds (sequence, head) rows; more than 65535 of them take several launches
     for (long long bh0 = 0; bh0 < bh_total; bh0 += 65535) {
         const dim3 grid((unsigned)(dv / kStepCols), (unsigned)std::min(65535LL, bh_total - bh0));
+        cudaError_t e = cudaSuccess;
         switch (dk) {
             case 64:
-                retention_step_kernel<T, 64><<<grid, kStepThreads, 0, stream>>>(
-                    (const T *)q, (const T *)k, (const T *)v, gam, rot, state, (T *)out, (int)bh0,
-                    heads, dv, rotate);
+                e = launch_overlapped(retention_step_kernel<T, 64>, grid, dim3(kStepThreads), 0,
+                                      stream, (const T *)q, (const T *)k, (const T *)v, gam, rot,
+                                      state, (T *)out, (int)bh0, heads, dv, rotate);
                 break;
             case 128:
-                retention_step_kernel<T, 128><<<grid, kStepThreads, 0, stream>>>(
-                    (const T *)q, (const T *)k, (const T *)v, gam, rot, state, (T *)out, (int)bh0,
-                    heads, dv, rotate);
+                e = launch_overlapped(retention_step_kernel<T, 128>, grid, dim3(kStepThreads), 0,
+                                      stream, (const T *)q, (const T *)k, (const T *)v, gam, rot,
+                                      state, (T *)out, (int)bh0, heads, dv, rotate);
                 break;
             case 256:
-                retention_step_kernel<T, 256><<<grid, kStepThreads, 0, stream>>>(
-                    (const T *)q, (const T *)k, (const T *)v, gam, rot, state, (T *)out, (int)bh0,
-                    heads, dv, rotate);
+                e = launch_overlapped(retention_step_kernel<T, 256>, grid, dim3(kStepThreads), 0,
+                                      stream, (const T *)q, (const T *)k, (const T *)v, gam, rot,
+                                      state, (T *)out, (int)bh0, heads, dv, rotate);
                 break;
             default:
                 return cudaErrorInvalidValue;
         }
         count_launch();
-        const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
