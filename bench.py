@@ -75,8 +75,8 @@ def workload_config(w: wl.Workload, chunk: int, form: str = "chunkwise") -> dict
 # source file at capture time; reported only while the source is unchanged.
 NCU_TRAFFIC = {
     "tc_output": {"source": "chunkwise_tc.cu",
-                  "sha256": "1b9aeee39cdcb809e7de5a39622746a9f229b95a4da317ef7d60397629b3fd50",
-                  "bytes": 160.23e6},
+                  "sha256": "cdc9c928156913a3a79892a46604b1b96884fb9158abaf38f1e3692f25bd6743",
+                  "bytes": 160.33e6},
 }
 
 
@@ -584,16 +584,29 @@ def run_decode(args, w):
         rn.retnet_retention_chunkwise(q, k, v, gam, w.chunk, state_out=state[b0:b1])
         del q, k, v
     torch.cuda.synchronize()
-    steps = w.decode_steps
+    T = args.tokens
     gen = torch.Generator(device=dev)
     gen.manual_seed(w.seed + 7)
-    qd, kd, vd = ((torch.randn(steps, B, H, d, generator=gen, device=dev) * w.scale)
-                  .to(torch.bfloat16) for _ in range(3))
-    o = torch.empty(B, H, d, dtype=torch.bfloat16, device=dev)
+    if T == 1:
+        steps = w.decode_steps
+        qd, kd, vd = ((torch.randn(steps, B, H, d, generator=gen, device=dev) * w.scale)
+                      .to(torch.bfloat16) for _ in range(3))
+        o = torch.empty(B, H, d, dtype=torch.bfloat16, device=dev)
 
-    def step(i):
-        rn.retnet_retention_step(qd[i % steps], kd[i % steps], vd[i % steps], gam, state,
-                                 n + i, out=o)
+        def step(i):
+            rn.retnet_retention_step(qd[i % steps], kd[i % steps], vd[i % steps], gam, state,
+                                     n + i, out=o)
+    else:
+        # T tokens per call (multi-token decode) through the recurrent form;
+        # a pool of four input sets, each call at its own positions
+        steps = 4
+        qd, kd, vd = ((torch.randn(steps, B, T, H, d, generator=gen, device=dev) * w.scale)
+                      .to(torch.bfloat16) for _ in range(3))
+        o = torch.empty(B, T, H, d, dtype=torch.bfloat16, device=dev)
+
+        def step(i):
+            rn.retnet_retention_recurrent(qd[i % steps], kd[i % steps], vd[i % steps], gam,
+                                          state, n + i * T, out=o)
 
     for i in range(args.warmup):
         step(i)
@@ -639,21 +652,25 @@ def run_decode(args, w):
     tot, cnt = kern["retention_step"]
     eager_avg_s = tot / cnt / 1e3          # includes launch latency when the host lags
     avg_s = ms / args.steps / 1e3          # graph replay: kernel time plus node gaps
-    bytes_step = B * H * (8 * d * d + 2 * 4 * d)
+    bytes_step = B * H * (8 * d * d + T * 2 * 4 * d)
     line = {
-        "metric": "decode steps/s (all sequences advance one token)", "value": args.steps / (ms / 1e3),
-        "unit": "steps/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "metric": "decode steps/s (all sequences advance one token)" if T == 1 else
+                  f"multi-token decode calls/s (all sequences advance {T} tokens per call)",
+        "value": args.steps / (ms / 1e3),
+        "unit": "steps/s" if T == 1 else "calls/s", "tokens_per_call": T,
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32 state, bf16 q/k/v", "data": "synthetic",
-        "config": {"workload": f"decode7b: H={H} d={d} batch {B}, state from an {n}-token prefill",
-                   "batch": B, "l2": "state larger than L2" if bytes_step > 126e6 else
+        "config": {"workload": f"decode7b: H={H} d={d} batch {B}, state from an {n}-token prefill"
+                               + ("" if T == 1 else f", {T} tokens per call"),
+                   "batch": B, "tokens_per_call": T, "l2": "state larger than L2" if bytes_step > 126e6 else
                    "state fits in L2 (L2-resident)"},
         "timing": "one replay of a CUDA graph holding all timed steps (one kernel per step); "
                   "the roofline divides by the replay's time per step",
         "eager": {"steps_per_s": args.steps / (eager_ms / 1e3), "ms_per_step": eager_ms / args.steps,
                   "kernel_event_us": eager_avg_s * 1e6, "clocks": clock_info,
                   "gpu_launches": launches_eager},
-        "tokens_per_s": B * args.steps / (ms / 1e3),
+        "tokens_per_s": B * T * args.steps / (ms / 1e3),
         "roofline": {"kernel": "retention_step", "bound": "hbm",
                      "state_l2_resident": bytes_step <= 126e6,
                      "achieved": bytes_step / avg_s / 1e9,
@@ -664,6 +681,15 @@ def run_decode(args, w):
         "gpu_launches": graph_launches, "clocks": clock_info2,
         "launch_overlap": not args.no_overlap,
     }
+    if T > 1:
+        # the state update and the output cost 4 dk dv flops per head-token
+        # (float32 FMA on CUDA cores: 148 SMs x 128 lanes x 2 flop x clock)
+        flops = B * H * T * 4 * d * d
+        alu_peak = 148 * 128 * 2 * (peaks.get("sm_max_mhz", 1965.0) * 1e6) / 1e12
+        line["roofline_alu"] = {"bound": "alu", "achieved": flops / avg_s / 1e12,
+                                "peak": alu_peak, "unit": "TFLOP/s",
+                                "frac": flops / avg_s / 1e12 / alu_peak,
+                                "work_per_launch": flops}
     print(json.dumps(line), flush=True)
 
 
@@ -676,7 +702,11 @@ def main():
     ap.add_argument("--workload", choices=["layer200m", "layer3b", "long7b", "decode7b"],
                     default="layer200m")
     ap.add_argument("--batch", type=int, default=128, help="decode7b batch")
+    ap.add_argument("--tokens", type=int, default=1,
+                    help="decode7b: tokens per call (above 1: the recurrent form)")
     ap.add_argument("--chunk", type=int, default=0)
+    ap.add_argument("--seqlen", type=int, default=0,
+                    help="override the workload's sequence length (length sweeps)")
     ap.add_argument("--algo", choices=["auto", "simt", "tensor"], default="auto")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -686,6 +716,11 @@ def main():
                     help="prefill form; 'parallel' times the parallel form alone (no decode)")
     args = ap.parse_args()
     w = wl.WORKLOADS[args.workload]
+    if args.seqlen:
+        # same shape with another sequence length (a length sweep, not a
+        # configuration of its own); the workload name records it
+        import dataclasses
+        w = dataclasses.replace(w, name=f"{w.name}@n{args.seqlen}", seqlen=args.seqlen)
     chunk = args.chunk or w.chunk
     if args.impl == "reference":
         run_reference(args, w, chunk)

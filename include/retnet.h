@@ -228,6 +228,26 @@ RETNET_API retnet_status retnet_retention_step(const void *q, const void *k, con
                                     int batch, int heads, int dk, int dv, retnet_dtype dtype,
                                     long long pos, int rotate, retnet_stream_t stream);
 
+/* Recurrent form over a run of tokens: multi-token decode, or continuing
+ * every sequence by a short chunk ("Summary": the recurrent form; the
+ * chunkwise form "passes the recurrent state between chunks").  For
+ * t = 0 .. seqlen-1 and every (sequence, head):
+ *     S <- gamma S + k_t^T v_t ;  o_t = q_t S,
+ * with q_t, k_t rotated by pos0 + t when rotate = 1.  Bit-identical to
+ * seqlen calls of retnet_retention_step at positions pos0, pos0 + 1, ...,
+ * but the state is read and written once per call instead of per token.
+ *   q, k  device [batch, seqlen, heads, dk]; v, out [batch, seqlen, heads, dv]
+ *         (shape->dtype; out receives every o_t).
+ *   state device float32 [batch, heads, dk, dv], updated in place to the
+ *         state after the last token.
+ * Work grows with seqlen on CUDA cores (4 dk dv flops per head-token); for
+ * long runs use retnet_retention_chunkwise with state_in.
+ * Errors: INVALID_ARG, UNSUPPORTED (dk/dv not in {64,128,256}), CUDA. */
+RETNET_API retnet_status retnet_retention_recurrent(const void *q, const void *k, const void *v,
+                                         const float *gammas, float *state, void *out,
+                                         const retnet_shape *shape, long long pos0, int rotate,
+                                         retnet_stream_t stream);
+
 /* Output epilogue Y = swish(G) (.) GroupNorm(O) ("Summary": a swish gate
  * and GroupNorm are added).  o, g, y: device [rows, heads, dv] of `dtype`
  * (rows = batch * seqlen); one group per (row, head) over its dv channels,

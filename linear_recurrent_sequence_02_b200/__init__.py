@@ -24,7 +24,7 @@ __all__ = [
     "retnet_default_gammas", "retnet_xpos_rotate", "retnet_chunkwise_workspace_size",
     "retnet_retention_chunkwise", "retnet_parallel_workspace_size", "retnet_retention_parallel",
     "retnet_workspace",
-    "retnet_retention_step", "retnet_groupnorm_swish",
+    "retnet_retention_step", "retnet_retention_recurrent", "retnet_groupnorm_swish",
     "retnet_check_device_errors", "retnet_profiler_enable", "retnet_profiler_select",
     "retnet_profiler_reset",
     "retnet_profiler_read", "ALGO_AUTO", "ALGO_SIMT", "ALGO_TENSOR", "LIB_PATH",
@@ -81,6 +81,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "retnet_retention_parallel": (i, [vp, vp, vp, vp, vp, ctypes.POINTER(_Shape), ll, i,
                                           ctypes.POINTER(_Gate), vp, sz, vp]),
         "retnet_retention_step": (i, [vp, vp, vp, vp, vp, vp, i, i, i, i, i, ll, i, vp]),
+        "retnet_retention_recurrent": (i, [vp, vp, vp, vp, vp, vp, ctypes.POINTER(_Shape), ll, i,
+                                           vp]),
         "retnet_groupnorm_swish": (i, [vp, vp, vp, vp, f, ll, i, i, i, vp, vp]),
         "retnet_check_device_errors": (i, [vp]),
         "retnet_profiler_enable": (i, [i]),
@@ -318,6 +320,32 @@ def retnet_retention_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
             _ptr(q), _ptr(k), _ptr(v), _gammas(gammas, H), _ptr(state), _ptr(out), B, H, dk, dv,
             _dtype_code(q), int(pos), int(bool(rotate)), _stream(q))
     _check("retnet_retention_step", st)
+    return out
+
+
+def retnet_retention_recurrent(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                               gammas: Sequence[float], state: torch.Tensor, pos0: int, *,
+                               rotate: bool = True,
+                               out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Recurrent form over a run of tokens, q, k, v [batch, seqlen, heads, d]:
+    for each token, state <- gamma state + k^T v, o = q state (state updated
+    in place).  Returns out [batch, seqlen, heads, dv]."""
+    _dev(q, "q")
+    if q.dim() != 4:
+        raise ValueError("q must be [batch, seqlen, heads, dk]")
+    B, n, H, dk = q.shape
+    dv = v.shape[-1]
+    _dev(k, "k", q.dtype, (B, n, H, dk))
+    _dev(v, "v", q.dtype, (B, n, H, dv))
+    _dev(state, "state", torch.float32, (B, H, dk, dv))
+    out = torch.empty((B, n, H, dv), dtype=q.dtype, device=q.device) if out is None else \
+        _dev(out, "out", q.dtype, (B, n, H, dv))
+    shape = _Shape(B, H, n, dk, dv, _dtype_code(q))
+    with torch.cuda.device(q.device):
+        st = load_library().retnet_retention_recurrent(
+            _ptr(q), _ptr(k), _ptr(v), _gammas(gammas, H), _ptr(state), _ptr(out),
+            ctypes.byref(shape), int(pos0), int(bool(rotate)), _stream(q))
+    _check("retnet_retention_recurrent", st)
     return out
 
 

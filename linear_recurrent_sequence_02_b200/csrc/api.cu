@@ -247,8 +247,32 @@ retnet_status retnet_retention_step(const void *q, const void *k, const void *v,
     if (!q || !k || !v || !state || !out) return RETNET_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(out))
         return RETNET_ERR_INVALID_ARG;
-    RETNET_CUDA_TRY(launch_retention_step(q, k, v, gam, state, out, batch, heads, dk, dv, dtype,
-                                          pos, rotate, (cudaStream_t)stream));
+    RETNET_CUDA_TRY(launch_retention_recurrent(q, k, v, gam, state, out, batch, 1, heads, dk, dv,
+                                               dtype, pos, rotate, (cudaStream_t)stream));
+    return RETNET_OK;
+}
+
+retnet_status retnet_retention_recurrent(const void *q, const void *k, const void *v,
+                                         const float *gammas, float *state, void *out,
+                                         const retnet_shape *shape, long long pos0, int rotate,
+                                         retnet_stream_t stream) {
+    if (!shape || shape->batch < 0 || shape->seqlen < 0 || shape->heads < 1 ||
+        shape->heads > kMaxHeads || !dtype_ok(shape->dtype) || pos0 < 0 ||
+        (rotate != 0 && rotate != 1))
+        return RETNET_ERR_INVALID_ARG;
+    if (shape->dk <= 0 || shape->dv <= 0) return RETNET_ERR_INVALID_ARG;
+    if (!head_dim_ok(shape->dk) || !head_dim_ok(shape->dv)) return RETNET_ERR_UNSUPPORTED;
+    HeadGammas gam;
+    retnet_status st = load_gammas(gammas, shape->heads, &gam);
+    if (st != RETNET_OK) return st;
+    if ((long long)shape->batch * shape->seqlen == 0) return RETNET_OK;
+    if (!q || !k || !v || !state || !out) return RETNET_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(out))
+        return RETNET_ERR_INVALID_ARG;
+    RETNET_CUDA_TRY(launch_retention_recurrent(q, k, v, gam, state, out, shape->batch,
+                                               shape->seqlen, shape->heads, shape->dk, shape->dv,
+                                               shape->dtype, pos0, rotate,
+                                               (cudaStream_t)stream));
     return RETNET_OK;
 }
 

@@ -49,10 +49,9 @@ struct TcHeadParams {
 };
 
 // ------------------------------------------------------------------ prep
-// One CTA per token t: its 128 (cos, sin) pairs are formed once (angle
-// (pos0 + t) * theta_j in float64, reduced to [-pi, pi], then a float32
-// sincos) and applied to every (sequence, head) row of q and k at that
-// token, together with the decay fold.  Writes Qt, Kt in [b*H + h][t][:].
+// One CTA per token t: its 128 (cos, sin) pairs are formed once
+// (rotation_cs of (pos0 + t) * theta_j) and applied to every (sequence,
+// head) row of q and k at that token, together with the decay fold.  Writes Qt, Kt in [b*H + h][t][:].
 struct TcPrepParams {
     double theta[kD / 2];          // 10000^(-2j/256), formed on the host
     float log2g[kMaxHeads];        // log2(gamma_h)
@@ -88,17 +87,8 @@ tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
     grid_dependency_wait();                         // q, k may come from the kernel before
     load_round(threadIdx.x);
     if (threadIdx.x < kD / 2) {
-        float2 v = make_float2(1.f, 0.f);
-        if (rotate) {
-            const double two_pi = 6.283185307179586476925286766559;
-            const double inv_two_pi = 0.15915494309189533576888376337251;
-            const double a = (double)(pos0 + t) * pp.theta[threadIdx.x];
-            const double red = a - two_pi * rint(a * inv_two_pi);
-            float sn, cn;
-            sincosf((float)red, &sn, &cn);
-            v = make_float2(cn, sn);
-        }
-        cs[threadIdx.x] = v;
+        cs[threadIdx.x] = rotate ? rotation_cs(pos0 + t, pp.theta[threadIdx.x])
+                                 : make_float2(1.f, 0.f);
     }
     __syncthreads();
     for (int base = threadIdx.x; base < tasks; base += kPrepBatch * blockDim.x) {

@@ -80,6 +80,21 @@ cudaError_t launch_overlapped(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// ------------------------------------------------------------------ rotation
+// (cos, sin) of the angle pos * theta in float32.  The angle is reduced in
+// float64 to a fraction of pi in [-1, 1], and sincospif, whose own argument
+// reduction is exact, turns it into the pair.  The prefill prologue, the
+// standalone rotation and the rotation table use this; the decode kernels
+// take pairs formed on the host in float64 instead.
+__device__ __forceinline__ float2 rotation_cs(long long pos, double theta) {
+    const double inv_pi = 0.31830988618379067153776752674503;
+    const double x = (double)pos * theta * inv_pi;           // angle / pi
+    const double xr = x - 2.0 * rint(0.5 * x);               // in [-1, 1]
+    float sn, cn;
+    sincospif((float)xr, &sn, &cn);
+    return make_float2(cn, sn);
+}
+
 // ---------------------------------------------------------------- element IO
 template <typename T> __device__ __forceinline__ float to_f32(T x);
 template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
@@ -122,17 +137,10 @@ __device__ __forceinline__ void store8(__nv_bfloat16 *p, const float *v) {
 }
 
 // ---------------------------------------------------------------- rotation
-// (cos, sin) of pos * theta_j with theta_j = 10000^(-2j/d).  The angle is
-// formed and reduced to [-pi, pi] in float64, then a float32 sincos is
-// taken, so the result is accurate to a few 1e-7 for any position.
+// (cos, sin) of pos * theta_j with theta_j = 10000^(-2j/d) formed here in
+// float64; accurate to a few 1e-7 for any position.
 __device__ __forceinline__ float2 rotation_cs(long long pos, int j, int d) {
-    const double two_pi = 6.283185307179586476925286766559;
-    double theta = pow(10000.0, -2.0 * (double)j / (double)d);
-    double a = (double)pos * theta;
-    double r = a - two_pi * rint(a / two_pi);
-    float s, c;
-    sincosf((float)r, &s, &c);
-    return make_float2(c, s);
+    return rotation_cs(pos, pow(10000.0, -2.0 * (double)j / (double)d));
 }
 
 // ---------------------------------------------------------------- launches

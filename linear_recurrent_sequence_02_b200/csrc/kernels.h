@@ -14,10 +14,13 @@ cudaError_t launch_xpos_rotate(const void *x, void *y, long long rows_bt, int he
                                cudaStream_t stream);
 
 // step.cu ----------------------------------------------------------------
-cudaError_t launch_retention_step(const void *q, const void *k, const void *v,
-                                  const HeadGammas &gam, float *state, void *out, int batch,
-                                  int heads, int dk, int dv, retnet_dtype dtype, long long pos,
-                                  int rotate, cudaStream_t stream);
+// q, k [batch, tokens, heads, dk]; v, out [batch, tokens, heads, dv] (with
+// tokens = 1 this is the [batch, heads, d] layout of a single step).
+cudaError_t launch_retention_recurrent(const void *q, const void *k, const void *v,
+                                       const HeadGammas &gam, float *state, void *out,
+                                       int batch, int tokens, int heads, int dk, int dv,
+                                       retnet_dtype dtype, long long pos, int rotate,
+                                       cudaStream_t stream);
 
 // groupnorm.cu -------------------------------------------------------------
 cudaError_t launch_groupnorm_swish(const void *o, const void *g, const float *weight,

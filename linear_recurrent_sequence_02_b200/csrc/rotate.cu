@@ -18,17 +18,10 @@ __global__ void __launch_bounds__(128)
 rotation_table_kernel(float2 *__restrict__ table, int n, int half, int d, long long pos0) {
     const int j = blockIdx.y * 128 + threadIdx.x;
     if (j >= half) return;
-    const double two_pi = 6.283185307179586476925286766559;
     const double theta = pow(10000.0, -2.0 * (double)j / (double)d);
     const int t0 = blockIdx.x * kTablePositions;
     const int t1 = min(n, t0 + kTablePositions);
-    for (int t = t0; t < t1; ++t) {
-        const double a = (double)(pos0 + t) * theta;
-        const double r = a - two_pi * rint(a / two_pi);
-        float sn, cs;
-        sincosf((float)r, &sn, &cs);
-        table[(size_t)t * half + j] = make_float2(cs, sn);
-    }
+    for (int t = t0; t < t1; ++t) table[(size_t)t * half + j] = rotation_cs(pos0 + t, theta);
 }
 
 cudaError_t launch_rotation_table(float2 *table, int n, int d, long long pos0,

@@ -170,3 +170,26 @@ def test_parallel_form_rejects_before_launch(lib):
     assert _parallel(lib, ws=1024 + 256) == 5                      # not 1024-byte aligned
     assert _parallel(lib, q=None, k=None, v=None, out=None, shape=_shape(B=0, dk=256, dv=256,
                                                                          dt=1)) == 0
+
+
+def test_recurrent_form_rejects_before_launch(lib):
+    P = ctypes.c_void_p
+    g4 = (ctypes.c_float * 4)(0.9, 0.9, 0.9, 0.9)
+
+    def call(q=16, state=16, shape=None, pos0=0, rotate=1, gam=g4):
+        s = shape or _shape(B=2, H=4, n=8, dk=64, dv=64, dt=1)
+        return lib.retnet_retention_recurrent(P(q), P(16), P(16), gam, P(state), P(16),
+                                              ctypes.byref(s), pos0, rotate, None)
+
+    assert lib.retnet_retention_recurrent(P(16), P(16), P(16), g4, P(16), P(16), None, 0, 1,
+                                          None) == 1                       # no shape
+    assert call(q=None) == 1
+    assert call(q=24) == 1                                                  # misaligned
+    assert call(state=None) == 1
+    assert call(pos0=-1) == 1
+    assert call(rotate=2) == 1
+    assert call(gam=None) == 1
+    assert call(shape=_shape(B=2, H=4, n=8, dk=96, dv=64, dt=1)) == 2       # head dim
+    assert call(shape=_shape(B=2, H=4, n=-1, dk=64, dv=64, dt=1)) == 1
+    # an empty run succeeds without touching memory
+    assert call(q=None, state=None, shape=_shape(B=2, H=4, n=0, dk=64, dv=64, dt=1)) == 0
