@@ -15,4 +15,7 @@ from .retention import (  # noqa: F401
     retention_step,
     groupnorm_swish,
     retention_prefill,
+    retention_parallel_backward,
+    xpos_rotate_backward,
+    retention_prefill_backward,
 )

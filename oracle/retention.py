@@ -42,7 +42,9 @@ than itself: hand-derived worked examples under tests/golden/, closed forms
 (gamma = 1 -> prefix-sum linear attention, gamma = 0 -> diagonal,
 d = 2 rotation -> complex multiplication, GroupNorm and SiLU against
 torch's library routines), brute-force state sums and the agreement of the
-three independently written forms.
+three independently written forms.  The gradients of the parallel form are
+pinned by central finite differences of the token-by-token recurrence and by
+closed forms at gamma = 0 and gamma = 1 (reverse prefix sums).
 """
 from __future__ import annotations
 
@@ -236,6 +238,67 @@ def groupnorm_swish(o, gate, weight=None, bias=None, eps: float = 1e-5):
 # --------------------------------------------------------------------------
 # Whole prefill pass: rotation -> chunkwise retention -> (gate epilogue)
 # --------------------------------------------------------------------------
+# --------------------------------------------------------------------------
+# Gradients of the parallel form  ([SUM] "Summary": the parallel form is the
+# one used for training).  The pages print no backward pass; these are the
+# derivatives of O = (Q K^T (.) D) V (zero initial state) written out with
+# the same D, by the product rule on each factor.
+# --------------------------------------------------------------------------
+def retention_parallel_backward(q, k, v, gammas, d_out):
+    """Gradients of O = (Q K^T (.) D) V with respect to Q, K and V.
+
+    With A = Q K^T (.) D and dA = (dO V^T) (.) D (D is constant):
+        dV = A^T dO,   dQ = dA K,   dK = dA^T Q,
+    per (batch, head).  Returns (dq, dk, dv) in the layouts of q, k, v.
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(d_out)
+    B, n, H, _ = q.shape
+    gam = _f64(gammas)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for h in range(H):
+        D = decay_mask(n, gam[h])
+        for b in range(B):
+            Q, K, V, dO = q[b, :, h, :], k[b, :, h, :], v[b, :, h, :], do[b, :, h, :]
+            A = (Q @ K.T) * D
+            dA = (dO @ V.T) * D
+            dv[b, :, h, :] = A.T @ dO
+            dq[b, :, h, :] = dA @ K
+            dk[b, :, h, :] = dA.T @ Q
+    return dq, dk, dv
+
+
+def xpos_rotate_backward(dy, pos0: int = 0) -> np.ndarray:
+    """Gradient of xpos_rotate: each pair's rotation is orthogonal, so the
+    gradient is the pair turned back by the same angle (R^T dy)."""
+    dy = _f64(dy)
+    n, d = dy.shape[1], dy.shape[3]
+    theta = rotation_thetas(d)
+    pos = pos0 + np.arange(n, dtype=F64)
+    ang = pos[:, None] * theta[None, :]
+    c = np.cos(ang)[None, :, None, :]
+    s = np.sin(ang)[None, :, None, :]
+    even = dy[..., 0::2]
+    odd = dy[..., 1::2]
+    out = np.empty_like(dy)
+    out[..., 0::2] = even * c + odd * s
+    out[..., 1::2] = -even * s + odd * c
+    return out
+
+
+def retention_prefill_backward(q, k, v, gammas, d_out, pos0: int = 0, rotate: bool = True):
+    """Gradients of O = retention(R q, R k, v) (zero initial state, no
+    epilogue) with respect to the raw q, k and v, by the chain rule through
+    the rotation.  Returns (dq, dk, dv)."""
+    if rotate:
+        qr, kr = xpos_rotate(q, pos0), xpos_rotate(k, pos0)
+    else:
+        qr, kr = _f64(q), _f64(k)
+    dqr, dkr, dv = retention_parallel_backward(qr, kr, v, gammas, d_out)
+    if rotate:
+        return xpos_rotate_backward(dqr, pos0), xpos_rotate_backward(dkr, pos0), dv
+    return dqr, dkr, dv
+
+
 def retention_prefill(q, k, v, gammas, chunk: int, pos0: int = 0, rotate: bool = True,
                       state_in=None, gate=None, weight=None, bias=None, eps: float = 1e-5):
     """The hot path in page order: rotate q, k; chunkwise retention; epilogue.

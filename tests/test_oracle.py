@@ -252,3 +252,83 @@ def test_slice_rel_err_measure():
     nan = ref.copy()
     nan[0, 0, 0, 0] = np.nan
     assert slice_rel_err(nan, ref) == float("inf")
+
+
+# ---------------------------------------------------------------- gradients
+def _loss_and_grads_fd(q, k, v, gam, w, pos0, h=1e-6):
+    """Central differences of L = sum(O * w), O from the token-by-token
+    recurrence (a form written independently of the gradient formulas)."""
+    def loss(q_, k_, v_):
+        o, _ = oracle.retention_recurrent(oracle.xpos_rotate(q_, pos0),
+                                          oracle.xpos_rotate(k_, pos0), v_, gam)
+        return float((o * w).sum())
+    grads = []
+    for x in (q, k, v):
+        g = np.zeros_like(x)
+        for idx in np.ndindex(*x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = [xp if y is x else y for y in (q, k, v)]
+            args_m = [xm if y is x else y for y in (q, k, v)]
+            g[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        grads.append(g)
+    return grads
+
+
+def test_backward_matches_finite_differences():
+    B, n, H, dk, dv = 1, 5, 2, 4, 6
+    q, k, v = _rand(B, n, H, dk), _rand(B, n, H, dk), _rand(B, n, H, dv)
+    w = _rand(B, n, H, dv)
+    gam = [0.9, 0.5]
+    fd = _loss_and_grads_fd(q, k, v, gam, w, pos0=3)
+    got = oracle.retention_prefill_backward(q, k, v, gam, w, pos0=3)
+    for g_fd, g in zip(fd, got):
+        assert np.allclose(g, g_fd, rtol=1e-6, atol=1e-7)
+
+
+def test_backward_gamma_zero_closed_form():
+    B, n, H, d = 2, 7, 1, 3
+    q, k, v, do = (_rand(B, n, H, d) for _ in range(4))
+    dq, dk, dv = oracle.retention_parallel_backward(q, k, v, [0.0], do)
+    s = (do * v).sum(-1, keepdims=True)                      # dO_t . v_t
+    assert np.allclose(dq, s * k, atol=1e-12)
+    assert np.allclose(dk, s * q, atol=1e-12)
+    assert np.allclose(dv, (q * k).sum(-1, keepdims=True) * do, atol=1e-12)
+
+
+def test_backward_gamma_one_reverse_prefix_sums():
+    # gamma = 1: dV_s = k_s . sum_{t>=s} q_t^T dO_t, dK_s = sum_{t>=s} (q_t dO_t^T) v_s,
+    # dQ_t = dO_t . (sum_{s<=t} v_s^T k_s): prefix sums from the library
+    B, n, H, dk, dv = 1, 9, 1, 3, 4
+    q, k, v, do = _rand(B, n, H, dk), _rand(B, n, H, dk), _rand(B, n, H, dv), _rand(B, n, H, dv)
+    dq, dk_, dv_ = oracle.retention_parallel_backward(q, k, v, [1.0], do)
+    qdo = q[..., :, None] * do[..., None, :]                  # [B, n, H, dk, dv]
+    rsum = np.flip(np.cumsum(np.flip(qdo, axis=1), axis=1), axis=1)
+    assert np.allclose(dv_, np.einsum("bnhk,bnhkv->bnhv", k, rsum), atol=1e-12)
+    assert np.allclose(dk_, np.einsum("bnhkv,bnhv->bnhk", rsum, v), atol=1e-12)
+    vk = v[..., :, None] * k[..., None, :]                    # [B, n, H, dv, dk]
+    psum = np.cumsum(vk, axis=1)
+    assert np.allclose(dq, np.einsum("bnhv,bnhvk->bnhk", do, psum), atol=1e-12)
+
+
+def test_backward_as_forward_calls_on_reversed_sequences():
+    """The decomposition the GPU backward uses: dQ is a causal retention of
+    (dO, V, K), and dK, dV are causal retentions in reversed time."""
+    B, n, H, d = 2, 11, 3, 4
+    q, k, v, do = (_rand(B, n, H, d) for _ in range(4))
+    gam = [0.9, 0.7, 0.97]
+    dq, dk, dv = oracle.retention_parallel_backward(q, k, v, gam, do)
+    rev = lambda x: np.flip(x, axis=1)                       # noqa: E731
+    fq, _ = oracle.retention_chunkwise(do, v, k, gam, 4)
+    fk, _ = oracle.retention_chunkwise(rev(v), rev(do), rev(q), gam, 4)
+    fv, _ = oracle.retention_chunkwise(rev(k), rev(q), rev(do), gam, 4)
+    assert np.allclose(dq, fq, atol=1e-12)
+    assert np.allclose(dk, rev(fk), atol=1e-12)
+    assert np.allclose(dv, rev(fv), atol=1e-12)
+
+
+def test_rotation_backward_is_the_inverse_turn():
+    x = _rand(2, 6, 2, 8)
+    y = oracle.xpos_rotate(x, 9)
+    assert np.allclose(oracle.xpos_rotate_backward(y, 9), x, atol=1e-12)
