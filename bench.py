@@ -562,6 +562,94 @@ def run_ours(args, w, chunk):
         dist.destroy_process_group()
 
 
+def run_backward(args, w, chunk):
+    """Backward pass (retnet_retention_backward) of the prefill without
+    epilogue: one timed step = dq, dk, dv for the whole batch, given dO."""
+    import torch
+
+    import linear_recurrent_sequence_02_b200 as rn
+    from linear_recurrent_sequence_02_b200.build import build
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    build()
+    rn.load_library()
+    rn.retnet_set_launch_overlap(not args.no_overlap)
+    B, n, H, d = w.batch, w.seqlen, w.heads, w.d
+    gam = rn.retnet_default_gammas(H)
+    sets = []
+    for i in range(3):                                  # rotating inputs, each beyond L2/3
+        q, k, v = wl.make_prefill_inputs_device(B, H, n, d, w.scale, w.seed + 31 * i, dev)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(w.seed + 31 * i + 5)
+        do = torch.randn(B, n, H, d, generator=gen, device=dev).to(torch.bfloat16)
+        sets.append((q, k, v, do))
+    dq, dk, dv = (torch.empty(B, n, H, d, dtype=torch.bfloat16, device=dev) for _ in range(3))
+    ws = rn.retnet_workspace(rn.retnet_backward_workspace_size(B, H, n, d, d, torch.bfloat16,
+                                                               chunk, args.algo), dev)
+
+    def step(i):
+        q, k, v, do = sets[i % 3]
+        rn.retnet_retention_backward(q, k, v, do, gam, chunk, algo=args.algo, dq=dq, dk=dk,
+                                     dv=dv, workspace=ws)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    rn.retnet_profiler_reset()
+    rn.retnet_profiler_select(None)
+    rn.retnet_profiler_enable(True)
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    rn.retnet_profiler_enable(False)
+    kern = rn.retnet_profiler_read()
+    rn.retnet_check_device_errors(dev)
+    launches0 = rn.retnet_kernel_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(args.steps):
+            step(i)
+    launches = rn.retnet_kernel_launch_count() - launches0
+    graph.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index or 0)
+    clocks.start()
+    ev0.record(stream)
+    graph.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    del graph
+    rn.retnet_check_device_errors(dev)
+    peaks, src = load_peaks()
+    # three forward retentions: 3 x the forward's algorithmic flops at this chunk
+    alg = 3 * algorithmic_flops_per_token_head(d, chunk) * B * n * H
+    step_s = ms / args.steps / 1e3
+    total = sum(v[0] for v in kern.values())
+    line = {
+        "metric": "retention backward tokens/s (dq, dk, dv of the prefill)",
+        "value": B * n / step_s, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": f"{w.name} backward: B={B} H={H} n={n} d={d} bf16 chunk {chunk}, "
+                               "no epilogue, zero initial state",
+                   "batch": B, "heads": H, "seqlen": n, "chunk": chunk,
+                   "l2": "3 rotating input sets"},
+        "tflops_algorithmic": alg / step_s / 1e12,
+        "frac_of_bf16_peak": alg / step_s / 1e12 / peaks["bf16_tflops"],
+        "kernels": {k: {"avg_us": 1e3 * v[0] / v[1], "launches_per_step": v[1] / 3,
+                        "share": v[0] / max(total, 1e-12)} for k, v in kern.items()},
+        "gpu_launches": launches, "clocks": clock_info, "peak_source": src,
+        "timing": "one replay of a CUDA graph holding the K timed steps; 'kernels' are 3 "
+                  "steps with every kernel bracketed by events",
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_decode(args, w):
     """Decode-only measurement: one timed step = one recurrent step for every
     sequence of the batch (state seeded by an 8192-token GPU prefill)."""
@@ -710,6 +798,8 @@ def main():
     ap.add_argument("--algo", choices=["auto", "simt", "tensor"], default="auto")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass of the prefill (no epilogue) instead")
     ap.add_argument("--no-overlap", action="store_true",
                     help="launch kernels without programmatic launch overlap")
     ap.add_argument("--form", choices=["chunkwise", "parallel"], default="chunkwise",
@@ -726,6 +816,8 @@ def main():
         run_reference(args, w, chunk)
     elif args.workload == "decode7b":
         run_decode(args, w)
+    elif args.backward:
+        run_backward(args, w, chunk)
     else:
         run_ours(args, w, chunk)
 

@@ -228,6 +228,33 @@ RETNET_API retnet_status retnet_retention_step(const void *q, const void *k, con
                                     int batch, int heads, int dk, int dv, retnet_dtype dtype,
                                     long long pos, int rotate, retnet_stream_t stream);
 
+/* ---- Backward pass (training) ------------------------------------------
+ * Gradients of the prefill without epilogue and without initial state
+ * ("Summary": the parallel form is the training form; the chunkwise form
+ * computes it in chunks): for O = retention(R q, R k, v) as
+ * retnet_retention_chunkwise returns it with gate = NULL and
+ * state_in = NULL, and d_out = dL/dO, writes dq = dL/dq, dk, dv.
+ * With A = QK^T (.) D and dA = (dO V^T) (.) D on the rotated Q, K:
+ *     dV = A^T dO,   dQ = R^T (dA K),   dK = R^T (dA^T Q).
+ * dQ is itself a causal retention of (dO, V, K); dK and dV are causal
+ * retentions of time-reversed sequences, so the pass runs three forward
+ * chunkwise retentions (tensor-core path when the shape admits it, else
+ * SIMT, as for the forward call) between reorder/rotate passes.
+ *   q, k [B, n, H, dk], v, d_out, dv [B, n, H, dv], dq, dk [B, n, H, dk]:
+ *            device, shape->dtype, distinct from each other.
+ *   chunk, algo: as for retnet_retention_chunkwise (each of the two
+ *            forward shapes, (dv, dk) and (dk, dv), must admit the algo).
+ *   workspace: retnet_backward_workspace_size() bytes, 1024-byte aligned.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+RETNET_API retnet_status retnet_backward_workspace_size(const retnet_shape *shape, int chunk,
+                                             retnet_algo algo, size_t *bytes);
+RETNET_API retnet_status retnet_retention_backward(const void *q, const void *k, const void *v,
+                                        const void *d_out, const float *gammas, int chunk,
+                                        void *dq, void *dk, void *dv,
+                                        const retnet_shape *shape, long long pos0, int rotate,
+                                        retnet_algo algo, void *workspace,
+                                        size_t workspace_bytes, retnet_stream_t stream);
+
 /* Recurrent form over a run of tokens: multi-token decode, or continuing
  * every sequence by a short chunk ("Summary": the recurrent form; the
  * chunkwise form "passes the recurrent state between chunks").  For

@@ -25,6 +25,7 @@ __all__ = [
     "retnet_retention_chunkwise", "retnet_parallel_workspace_size", "retnet_retention_parallel",
     "retnet_workspace",
     "retnet_retention_step", "retnet_retention_recurrent", "retnet_groupnorm_swish",
+    "retnet_backward_workspace_size", "retnet_retention_backward",
     "retnet_check_device_errors", "retnet_profiler_enable", "retnet_profiler_select",
     "retnet_profiler_reset",
     "retnet_profiler_read", "ALGO_AUTO", "ALGO_SIMT", "ALGO_TENSOR", "LIB_PATH",
@@ -83,6 +84,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "retnet_retention_step": (i, [vp, vp, vp, vp, vp, vp, i, i, i, i, i, ll, i, vp]),
         "retnet_retention_recurrent": (i, [vp, vp, vp, vp, vp, vp, ctypes.POINTER(_Shape), ll, i,
                                            vp]),
+        "retnet_backward_workspace_size": (i, [ctypes.POINTER(_Shape), i, i, ctypes.POINTER(sz)]),
+        "retnet_retention_backward": (i, [vp, vp, vp, vp, vp, i, vp, vp, vp,
+                                          ctypes.POINTER(_Shape), ll, i, i, vp, sz, vp]),
         "retnet_groupnorm_swish": (i, [vp, vp, vp, vp, f, ll, i, i, i, vp, vp]),
         "retnet_check_device_errors": (i, [vp]),
         "retnet_profiler_enable": (i, [i]),
@@ -347,6 +351,51 @@ def retnet_retention_recurrent(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor
             ctypes.byref(shape), int(pos0), int(bool(rotate)), _stream(q))
     _check("retnet_retention_recurrent", st)
     return out
+
+
+def retnet_backward_workspace_size(batch: int, heads: int, seqlen: int, dk: int, dv: int,
+                                   dtype: torch.dtype, chunk: int, algo="auto") -> int:
+    shape = _Shape(batch, heads, seqlen, dk, dv, BF16 if dtype == torch.bfloat16 else F32)
+    n = ctypes.c_size_t(0)
+    _check("retnet_backward_workspace_size",
+           load_library().retnet_backward_workspace_size(ctypes.byref(shape), int(chunk),
+                                                         _ALGOS[algo], ctypes.byref(n)))
+    return int(n.value)
+
+
+def retnet_retention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                              d_out: torch.Tensor, gammas: Sequence[float], chunk: int, *,
+                              pos0: int = 0, rotate: bool = True, algo="auto",
+                              dq: Optional[torch.Tensor] = None,
+                              dk: Optional[torch.Tensor] = None,
+                              dv: Optional[torch.Tensor] = None,
+                              workspace: Optional[torch.Tensor] = None):
+    """Gradients (dq, dk, dv) of O = retention(R q, R k, v) (no epilogue, zero
+    initial state) given d_out = dL/dO; shapes as for the forward call."""
+    _dev(q, "q")
+    if q.dim() != 4:
+        raise ValueError("q must be [batch, seqlen, heads, dk]")
+    B, n, H, Dk = q.shape
+    Dv = v.shape[-1]
+    _dev(k, "k", q.dtype, (B, n, H, Dk))
+    _dev(v, "v", q.dtype, (B, n, H, Dv))
+    _dev(d_out, "d_out", q.dtype, (B, n, H, Dv))
+    dq = torch.empty_like(q) if dq is None else _dev(dq, "dq", q.dtype, (B, n, H, Dk))
+    dk = torch.empty_like(k) if dk is None else _dev(dk, "dk", q.dtype, (B, n, H, Dk))
+    dv = torch.empty_like(v) if dv is None else _dev(dv, "dv", q.dtype, (B, n, H, Dv))
+    need = retnet_backward_workspace_size(B, H, n, Dk, Dv, q.dtype, chunk, algo)
+    if workspace is None:
+        workspace = retnet_workspace(need, q.device)
+    else:
+        _dev(workspace, "workspace", torch.uint8)
+    shape = _Shape(B, H, n, Dk, Dv, _dtype_code(q))
+    with torch.cuda.device(q.device):
+        st = load_library().retnet_retention_backward(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(d_out), _gammas(gammas, H), int(chunk), _ptr(dq),
+            _ptr(dk), _ptr(dv), ctypes.byref(shape), int(pos0), int(bool(rotate)), _ALGOS[algo],
+            _ptr(workspace), workspace.numel(), _stream(q))
+    _check("retnet_retention_backward", st)
+    return dq, dk, dv
 
 
 def retnet_groupnorm_swish(o: torch.Tensor, g: torch.Tensor, weight: Optional[torch.Tensor] = None,

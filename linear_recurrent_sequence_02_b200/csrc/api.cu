@@ -66,6 +66,58 @@ static size_t workspace_for(const retnet_shape *s, int chunk, retnet_algo resolv
     return simt_workspace_bytes(s->batch, s->heads, s->seqlen, s->dk, s->dv, chunk);
 }
 
+// Backward pass layout of the caller's workspace: five [B, n, H, d] buffers
+// (rotated k; reversed v, dO, rotated q, rotated k), then the workspace of
+// the forward calls it makes.
+struct BackwardLayout {
+    size_t kh, rv, rdo, rqh, rkh, fwd, fwd_bytes, total;
+};
+static size_t align1k(size_t x) { return (x + 1023) & ~(size_t)1023; }
+// the forward call shapes: (q, k in dv, values in dk) and (q, k in dk, values in dv)
+static retnet_shape backward_shape_a(const retnet_shape *s) {
+    retnet_shape t = *s;
+    t.dk = s->dv;
+    t.dv = s->dk;
+    return t;
+}
+// Forward workspace for either call shape; gammas == nullptr takes the
+// larger of the two kernel families where AUTO could pick either.
+static size_t backward_fwd_bytes(const retnet_shape *s, int chunk, retnet_algo algo,
+                                 const float *gammas) {
+    size_t n = 0;
+    const retnet_shape shapes[2] = {backward_shape_a(s), *s};
+    for (const retnet_shape &t : shapes) {
+        size_t m;
+        if (gammas) {
+            m = workspace_for(&t, chunk, resolve_algo(&t, chunk, algo, gammas));
+        } else {
+            m = workspace_for(&t, chunk, RETNET_ALGO_SIMT);
+            if (resolve_algo(&t, chunk, algo, nullptr) == RETNET_ALGO_TENSOR) {
+                const size_t tc = workspace_for(&t, chunk, RETNET_ALGO_TENSOR);
+                m = algo == RETNET_ALGO_TENSOR ? tc : (tc > m ? tc : m);
+            }
+        }
+        n = m > n ? m : n;
+    }
+    return n;
+}
+static BackwardLayout backward_layout(const retnet_shape *s, int chunk, retnet_algo algo,
+                                      const float *gammas) {
+    const size_t es = elem_size(s->dtype);
+    const size_t rows = (size_t)s->batch * s->seqlen * s->heads;
+    const size_t bk = align1k(rows * s->dk * es), bv = align1k(rows * s->dv * es);
+    BackwardLayout l;
+    l.kh = 0;
+    l.rv = l.kh + bk;
+    l.rdo = l.rv + bv;
+    l.rqh = l.rdo + bv;
+    l.rkh = l.rqh + bk;
+    l.fwd = l.rkh + bk;
+    l.fwd_bytes = backward_fwd_bytes(s, chunk, algo, gammas);
+    l.total = l.fwd + l.fwd_bytes;
+    return l;
+}
+
 }  // namespace retnet
 
 using namespace retnet;
@@ -228,6 +280,94 @@ retnet_status retnet_retention_parallel(const void *q, const void *k, const void
     a.pos0 = pos0; a.rotate = rotate; a.workspace = workspace;
     a.workspace_bytes = workspace_bytes;
     RETNET_CUDA_TRY(launch_chunkwise_tc(a, gammas, (cudaStream_t)stream, true));
+    return RETNET_OK;
+}
+
+retnet_status retnet_backward_workspace_size(const retnet_shape *shape, int chunk,
+                                             retnet_algo algo, size_t *bytes) {
+    if (!bytes) return RETNET_ERR_INVALID_ARG;
+    retnet_status st = check_shape(shape, chunk);
+    if (st != RETNET_OK) return st;
+    if (algo != RETNET_ALGO_AUTO && algo != RETNET_ALGO_SIMT && algo != RETNET_ALGO_TENSOR)
+        return RETNET_ERR_INVALID_ARG;
+    if (algo == RETNET_ALGO_TENSOR && !tc_shape_ok(shape->dk, shape->dv, shape->dtype, chunk))
+        return RETNET_ERR_UNSUPPORTED;
+    *bytes = (long long)shape->batch * shape->seqlen == 0
+                 ? 0
+                 : backward_layout(shape, chunk, algo, nullptr).total;
+    return RETNET_OK;
+}
+
+retnet_status retnet_retention_backward(const void *q, const void *k, const void *v,
+                                        const void *d_out, const float *gammas, int chunk,
+                                        void *dq, void *dk, void *dv, const retnet_shape *shape,
+                                        long long pos0, int rotate, retnet_algo algo,
+                                        void *workspace, size_t workspace_bytes,
+                                        retnet_stream_t stream) {
+    retnet_status st = check_shape(shape, chunk);
+    if (st != RETNET_OK) return st;
+    if (pos0 < 0 || (rotate != 0 && rotate != 1)) return RETNET_ERR_INVALID_ARG;
+    if (algo != RETNET_ALGO_AUTO && algo != RETNET_ALGO_SIMT && algo != RETNET_ALGO_TENSOR)
+        return RETNET_ERR_INVALID_ARG;
+    ChunkwiseArgs base;
+    st = load_gammas(gammas, shape->heads, &base.gam);
+    if (st != RETNET_OK) return st;
+    const long long tokens = (long long)shape->batch * shape->seqlen;
+    if (tokens > 0) {
+        const void *ptrs[7] = {q, k, v, d_out, dq, dk, dv};
+        for (const void *p : ptrs)
+            if (!p || !aligned16(p)) return RETNET_ERR_INVALID_ARG;
+    }
+    const retnet_shape sa = backward_shape_a(shape);
+    const retnet_algo ra = resolve_algo(&sa, chunk, algo, gammas);
+    const retnet_algo rb = resolve_algo(shape, chunk, algo, gammas);
+    for (int x = 0; x < 2; ++x) {
+        const retnet_shape &t = x ? *shape : sa;
+        if ((x ? rb : ra) == RETNET_ALGO_TENSOR &&
+            (!tc_shape_ok(t.dk, t.dv, t.dtype, chunk) || !tc_gammas_ok(chunk, gammas, t.heads)))
+            return RETNET_ERR_UNSUPPORTED;
+    }
+    if (tokens == 0) return RETNET_OK;
+    const BackwardLayout lay = backward_layout(shape, chunk, algo, gammas);
+    if (!workspace || workspace_bytes < lay.total || ((uintptr_t)workspace & 1023u))
+        return RETNET_ERR_WORKSPACE;
+
+    const cudaStream_t s = (cudaStream_t)stream;
+    const int B = shape->batch, n = shape->seqlen, H = shape->heads;
+    const int DK = shape->dk, DV = shape->dv;
+    const retnet_dtype dt = shape->dtype;
+    char *ws = (char *)workspace;
+    void *kh = ws + lay.kh, *rv = ws + lay.rv, *rdo = ws + lay.rdo, *rqh = ws + lay.rqh,
+         *rkh = ws + lay.rkh;
+    // rotated k; the reversed sequences of v, dO, rotated q and rotated k
+    RETNET_CUDA_TRY(launch_backward_prep(q, k, v, d_out, kh, rkh, rqh, rv, rdo, B, H, n, DK, DV,
+                                         dt, pos0, rotate, s));
+
+    // three forward retentions without rotation, state or epilogue
+    base.state_in = nullptr;
+    base.state_out = nullptr;
+    base.gate = nullptr;
+    base.batch = B; base.heads = H; base.seqlen = n; base.chunk = chunk; base.dtype = dt;
+    base.pos0 = 0; base.rotate = 0;
+    base.workspace = ws + lay.fwd;
+    base.workspace_bytes = lay.fwd_bytes;
+    auto forward = [&](const retnet_shape &t, retnet_algo r, const void *fq, const void *fk,
+                       const void *fv, void *fo) -> cudaError_t {
+        ChunkwiseArgs a = base;
+        a.q = fq; a.k = fk; a.v = fv; a.out = fo;
+        a.dk = t.dk; a.dv = t.dv;
+        return r == RETNET_ALGO_TENSOR ? launch_chunkwise_tc(a, gammas, s)
+                                       : launch_chunkwise_simt(a, s);
+    };
+    // dQ^ = causal retention of (dO, V, K^)            -> dq (rotated frame)
+    RETNET_CUDA_TRY(forward(sa, ra, d_out, v, kh, dq));
+    // rev(dK^) = causal retention of rev(V, dO, Q^)     -> the k^ buffer
+    RETNET_CUDA_TRY(forward(sa, ra, rv, rdo, rqh, kh));
+    // rev(dV) = causal retention of rev(K^, Q^, dO)     -> the rev(v) buffer
+    RETNET_CUDA_TRY(forward(*shape, rb, rkh, rqh, rdo, rv));
+    // back to the caller's frame and time order
+    RETNET_CUDA_TRY(launch_backward_post(dq, kh, rv, dk, dv, B, H, n, DK, DV, dt, pos0, rotate,
+                                         s));
     return RETNET_OK;
 }
 

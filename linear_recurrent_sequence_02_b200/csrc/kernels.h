@@ -13,6 +13,22 @@ cudaError_t launch_xpos_rotate(const void *x, void *y, long long rows_bt, int he
                                retnet_dtype dtype, int seqlen, long long pos0,
                                cudaStream_t stream);
 
+// backward.cu --------------------------------------------------------------
+// theta_j = 10000^(-2j/dk) for j < dk/2 <= 128, formed on the host.
+struct BackwardThetas {
+    double theta[128];
+};
+// K^ = R k; rev(R k), rev(R q), rev(v), rev(dO) (rev: token t -> n-1-t).
+cudaError_t launch_backward_prep(const void *q, const void *k, const void *v, const void *dout,
+                                 void *kh, void *rkh, void *rqh, void *rv, void *rdo, int batch,
+                                 int heads, int n, int dk, int dv, retnet_dtype dtype,
+                                 long long pos0, int rotate, cudaStream_t stream);
+// dq <- R^T dq (in place); dk = R^T rev(dk_rev); dv = rev(dv_rev).
+cudaError_t launch_backward_post(void *dq, const void *dk_rev, const void *dv_rev, void *dk,
+                                 void *dv, int batch, int heads, int n, int dkd, int dvd,
+                                 retnet_dtype dtype, long long pos0, int rotate,
+                                 cudaStream_t stream);
+
 // step.cu ----------------------------------------------------------------
 // q, k [batch, tokens, heads, dk]; v, out [batch, tokens, heads, dv] (with
 // tokens = 1 this is the [batch, heads, d] layout of a single step).

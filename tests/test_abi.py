@@ -193,3 +193,38 @@ def test_recurrent_form_rejects_before_launch(lib):
     assert call(shape=_shape(B=2, H=4, n=-1, dk=64, dv=64, dt=1)) == 1
     # an empty run succeeds without touching memory
     assert call(q=None, state=None, shape=_shape(B=2, H=4, n=0, dk=64, dv=64, dt=1)) == 0
+
+
+def test_backward_rejects_before_launch(lib):
+    P = ctypes.c_void_p
+    g4 = (ctypes.c_float * 4)(0.9, 0.9, 0.9, 0.9)
+    n = ctypes.c_size_t(0)
+    s = _shape(B=2, H=4, n=300, dk=256, dv=256, dt=1)
+    assert lib.retnet_backward_workspace_size(ctypes.byref(s), 512, 0, ctypes.byref(n)) == 0
+    assert n.value > 0
+    assert lib.retnet_backward_workspace_size(ctypes.byref(s), 0, 0, ctypes.byref(n)) == 1
+    odd = _shape(B=2, H=4, n=300, dk=64, dv=128, dt=1)
+    assert lib.retnet_backward_workspace_size(ctypes.byref(odd), 512, 2, ctypes.byref(n)) == 2
+
+    def call(q=1024, dout=1024, dq=1024, shape=None, chunk=512, pos0=0, rotate=1, algo=0,
+             gam=g4, ws=1024, wsb=1 << 40):
+        sh = shape or s
+        return lib.retnet_retention_backward(P(q), P(1024), P(1024), P(dout), gam, chunk, P(dq),
+                                             P(1024), P(1024), ctypes.byref(sh), pos0, rotate,
+                                             algo, P(ws), wsb, None)
+
+    assert call(q=None) == 1
+    assert call(dout=24) == 1                                   # misaligned
+    assert call(dq=None) == 1
+    assert call(pos0=-1) == 1
+    assert call(rotate=2) == 1
+    assert call(algo=9) == 1
+    assert call(gam=None) == 1
+    assert call(chunk=0) == 1
+    assert call(shape=_shape(B=2, H=4, n=300, dk=96, dv=256, dt=1)) == 2
+    assert call(algo=2, shape=_shape(B=2, H=4, n=300, dk=64, dv=64, dt=1)) == 2
+    assert call(ws=None) == 5
+    assert call(wsb=64) == 5
+    assert call(ws=1024 + 512) == 5                             # not 1024-byte aligned
+    assert call(q=None, dout=None, dq=None, shape=_shape(B=0, H=4, n=300, dk=256, dv=256,
+                                                         dt=1)) == 0
