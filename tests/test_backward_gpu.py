@@ -80,3 +80,9 @@ def test_backward_layer200m_shape(rn):
     # the 200M-layer prefill shape (B = 8, H = 4, n = 2048, d = 256, chunk 512)
     w = wl.WORKLOADS["layer200m"]
     check(rn, "bf16", w.batch, w.seqlen, w.heads, w.d, w.d, w.chunk, algo="auto", seed=11)
+
+
+@pytest.mark.parametrize("n", [1, 2])
+def test_backward_shortest_sequences(rn, n):
+    check(rn, "bf16", 3, n, 2, 256, 256, 128, pos0=40, algo="tensor", seed=50 + n)
+    check(rn, "f32", 3, n, 2, 64, 128, 64, pos0=40, seed=60 + n)

@@ -83,6 +83,31 @@ def test_recurrent_equals_single_steps_bitwise(rn, dtype):
     assert torch.equal(Sa, Sb)
 
 
+@pytest.mark.parametrize("d,T", [(256, 30), (64, 100)])
+def test_recurrent_runs_longer_than_one_launch(rn, d, T):
+    """A launch carries the rotation of 3072 / (d/2) tokens (24 at d = 256,
+    96 at 64); longer runs take several launches with the state carried in
+    memory between them."""
+    B, H, pos0 = 2, 2, 300
+    rng = np.random.default_rng(d + T)
+    q, k, v = (wl.normal(rng, (B, T, H, d), 1.0 / np.sqrt(d), "bf16") for _ in range(3))
+    S0 = rng.standard_normal((B, H, d, d)).astype(np.float32) * 0.05
+    gam = rn.retnet_default_gammas(H)
+    qd, kd, vd = dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16")
+    Sa = torch.from_numpy(S0).cuda()
+    out = rn.retnet_retention_recurrent(qd, kd, vd, gam, Sa, pos0)
+    Sb = torch.from_numpy(S0).cuda()
+    steps = [rn.retnet_retention_step(qd[:, t].contiguous(), kd[:, t].contiguous(),
+                                      vd[:, t].contiguous(), gam, Sb, pos0 + t)
+             for t in range(T)]
+    torch.cuda.synchronize()
+    assert torch.equal(out, torch.stack(steps, dim=1))
+    assert torch.equal(Sa, Sb)
+    o_ref, S_ref = want(q, k, v, gam, S0, pos0)
+    assert slice_rel_err(host(out), o_ref) < TOL["bf16"]
+    assert slice_rel_err(Sa.cpu().numpy(), S_ref, head_axis=1) < 1e-5
+
+
 def test_prefill_then_recurrent_continuation(rn):
     """A 1000-token chunkwise prefill continued by 24 tokens of the recurrent
     form equals the 1024-token prefill (outputs of the last 24 tokens and
