@@ -38,7 +38,8 @@ def host(t):
     return t.float().cpu().numpy().astype(np.float64)
 
 
-def check(rn, dtype, B, n, H, dk, dv, chunk, pos0=0, rotate=True, algo="auto", seed=0, gam=None):
+def check(rn, dtype, B, n, H, dk, dv, chunk, pos0=0, rotate=True, algo="auto", seed=0, gam=None,
+          term_scale=False):
     rng = np.random.default_rng(seed)
     q = wl.normal(rng, (B, n, H, dk), 1.0 / np.sqrt(dk), dtype)
     k = wl.normal(rng, (B, n, H, dk), 1.0 / np.sqrt(dk), dtype)
@@ -52,8 +53,20 @@ def check(rn, dtype, B, n, H, dk, dv, chunk, pos0=0, rotate=True, algo="auto", s
     rn.retnet_check_device_errors()
     wq, wk, wv = oracle.retention_prefill_backward(q, k, v, np.float32(gam), do, pos0=pos0,
                                                    rotate=rotate)
-    for got, want, name in ((dq, wq, "dq"), (dk_, wk, "dk"), (dv_, wv, "dv")):
-        err = slice_rel_err(host(got), want)
+    scales = (None, None, None)
+    if term_scale:
+        # Normalise by the size of the terms rather than of the result: the
+        # same gradients of |q|, |k|, |v|, |dO| without rotation, which bound
+        # every sum of products the result is made of.
+        scales = oracle.retention_prefill_backward(np.abs(q), np.abs(k), np.abs(v),
+                                                   np.float32(gam), np.abs(do), rotate=False)
+    for got, want, scale, name in ((dq, wq, scales[0], "dq"), (dk_, wk, scales[1], "dk"),
+                                   (dv_, wv, scales[2], "dv")):
+        if scale is None:
+            err = slice_rel_err(host(got), want)
+        else:
+            diff = np.abs(host(got) - want).max(axis=(1, 3))
+            err = float((diff / np.abs(scale).max(axis=(1, 3))).max())
         assert err < TOL[dtype], (name, err)
 
 
@@ -84,5 +97,10 @@ def test_backward_layer200m_shape(rn):
 
 @pytest.mark.parametrize("n", [1, 2])
 def test_backward_shortest_sequences(rn, n):
-    check(rn, "bf16", 3, n, 2, 256, 256, 128, pos0=40, algo="tensor", seed=50 + n)
+    # With one or two tokens each gradient slice is a multiple of one or two
+    # dot products; where one nearly cancels, the slice is tiny while the
+    # bf16 rounding of the folded operands is set by the size of its terms,
+    # so the bf16 case is measured against that size.
+    check(rn, "bf16", 3, n, 2, 256, 256, 128, pos0=40, algo="tensor", seed=50 + n,
+          term_scale=True)
     check(rn, "f32", 3, n, 2, 64, 128, 64, pos0=40, seed=60 + n)
