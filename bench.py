@@ -204,11 +204,40 @@ def oracle_step(inputs, gam, chunk, b):
     return y, o
 
 
-def host_inputs(w: wl.Workload):
+# ------------------------------------------------------------- ranks (N > 1)
+# Every rank runs its own replica of the workload on its own sequences (no
+# data-path collective); the job's time is the slowest rank's, and the
+# job's throughput counts the units of all ranks.
+def rank_env():
+    """(rank, world size, local rank) from torchrun's environment."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def shard_seed(seed: int, rank: int) -> int:
+    """Seed of a rank's replica: rank 0 keeps the workload's own seed."""
+    return seed + 7919 * rank
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest value over the ranks (the job's time is the slowest rank's)."""
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world: int, units_per_step: int, steps: int, ms: float) -> float:
+    """Whole-job throughput: the units every rank processed over the time."""
+    return world * units_per_step * steps / (ms / 1e3)
+
+
+def host_inputs(w: wl.Workload, rank: int = 0):
+    seed = shard_seed(w.seed, rank)
     q, k, v, g = wl.make_prefill_inputs(w.batch, w.heads, w.seqlen, w.d, w.dtype, w.scale,
-                                        w.seed, hidden=w.hidden)
+                                        seed, hidden=w.hidden)
     qd, kd, vd = (x[0] for x in wl.make_decode_inputs(w.batch, w.heads, 1, w.d, w.dtype,
-                                                      w.scale, w.seed + 100))
+                                                      w.scale, seed + 100))
     return q, k, v, g, qd, kd, vd
 
 
@@ -265,9 +294,7 @@ def run_ours(args, w, chunk):
 
     import linear_recurrent_sequence_02_b200 as rn
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = rank_env()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     if world > 1:
@@ -283,7 +310,7 @@ def run_ours(args, w, chunk):
     rn.retnet_set_launch_overlap(not args.no_overlap)
 
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-    q, k, v, g, qd, kd, vd = host_inputs(w)
+    q, k, v, g, qd, kd, vd = host_inputs(w, rank)
 
     def pinned(x):
         return torch.from_numpy(x).to(tdt).pin_memory()
@@ -348,6 +375,8 @@ def run_ours(args, w, chunk):
     ev1.record(stream)
     torch.cuda.synchronize()
     eager_ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        eager_ms = max_over_ranks(eager_ms, dist, dev)
 
     # ---- device-timed region: the K steps captured once as a CUDA graph
     # (inputs of each step baked into its nodes), replayed once to warm up and
@@ -395,13 +424,11 @@ def run_ours(args, w, chunk):
         dist.barrier()
     ms = ev0.elapsed_time(ev1)
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, dist, dev)
     rn.retnet_check_device_errors(dev)
 
     tokens_per_step = B * n + (0 if par else B)
-    value = world * tokens_per_step * args.steps / (ms / 1e3)
+    value = job_rate(world, tokens_per_step, args.steps, ms)
 
     # ---- end to end through the public API with host buffers
     # Every step copies its inputs from pinned host memory, runs the hot path
@@ -468,10 +495,8 @@ def run_ours(args, w, chunk):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
     if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * tokens_per_step * e2e_steps / (e2e_ms / 1e3)
+        e2e_ms = max_over_ranks(e2e_ms, dist, dev)
+    e2e_value = job_rate(world, tokens_per_step, e2e_steps, e2e_ms)
 
     # ---- roofline of the dominant kernel
     peaks, peak_src = load_peaks()
@@ -553,7 +578,7 @@ def run_ours(args, w, chunk):
                       "event-record nodes around it; 'kernels' are 3 steps after the warm-up "
                       "with every kernel bracketed by events",
             "launch_overlap": not args.no_overlap,
-            "eager": {"value": world * tokens_per_step * args.steps / (eager_ms / 1e3),
+            "eager": {"value": job_rate(world, tokens_per_step, args.steps, eager_ms),
                       "ms_per_step": eager_ms / args.steps},
         }
         print(json.dumps(line), flush=True)
