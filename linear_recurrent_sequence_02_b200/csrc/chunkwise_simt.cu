@@ -11,7 +11,7 @@
 // the 1e-4 tolerance) and any shape the tensor-core path does not take.
 //
 // Two kernels:
-//   state pass   one CTA per (sequence, head, 64-column slab of S) walks the
+//   state pass   one CTA per (sequence, head, 64 x 64 block of S) walks the
 //                chunks in order, writing S_prev of every chunk to the
 //                workspace and the final state to state_out;
 //   output pass  one CTA per (sequence, head, chunk, 32-row tile) forms the
@@ -52,6 +52,33 @@ __device__ __forceinline__ void load_rot_tile(float *sm, int ld, const T *x, int
     }
 }
 
+// Columns [c0, c0 + 64) of the same rows into sm[32][64] (c0 even, so
+// rotation pairs stay whole): the state pass's slice of d_k.
+template <typename T, int D>
+__device__ __forceinline__ void load_rot_slice(float *sm, const T *x, int b, int h, int heads,
+                                               int n, int t0, int valid, const float2 *table,
+                                               int rotate, int c0) {
+    constexpr int HALF = D / 2;
+    for (int idx = threadIdx.x; idx < kTile * 32; idx += kSimtThreads) {
+        int jj = idx / 32, p = idx - jj * 32;             // pair p of the slice
+        float x0 = 0.f, x1 = 0.f;
+        if (jj < valid) {
+            int t = t0 + jj;
+            const T *row = x + (((size_t)b * n + t) * heads + h) * D + c0;
+            x0 = to_f32(row[2 * p]);
+            x1 = to_f32(row[2 * p + 1]);
+            if (rotate) {
+                float2 cs = table[(size_t)t * HALF + c0 / 2 + p];
+                float a = x0;
+                x0 = a * cs.x - x1 * cs.y;
+                x1 = a * cs.y + x1 * cs.x;
+            }
+        }
+        sm[jj * 64 + 2 * p] = x0;
+        sm[jj * 64 + 2 * p + 1] = x1;
+    }
+}
+
 // ------------------------------------------------------------- state pass
 template <typename T, int DK>
 __global__ void __launch_bounds__(kSimtThreads)
@@ -59,22 +86,26 @@ simt_state_kernel(const T *__restrict__ k, const T *__restrict__ v,
                   const float2 *__restrict__ table, HeadGammas gam, const float *state_in,
                   float *state_out, float *__restrict__ s_prev, int heads, int n, int dv,
                   int chunk, int nchunks, int rotate) {
-    constexpr int RPT = DK / 16;                  // state rows per thread
+    // CTA (sequence-head, 64-column slab, 64-row slice of d_k): rows of
+    // U = K^T V are independent, so the slices need no reduction, and
+    // DK/64 times as many CTAs stream as with whole-height slabs.
+    constexpr int RPT = 4;                        // state rows per thread (64 / 16)
     const int bh = blockIdx.x, b = bh / heads, h = bh % heads;
     const int col0 = blockIdx.y * 64;
+    const int row0 = blockIdx.z * 64;
     const int rl = threadIdx.x / 16, cq = threadIdx.x % 16;
     const float g = gam.g[h];
 
     extern __shared__ float smem[];
-    float *ksm = smem;                            // [32][DK]
-    float *vsm = ksm + kTile * DK;                // [32][64]
+    float *ksm = smem;                            // [32][64]: this slice of d_k
+    float *vsm = ksm + kTile * 64;                // [32][64]
     float *gpow = vsm + kTile * 64;               // [chunk + 1]
     for (int e = threadIdx.x; e <= chunk; e += kSimtThreads) gpow[e] = powf(g, (float)e);
 
     float S[RPT][4];
 #pragma unroll
     for (int i = 0; i < RPT; ++i) {
-        int a = rl + 16 * i;
+        int a = row0 + rl + 16 * i;
         float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
         if (state_in)
             s = *reinterpret_cast<const float4 *>(state_in + ((size_t)bh * DK + a) * dv + col0 +
@@ -90,7 +121,7 @@ simt_state_kernel(const T *__restrict__ k, const T *__restrict__ v,
         const float gL = gpow[L];
 #pragma unroll
         for (int i = 0; i < RPT; ++i) {
-            int a = rl + 16 * i;
+            int a = row0 + rl + 16 * i;
             *reinterpret_cast<float4 *>(sp + (size_t)a * dv + col0 + cq * 4) =
                 make_float4(S[i][0], S[i][1], S[i][2], S[i][3]);
 #pragma unroll
@@ -99,7 +130,7 @@ simt_state_kernel(const T *__restrict__ k, const T *__restrict__ v,
         for (int j0 = 0; j0 < L; j0 += kTile) {
             __syncthreads();
             const int valid = min(kTile, L - j0);
-            load_rot_tile<T, DK>(ksm, DK, k, b, h, heads, n, c0 + j0, valid, table, rotate);
+            load_rot_slice<T, DK>(ksm, k, b, h, heads, n, c0 + j0, valid, table, rotate, row0);
             for (int idx = threadIdx.x; idx < kTile * 64; idx += kSimtThreads) {
                 int jj = idx / 64, cc = idx % 64;
                 float val = 0.f;
@@ -116,7 +147,7 @@ simt_state_kernel(const T *__restrict__ k, const T *__restrict__ v,
                 float4 vv = *reinterpret_cast<const float4 *>(vsm + jj * 64 + cq * 4);
 #pragma unroll
                 for (int i = 0; i < RPT; ++i) {
-                    float kr = ksm[jj * DK + rl + 16 * i];
+                    float kr = ksm[jj * 64 + rl + 16 * i];
                     S[i][0] = fmaf(kr, vv.x, S[i][0]);
                     S[i][1] = fmaf(kr, vv.y, S[i][1]);
                     S[i][2] = fmaf(kr, vv.z, S[i][2]);
@@ -128,7 +159,7 @@ simt_state_kernel(const T *__restrict__ k, const T *__restrict__ v,
     if (state_out) {
 #pragma unroll
         for (int i = 0; i < RPT; ++i) {
-            int a = rl + 16 * i;
+            int a = row0 + rl + 16 * i;
             *reinterpret_cast<float4 *>(state_out + ((size_t)bh * DK + a) * dv + col0 + cq * 4) =
                 make_float4(S[i][0], S[i][1], S[i][2], S[i][3]);
         }
@@ -266,13 +297,13 @@ static cudaError_t launch_simt_typed(const ChunkwiseArgs &a, cudaStream_t stream
     const int bh = a.batch * a.heads;
     if (bh == 0) return cudaSuccess;
 
-    size_t smem_a = (size_t)(kTile * DK + kTile * 64 + a.chunk + 1) * sizeof(float);
+    size_t smem_a = (size_t)(kTile * 64 + kTile * 64 + a.chunk + 1) * sizeof(float);
     auto ka = simt_state_kernel<T, DK>;
     err = cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_a);
     if (err != cudaSuccess) return err;
     {
         KernelTimer timer("simt_state", stream);
-        ka<<<dim3(bh, DV / 64), kSimtThreads, smem_a, stream>>>(
+        ka<<<dim3(bh, DV / 64, DK / 64), kSimtThreads, smem_a, stream>>>(
             (const T *)a.k, (const T *)a.v, table, a.gam, a.state_in, a.state_out, s_prev,
             a.heads, a.seqlen, DV, a.chunk, nchunks, a.rotate);
     }
