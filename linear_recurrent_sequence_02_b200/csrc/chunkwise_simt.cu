@@ -16,7 +16,8 @@
 //                workspace and the final state to state_out;
 //   output pass  one CTA per (sequence, head, chunk, 32-row tile) forms the
 //                cross-chunk term from S_prev and the masked intra-chunk
-//                contraction, all from shared-memory tiles.
+//                contraction, all from shared-memory tiles, each thread
+//                accumulating a 4-row register tile.
 // Powers g^e for e = 0..chunk are tabulated per CTA with powf.
 #include "kernels.h"
 
@@ -173,7 +174,14 @@ simt_output_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__
                    const float2 *__restrict__ table, HeadGammas gam,
                    const float *__restrict__ s_prev, T *__restrict__ out, int heads, int n,
                    int chunk, int nchunks, int rotate) {
-    constexpr int NQ = DV / 32;                   // float4 column groups per thread
+    // Accumulators: each thread owns a 4-row x (DV/32)-column tile of the
+    // output (rows 4 rg .. 4 rg + 3; columns u * 32 VW + VW cg + e), so every
+    // S_prev or V value read from shared memory serves four rows and the
+    // column vectors of a warp are contiguous (conflict-free).
+    constexpr int RO = kTile / 8;                 // rows per thread
+    constexpr int VW = DV >= 128 ? 4 : 2;         // column vector width
+    constexpr int NG = DV / (32 * VW);            // column vectors per thread
+    constexpr int CPT = NG * VW;                  // columns per thread
     constexpr int LDQ = DK + 1;
     const int bh = blockIdx.x, b = bh / heads, h = bh % heads;
     const int c = blockIdx.y;
@@ -182,7 +190,8 @@ simt_output_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__
     const int r0 = blockIdx.z * kTile;
     if (r0 >= L) return;
     const int rows = min(kTile, L - r0);
-    const int r = threadIdx.x / 8, cq = threadIdx.x % 8;
+    const int rg = threadIdx.x / 32, cg = threadIdx.x % 32;     // accumulator tile
+    const int r = threadIdx.x / 8, cq = threadIdx.x % 8;         // score layout
     const float g = gam.g[h];
 
     extern __shared__ float smem[];
@@ -194,9 +203,32 @@ simt_output_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__
     for (int e = threadIdx.x; e <= chunk; e += kSimtThreads) gpow[e] = powf(g, (float)e);
     load_rot_tile<T, DK>(qsm, LDQ, q, b, h, heads, n, c0 + r0, rows, table, rotate);
 
-    float acc[NQ][4];
+    float acc[RO][CPT];
 #pragma unroll
-    for (int i = 0; i < NQ; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    for (int i = 0; i < RO; ++i)
+#pragma unroll
+        for (int e = 0; e < CPT; ++e) acc[i][e] = 0.f;
+
+    // acc[i][:] += w[i] * (the thread's columns of row `row` of vsm)
+    auto axpy_rows = [&](const float *w, int row) {
+#pragma unroll
+        for (int u = 0; u < NG; ++u) {
+            float x[VW];
+            const float *src = vsm + row * DV + u * 32 * VW + cg * VW;
+            if constexpr (VW == 4) {
+                const float4 f = *reinterpret_cast<const float4 *>(src);
+                x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
+            } else {
+                const float2 f = *reinterpret_cast<const float2 *>(src);
+                x[0] = f.x; x[1] = f.y;
+            }
+#pragma unroll
+            for (int i = 0; i < RO; ++i)
+#pragma unroll
+                for (int e = 0; e < VW; ++e)
+                    acc[i][u * VW + e] = fmaf(w[i], x[e], acc[i][u * VW + e]);
+        }
+    };
 
     // cross-chunk term (Q (.) xi) S_prev
     const float *sp = s_prev + ((size_t)bh * nchunks + c) * DK * DV;
@@ -208,23 +240,17 @@ simt_output_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__
         __syncthreads();
 #pragma unroll 4
         for (int aa = 0; aa < kTile; ++aa) {
-            float qa = qsm[r * LDQ + a0 + aa];
+            float w[RO];
 #pragma unroll
-            for (int i = 0; i < NQ; ++i) {
-                float4 s = *reinterpret_cast<const float4 *>(vsm + aa * DV + (cq + 8 * i) * 4);
-                acc[i][0] = fmaf(qa, s.x, acc[i][0]);
-                acc[i][1] = fmaf(qa, s.y, acc[i][1]);
-                acc[i][2] = fmaf(qa, s.z, acc[i][2]);
-                acc[i][3] = fmaf(qa, s.w, acc[i][3]);
-            }
+            for (int i = 0; i < RO; ++i) w[i] = qsm[(RO * rg + i) * LDQ + a0 + aa];
+            axpy_rows(w, aa);
         }
     }
-    {
-        const float xi = gpow[min(r0 + r + 1, chunk)];
 #pragma unroll
-        for (int i = 0; i < NQ; ++i)
+    for (int i = 0; i < RO; ++i) {
+        const float xi = gpow[min(r0 + RO * rg + i + 1, chunk)];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[i][e] *= xi;
+        for (int e = 0; e < CPT; ++e) acc[i][e] *= xi;
     }
 
     // intra-chunk term (Q K^T (.) D) V over key tiles up to this row tile
@@ -252,24 +278,24 @@ simt_output_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__
         __syncthreads();
 #pragma unroll 4
         for (int jj = 0; jj < kTile; ++jj) {
-            float p = psm[r * 33 + jj];
+            float w[RO];
 #pragma unroll
-            for (int i = 0; i < NQ; ++i) {
-                float4 vv = *reinterpret_cast<const float4 *>(vsm + jj * DV + (cq + 8 * i) * 4);
-                acc[i][0] = fmaf(p, vv.x, acc[i][0]);
-                acc[i][1] = fmaf(p, vv.y, acc[i][1]);
-                acc[i][2] = fmaf(p, vv.z, acc[i][2]);
-                acc[i][3] = fmaf(p, vv.w, acc[i][3]);
-            }
+            for (int i = 0; i < RO; ++i) w[i] = psm[(RO * rg + i) * 33 + jj];
+            axpy_rows(w, jj);
         }
     }
 
-    if (r < rows) {
-        T *orow = out + (((size_t)b * n + c0 + r0 + r) * heads + h) * DV;
 #pragma unroll
-        for (int i = 0; i < NQ; ++i)
+    for (int i = 0; i < RO; ++i) {
+        const int row = RO * rg + i;
+        if (row < rows) {
+            T *orow = out + (((size_t)b * n + c0 + r0 + row) * heads + h) * DV;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) orow[(cq + 8 * i) * 4 + e] = from_f32<T>(acc[i][e]);
+            for (int u = 0; u < NG; ++u)
+#pragma unroll
+                for (int e = 0; e < VW; ++e)
+                    orow[u * 32 * VW + cg * VW + e] = from_f32<T>(acc[i][u * VW + e]);
+        }
     }
 }
 
