@@ -144,7 +144,8 @@ RETNET_API retnet_status retnet_chunkwise_workspace_size(const retnet_shape *sha
  *              (the last chunk is then shorter).  The tensor path takes
  *              chunk in {128, 256, 512, 1024}.
  *   out        device output [batch, seqlen, heads, dv]: O, or Y when `gate`
- *              is given.
+ *              is given.  Must not overlap q, k, v, the gate input, the
+ *              states or the workspace.
  *   pos0       position of token 0 for the rotation (split prefills pass
  *              the number of tokens already consumed).
  *   rotate     1: rotate q and k by position first; 0: use them as given.
@@ -219,7 +220,9 @@ RETNET_API retnet_status retnet_retention_chunkwise_noalloc(
  *   gammas   HOST float array [heads].
  *   state    device float32 [batch, heads, dk, dv], updated in place:
  *            S <- gamma S + k^T v.
- *   out      device [batch, heads, dv]: o = q S (after the update).
+ *   out      device [batch, heads, dv]: o = q S (after the update).  Must
+ *            not overlap q, k, v or state (every CTA reads the whole q, k
+ *            rows while others write their columns of out).
  *   pos      rotation position of this token (prefill length + steps done).
  *   rotate   1: rotate q and k by pos first; 0: use them as given.
  * Errors: INVALID_ARG, UNSUPPORTED (dk/dv not in {64,128,256}), CUDA. */
@@ -264,7 +267,8 @@ RETNET_API retnet_status retnet_retention_backward(const void *q, const void *k,
  * seqlen calls of retnet_retention_step at positions pos0, pos0 + 1, ...,
  * but the state is read and written once per call instead of per token.
  *   q, k  device [batch, seqlen, heads, dk]; v, out [batch, seqlen, heads, dv]
- *         (shape->dtype; out receives every o_t).
+ *         (shape->dtype; out receives every o_t and must not overlap q, k,
+ *         v or state).
  *   state device float32 [batch, heads, dk, dv], updated in place to the
  *         state after the last token.
  * Work grows with seqlen on CUDA cores (4 dk dv flops per head-token); for
