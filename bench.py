@@ -1,7 +1,9 @@
 """Benchmark of the retention hot path on B200: prints one JSON line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload layer200m|layer3b|long7b] [--chunk C]
+                    [--workload layer200m|layer3b|long7b|decode7b] [--chunk C]
+                    [--form chunkwise|parallel] [--backward] [--seqlen n]
+                    [--batch B] [--tokens T] [--no-overlap]
 
 One step = one pass of the whole hot path over one batch of the workload:
 rotation prologue, chunkwise prefill with the state carried out, the
@@ -15,13 +17,24 @@ are well beyond it).
 
 The K timed steps are captured once as a CUDA graph and replayed (after one
 warm-up replay), so the GPU runs them back to back without host launch
-gaps; the library's kernel timer becomes event-record nodes around every
-kernel in that replay, and the roofline uses those times.  The same K steps
-launched one by one from Python are reported under "eager".
+gaps; that replay holds no timer events.  The dominant kernel's time comes
+from a second capture of the same steps in which the library's kernel timer
+brackets that kernel with event-record nodes, and the roofline uses it.
+The same K steps launched one by one from Python are reported under
+"eager".
 
-Under torchrun each rank runs its own replica (no data-path collective;
-weak scaling).  `--impl reference` times the CPU oracle (float64 numpy) on
-rank 0 on a bounded sample of the same workload.
+Other modes print their own line with their own metric:
+  --form parallel    the parallel form instead of the chunkwise prefill
+                     (prefill only, no state, no decode step);
+  --backward         the backward pass of the prefill (dq, dk, dv);
+  --workload decode7b [--batch B] [--tokens T]
+                     decode steps (T = 1) or T-token recurrent calls from
+                     states seeded by an 8192-token prefill;
+  --seqlen n         the workload's shape at another sequence length.
+
+Under torchrun each rank runs its own replica on its own sequences (no
+data-path collective; weak scaling).  `--impl reference` times the CPU
+oracle (float64 numpy) on rank 0 on a bounded sample of the same workload.
 """
 from __future__ import annotations
 
