@@ -228,3 +228,35 @@ def test_backward_rejects_before_launch(lib):
     assert call(ws=1024 + 512) == 5                             # not 1024-byte aligned
     assert call(q=None, dout=None, dq=None, shape=_shape(B=0, H=4, n=300, dk=256, dv=256,
                                                          dt=1)) == 0
+
+
+def test_bindings_refuse_host_tensors(lib):
+    """Every binding checks device, dtype and shape before calling the
+    library, so no host pointer ever reaches a kernel."""
+    import torch
+    q = torch.zeros(1, 4, 2, 64)
+    gam = [0.9, 0.9]
+    state = torch.zeros(1, 2, 64, 64)
+    with pytest.raises(ValueError):
+        rn.retnet_retention_chunkwise(q, q, q, gam, 64)
+    with pytest.raises(ValueError):
+        rn.retnet_retention_parallel(q, q, q, gam)
+    with pytest.raises(ValueError):
+        rn.retnet_retention_recurrent(q, q, q, gam, state, 0)
+    with pytest.raises(ValueError):
+        rn.retnet_retention_backward(q, q, q, q, gam, 64)
+    with pytest.raises(ValueError):
+        rn.retnet_retention_step(q[:, 0], q[:, 0], q[:, 0], gam, state, 0)
+    with pytest.raises(ValueError):
+        rn.retnet_groupnorm_swish(q, q)
+
+
+def test_bench_work_counts_match_the_formulas():
+    """The per-unit figures bench.py divides by are the algorithmic counts
+    written out for d = 256 and chunk 512."""
+    import bench
+    d, C = 256, 512
+    assert bench.algorithmic_flops_per_token_head(d, C) == 524_800          # (dk+dv)(C+1) + 4 dk dv
+    assert bench.output_kernel_flops_per_token_head(d, C) == 2 * d * (C + 1) + 2 * d * d
+    assert bench.state_kernel_flops_per_token_head(d) == 2 * d * d
+    assert bench.parallel_flops_per_token_head(d, 2047) == 2 * d * 2048
