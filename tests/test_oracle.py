@@ -332,3 +332,40 @@ def test_rotation_backward_is_the_inverse_turn():
     x = _rand(2, 6, 2, 8)
     y = oracle.xpos_rotate(x, 9)
     assert np.allclose(oracle.xpos_rotate_backward(y, 9), x, atol=1e-12)
+
+
+# ---------------------------------------------------------------- properties
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=60, deadline=None)
+@given(B=st.integers(1, 2), n=st.integers(1, 20), H=st.integers(1, 3),
+       dk=st.sampled_from([2, 4, 6]), dv=st.sampled_from([2, 4, 6]),
+       chunk=st.integers(1, 24), seed=st.integers(0, 2**31 - 1),
+       gam=st.lists(st.floats(0.0, 1.0), min_size=3, max_size=3),
+       with_state=st.booleans())
+def test_three_forms_agree_on_random_shapes(B, n, H, dk, dv, chunk, seed, gam, with_state):
+    r = np.random.default_rng(seed)
+    q, k = r.standard_normal((B, n, H, dk)), r.standard_normal((B, n, H, dk))
+    v = r.standard_normal((B, n, H, dv))
+    s0 = r.standard_normal((B, H, dk, dv)) if with_state else None
+    g = gam[:H]
+    op, sp = oracle.retention_parallel(q, k, v, g, s0)
+    orr, sr = oracle.retention_recurrent(q, k, v, g, s0)
+    oc, sc = oracle.retention_chunkwise(q, k, v, g, chunk, s0)
+    assert np.allclose(op, orr, rtol=1e-10, atol=1e-10)
+    assert np.allclose(oc, orr, rtol=1e-10, atol=1e-10)
+    assert np.allclose(sp, sr, rtol=1e-10, atol=1e-10)
+    assert np.allclose(sc, sr, rtol=1e-10, atol=1e-10)
+
+
+@settings(max_examples=15, deadline=None)
+@given(n=st.integers(1, 6), d=st.sampled_from([2, 4]), seed=st.integers(0, 2**31 - 1),
+       g=st.floats(0.05, 1.0), pos0=st.integers(0, 50))
+def test_backward_matches_finite_differences_on_random_cases(n, d, seed, g, pos0):
+    r = np.random.default_rng(seed)
+    q, k, v, w = (r.standard_normal((1, n, 1, d)) for _ in range(4))
+    fd = _loss_and_grads_fd(q, k, v, [g], w, pos0)
+    got = oracle.retention_prefill_backward(q, k, v, [g], w, pos0=pos0)
+    for g_fd, g_an in zip(fd, got):
+        assert np.allclose(g_an, g_fd, rtol=1e-5, atol=1e-6)
