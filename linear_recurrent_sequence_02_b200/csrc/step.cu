@@ -249,10 +249,23 @@ retention_tokens_kernel(const T *__restrict__ q, const T *__restrict__ k,
         *reinterpret_cast<float4 *>(S + (size_t)(rl + i * kStepLanes) * dv) = s[i];
 }
 
+// theta_j = 10000^(-2j/dk) for the three head sizes, formed once per process
+// (every decode step needs all of them; the power is the costly part).
+static const double *host_thetas(int dk) {
+    struct Table {
+        double t[128];
+        explicit Table(int d) {
+            for (int j = 0; j < 128; ++j) t[j] = j < d / 2 ? std::pow(10000.0, -2.0 * j / d) : 0.0;
+        }
+    };
+    static const Table t64(64), t128(128), t256(256);
+    return dk == 64 ? t64.t : dk == 128 ? t128.t : t256.t;
+}
+
 // (cos, sin) of pos * theta_j, theta_j = 10000^(-2j/dk), in float64 on the host
 static float2 host_cs(long long pos, int j, int dk) {
     const double two_pi = 6.283185307179586476925286766559;
-    const double theta = std::pow(10000.0, -2.0 * j / dk);
+    const double theta = host_thetas(dk)[j];
     const double a = (double)pos * theta;
     const double r = a - two_pi * std::nearbyint(a / two_pi);
     return make_float2((float)std::cos(r), (float)std::sin(r));
