@@ -15,6 +15,15 @@ HBM.  Three input sets rotate so that every step reads inputs that are not
 in L2 (each set is larger than a third of the 126 MB L2 and three together
 are well beyond it).
 
+The default workload is the largest single-GPU prefill, the 7B-like long
+prefill (B=1, H=16, n=8192, d=256, bf16, chunk 512, final state out).  The
+default line adds two measurements of their own (skip with --no-legs):
+"decode_legs", the decode configuration (H=16, d=256, states seeded by an
+8192-token prefill) at batch 32 and 128, where the state (269 MB, 1.08 GB)
+is beyond L2, each with its HBM roofline; and "secondary", the 200M-layer
+step (B=8, H=4, n=2048, chunk 512, gate) measured the same way as the main
+workload.
+
 The K timed steps are captured once as a CUDA graph and replayed (after one
 warm-up replay), so the GPU runs them back to back without host launch
 gaps; that replay holds no timer events.  The dominant kernel's time comes
@@ -322,6 +331,33 @@ def run_ours(args, w, chunk):
     rn.load_library()
     rn.retnet_set_launch_overlap(not args.no_overlap)
 
+    line = measure_prefill(args, w, chunk, rank, world, dev, full=True)
+    if args.form == "chunkwise" and not args.no_legs:
+        # the decode configuration at the batches whose state is beyond L2,
+        # and the 200M-layer step as a second prefill shape
+        dw = wl.WORKLOADS["decode7b"]
+        line["decode_legs"] = {f"batch{b}": measure_decode(args, dw, b, 1, dev, world)
+                               for b in (32, 128)}
+        if w.name != "layer200m":
+            sw = wl.WORKLOADS["layer200m"]
+            line["secondary"] = {"layer200m": measure_prefill(args, sw, sw.chunk, rank, world,
+                                                              dev, full=False)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def measure_prefill(args, w, chunk, rank, world, dev, full=True):
+    """Times K steps of the workload (prefill + one decode step per sequence)
+    as one CUDA graph replay; returns the bench line's fields.  `full` adds
+    the eager timing, the end-to-end leg and the CPU baseline."""
+    import torch
+    import torch.distributed as dist
+
+    import linear_recurrent_sequence_02_b200 as rn
+
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     q, k, v, g, qd, kd, vd = host_inputs(w, rank)
 
@@ -379,17 +415,19 @@ def run_ours(args, w, chunk):
     ev1 = torch.cuda.Event(enable_timing=True)
 
     # ---- the same steps launched one by one from Python (reported as "eager")
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    ev0.record(stream)
-    for i in range(args.steps):
-        step(sets[i % nsets])
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    eager_ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        eager_ms = max_over_ranks(eager_ms, dist, dev)
+    eager_ms = None
+    if full:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(sets[i % nsets])
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        eager_ms = ev0.elapsed_time(ev1)
+        if world > 1:
+            eager_ms = max_over_ranks(eager_ms, dist, dev)
 
     # ---- device-timed region: the K steps captured once as a CUDA graph
     # (inputs of each step baked into its nodes), replayed once to warm up and
@@ -448,68 +486,72 @@ def run_ours(args, w, chunk):
     # and copies y and the decode output back.  Copies run on their own
     # streams, double-buffered, so step i's upload overlaps step i-1's
     # compute and download (PCIe is full duplex).
-    h2d = sum(x.numel() * x.element_size() for x in host[:4 if par else 7] if x is not None)
-    d2h = y.numel() * y.element_size() + (0 if par else o.numel() * o.element_size())
-    e2e_steps = max(1, min(args.steps, args.e2e_steps))
-    s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
-    dsets = [[None if x is None else torch.empty_like(x, device=dev) for x in host]
-             for _ in range(2)]
-    ys = [torch.empty_like(y) for _ in range(2)]
-    os_ = [torch.empty_like(o) for _ in range(2)]
-    yh = [torch.empty_like(y, device="cpu").pin_memory() for _ in range(2)]
-    oh = [torch.empty_like(o, device="cpu").pin_memory() for _ in range(2)]
-    st2 = [torch.empty_like(state) for _ in range(2)]
-    ws2 = [rn.retnet_workspace(wsb, dev) for _ in range(2)]
-    nin = 4 if par else 7                 # the parallel form uploads no decode inputs
+    e2e = None
+    if full:
+        h2d = sum(x.numel() * x.element_size() for x in host[:4 if par else 7] if x is not None)
+        d2h = y.numel() * y.element_size() + (0 if par else o.numel() * o.element_size())
+        e2e_steps = max(1, min(args.steps, args.e2e_steps))
+        s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+        dsets = [[None if x is None else torch.empty_like(x, device=dev) for x in host]
+                 for _ in range(2)]
+        ys = [torch.empty_like(y) for _ in range(2)]
+        os_ = [torch.empty_like(o) for _ in range(2)]
+        yh = [torch.empty_like(y, device="cpu").pin_memory() for _ in range(2)]
+        oh = [torch.empty_like(o, device="cpu").pin_memory() for _ in range(2)]
+        st2 = [torch.empty_like(state) for _ in range(2)]
+        ws2 = [rn.retnet_workspace(wsb, dev) for _ in range(2)]
+        nin = 4 if par else 7                 # the parallel form uploads no decode inputs
 
-    def run_e2e(nsteps):
-        in_ready = [torch.cuda.Event() for _ in range(nsteps)]
-        done = [torch.cuda.Event() for _ in range(nsteps)]
-        out_done = [torch.cuda.Event() for _ in range(nsteps)]
-        for i in range(nsteps):
-            j = i % 2
-            with torch.cuda.stream(s_in):
-                if i >= 2:
-                    s_in.wait_event(done[i - 2])
-                for dst, src in zip(dsets[j][:nin], host[:nin]):
-                    if src is not None:
-                        dst.copy_(src, non_blocking=True)
-                in_ready[i].record(s_in)
-            with torch.cuda.stream(s_cmp):
-                s_cmp.wait_event(in_ready[i])
-                if i >= 2:
-                    s_cmp.wait_event(out_done[i - 2])
-                qq, kk, vv, gg, q1, k1, v1 = dsets[j]
-                prefill(qq, kk, vv, gg, st2[j], ys[j], ws2[j])
-                if not par:
-                    rn.retnet_retention_step(q1, k1, v1, gam, st2[j], n, out=os_[j])
-                done[i].record(s_cmp)
-            with torch.cuda.stream(s_out):
-                s_out.wait_event(done[i])
-                yh[j].copy_(ys[j], non_blocking=True)
-                if not par:
-                    oh[j].copy_(os_[j], non_blocking=True)
-                out_done[i].record(s_out)
-        return out_done[-1]
+        def run_e2e(nsteps):
+            in_ready = [torch.cuda.Event() for _ in range(nsteps)]
+            done = [torch.cuda.Event() for _ in range(nsteps)]
+            out_done = [torch.cuda.Event() for _ in range(nsteps)]
+            for i in range(nsteps):
+                j = i % 2
+                with torch.cuda.stream(s_in):
+                    if i >= 2:
+                        s_in.wait_event(done[i - 2])
+                    for dst, src in zip(dsets[j][:nin], host[:nin]):
+                        if src is not None:
+                            dst.copy_(src, non_blocking=True)
+                    in_ready[i].record(s_in)
+                with torch.cuda.stream(s_cmp):
+                    s_cmp.wait_event(in_ready[i])
+                    if i >= 2:
+                        s_cmp.wait_event(out_done[i - 2])
+                    qq, kk, vv, gg, q1, k1, v1 = dsets[j]
+                    prefill(qq, kk, vv, gg, st2[j], ys[j], ws2[j])
+                    if not par:
+                        rn.retnet_retention_step(q1, k1, v1, gam, st2[j], n, out=os_[j])
+                    done[i].record(s_cmp)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(done[i])
+                    yh[j].copy_(ys[j], non_blocking=True)
+                    if not par:
+                        oh[j].copy_(os_[j], non_blocking=True)
+                    out_done[i].record(s_out)
+            return out_done[-1]
 
-    run_e2e(2)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(s_in)
-    s_cmp.wait_stream(s_in)
-    s_out.wait_stream(s_in)
-    last = run_e2e(e2e_steps)
-    s_in.wait_event(last)
-    s_in.wait_stream(s_cmp)
-    e1.record(s_in)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        e2e_ms = max_over_ranks(e2e_ms, dist, dev)
-    e2e_value = job_rate(world, tokens_per_step, e2e_steps, e2e_ms)
+        run_e2e(2)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(s_in)
+        s_cmp.wait_stream(s_in)
+        s_out.wait_stream(s_in)
+        last = run_e2e(e2e_steps)
+        s_in.wait_event(last)
+        s_in.wait_stream(s_cmp)
+        e1.record(s_in)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            e2e_ms = max_over_ranks(e2e_ms, dist, dev)
+        e2e = {"value": job_rate(world, tokens_per_step, e2e_steps, e2e_ms), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+        del dsets, ys, os_, yh, oh, st2, ws2
 
     # ---- roofline of the dominant kernel
     peaks, peak_src = load_peaks()
@@ -534,7 +576,8 @@ def run_ours(args, w, chunk):
             roof = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak,
                     "unit": "TFLOP/s", "frac": achieved / peak,
                     "traffic": None if par else measured_traffic(dom, w.name),
-                    "peak_source": peak_src, "work_per_launch": flops}
+                    "peak_source": peak_src, "work_per_launch": flops,
+                    "avg_us": avg_s * 1e6}
         elif dom in ("tc_state", "simt_state"):
             flops = state_kernel_flops_per_token_head(d) * th
             achieved = flops / avg_s / 1e12
@@ -543,7 +586,7 @@ def run_ours(args, w, chunk):
                 148 * 128 * 2 * (peaks.get("sm_max_mhz", 1965.0) * 1e6) / 1e12
             roof = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak,
                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
-                    "peak_source": peak_src, "work_per_launch": flops}
+                    "peak_source": peak_src, "work_per_launch": flops, "avg_us": avg_s * 1e6}
         else:
             roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": None, "traffic": None, "peak_source": peak_src}
@@ -553,51 +596,48 @@ def run_ours(args, w, chunk):
     dec_ms = (kern_warm["retention_step"][0] / kern_warm["retention_step"][1]
               if "retention_step" in kern_warm else 0.0)
     pre_ms = ms / max(args.steps, 1) - dec_ms
-    prefill = None
+    prefill_info = None
     if pre_ms > 0:
         alg = (parallel_flops_per_token_head(d, n) if par else
                algorithmic_flops_per_token_head(d, chunk)) * B * n * H
-        prefill = {"tokens_per_s": B * n / (pre_ms / 1e3),
-                   "ms": pre_ms,
-                   "tflops_algorithmic": alg / (pre_ms / 1e3) / 1e12,
-                   "frac_of_bf16_peak": alg / (pre_ms / 1e3) / 1e12 / peaks["bf16_tflops"]}
-    decode = None
+        prefill_info = {"tokens_per_s": B * n / (pre_ms / 1e3), "ms": pre_ms,
+                        "tflops_algorithmic": alg / (pre_ms / 1e3) / 1e12,
+                        "frac_of_bf16_peak": alg / (pre_ms / 1e3) / 1e12 / peaks["bf16_tflops"]}
+    step_decode = None
     if "retention_step" in kern_warm:
         tot, cnt = kern_warm["retention_step"]
         avg_s = tot / cnt / 1e3
-        esz = 2 if w.dtype == "bf16" else 4
-        bytes_step = B * H * (8 * d * d + esz * 4 * d)
-        decode = {"steps_per_s": 1.0 / avg_s, "batch": B, "us_per_step": avg_s * 1e6,
-                  "gbs": bytes_step / avg_s / 1e9, "hbm_frac": bytes_step / avg_s / 1e9 /
-                  peaks["hbm_gbs"], "note": "state just written by the prefill (L2-warm)"}
+        step_decode = {"batch": B, "us_per_step": avg_s * 1e6,
+                       "note": f"the step's own decode of {B} sequence(s), state just written "
+                               "by the prefill and L2-resident; the HBM-bound decode "
+                               "measurement is decode_legs"}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not par:
+    if full and rank == 0 and world == 1 and not args.no_cpu_baseline and not par:
         cpu = cpu_baseline(w, chunk)
 
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": w.dtype, "data": "synthetic", "config": workload_config(w, chunk, args.form),
-            "algo": "tensor" if par else args.algo, "roofline": roof, "prefill": prefill, "decode": decode,
-            "kernels": kernels_json, "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-            "gpu_launches": launches, "clocks": clock_info,
-            "timing": "one replay of a CUDA graph holding the K timed steps; the roofline "
-                      "kernel is timed in a second replay of the same steps captured with "
-                      "event-record nodes around it; 'kernels' are 3 steps after the warm-up "
-                      "with every kernel bracketed by events",
-            "launch_overlap": not args.no_overlap,
-            "eager": {"value": job_rate(world, tokens_per_step, args.steps, eager_ms),
-                      "ms_per_step": eager_ms / args.steps},
-        }
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic", "config": workload_config(w, chunk, args.form),
+        "algo": "tensor" if par else args.algo, "roofline": roof, "prefill": prefill_info,
+        "step_decode": step_decode, "kernels": kernels_json, "gpu_launches": launches,
+        "clocks": clock_info,
+        "timing": "one replay of a CUDA graph holding the K timed steps; the roofline "
+                  "kernel is timed in a second replay of the same steps captured with "
+                  "event-record nodes around it; 'kernels' are 3 steps after the warm-up "
+                  "with every kernel bracketed by events",
+        "launch_overlap": not args.no_overlap,
+    }
+    if full:
+        line["cpu_baseline"] = cpu
+        line["e2e"] = e2e
+        line["eager"] = {"value": job_rate(world, tokens_per_step, args.steps, eager_ms),
+                         "ms_per_step": eager_ms / args.steps}
+    del sets, ws, y, o, state
+    torch.cuda.empty_cache()
+    return line
 
 
 def run_backward(args, w, chunk):
@@ -688,20 +728,15 @@ def run_backward(args, w, chunk):
     print(json.dumps(line), flush=True)
 
 
-def run_decode(args, w):
-    """Decode-only measurement: one timed step = one recurrent step for every
-    sequence of the batch (state seeded by an 8192-token GPU prefill)."""
+def measure_decode(args, w, B, T, dev, world=1):
+    """Decode at batch B from states seeded by an 8192-token GPU prefill:
+    K steps (T = 1) or T-token recurrent calls, captured as one CUDA graph
+    and replayed; returns the measurement's fields (max over ranks)."""
     import torch
 
     import linear_recurrent_sequence_02_b200 as rn
-    from linear_recurrent_sequence_02_b200.build import build
 
-    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
-    torch.cuda.set_device(dev)
-    build()
-    rn.load_library()
-    rn.retnet_set_launch_overlap(not args.no_overlap)
-    B, H, d, n = args.batch, w.heads, w.d, w.seqlen
+    H, d, n = w.heads, w.d, w.seqlen
     gam = rn.retnet_default_gammas(H)
     state = torch.empty(B, H, d, d, device=dev)
     for b0 in range(0, B, 16):                       # seed the state slice by slice
@@ -710,28 +745,29 @@ def run_decode(args, w):
         rn.retnet_retention_chunkwise(q, k, v, gam, w.chunk, state_out=state[b0:b1])
         del q, k, v
     torch.cuda.synchronize()
-    T = args.tokens
+    torch.cuda.empty_cache()
     gen = torch.Generator(device=dev)
     gen.manual_seed(w.seed + 7)
+    steps = max(args.steps, 20)
     if T == 1:
-        steps = w.decode_steps
-        qd, kd, vd = ((torch.randn(steps, B, H, d, generator=gen, device=dev) * w.scale)
+        pool = w.decode_steps
+        qd, kd, vd = ((torch.randn(pool, B, H, d, generator=gen, device=dev) * w.scale)
                       .to(torch.bfloat16) for _ in range(3))
         o = torch.empty(B, H, d, dtype=torch.bfloat16, device=dev)
 
         def step(i):
-            rn.retnet_retention_step(qd[i % steps], kd[i % steps], vd[i % steps], gam, state,
+            rn.retnet_retention_step(qd[i % pool], kd[i % pool], vd[i % pool], gam, state,
                                      n + i, out=o)
     else:
         # T tokens per call (multi-token decode) through the recurrent form;
         # a pool of four input sets, each call at its own positions
-        steps = 4
-        qd, kd, vd = ((torch.randn(steps, B, T, H, d, generator=gen, device=dev) * w.scale)
+        pool = 4
+        qd, kd, vd = ((torch.randn(pool, B, T, H, d, generator=gen, device=dev) * w.scale)
                       .to(torch.bfloat16) for _ in range(3))
         o = torch.empty(B, T, H, d, dtype=torch.bfloat16, device=dev)
 
         def step(i):
-            rn.retnet_retention_recurrent(qd[i % steps], kd[i % steps], vd[i % steps], gam,
+            rn.retnet_retention_recurrent(qd[i % pool], kd[i % pool], vd[i % pool], gam,
                                           state, n + i * T, out=o)
 
     for i in range(args.warmup):
@@ -745,7 +781,7 @@ def run_decode(args, w):
     launches0 = rn.retnet_kernel_launch_count()
     clocks.start()
     ev0.record(stream)
-    for i in range(args.steps):
+    for i in range(steps):
         step(i)
     ev1.record(stream)
     torch.cuda.synchronize()
@@ -760,12 +796,16 @@ def run_decode(args, w):
     graph = torch.cuda.CUDAGraph()
     launches1 = rn.retnet_kernel_launch_count()
     with torch.cuda.graph(graph):
-        for i in range(args.steps):
-            step(args.steps + i)
+        for i in range(steps):
+            step(steps + i)
     graph_launches = rn.retnet_kernel_launch_count() - launches1
     graph.replay()                                    # warm-up replay
     torch.cuda.synchronize()
     clocks2 = ClockSampler(dev.index or 0)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
     clocks2.start()
     ev0.record(stream)
     graph.replay()
@@ -773,49 +813,82 @@ def run_decode(args, w):
     torch.cuda.synchronize()
     clock_info2 = clocks2.stop()
     ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        import torch.distributed as dist
+        ms = max_over_ranks(ms, dist, dev)
     del graph
+    rn.retnet_check_device_errors(dev)
     peaks, src = load_peaks()
     tot, cnt = kern["retention_step"]
     eager_avg_s = tot / cnt / 1e3          # includes launch latency when the host lags
-    avg_s = ms / args.steps / 1e3          # graph replay: kernel time plus node gaps
+    avg_s = ms / steps / 1e3               # graph replay: kernel time plus node gaps
     bytes_step = B * H * (8 * d * d + T * 2 * 4 * d)
-    line = {
-        "metric": "decode steps/s (all sequences advance one token)" if T == 1 else
-                  f"multi-token decode calls/s (all sequences advance {T} tokens per call)",
-        "value": args.steps / (ms / 1e3),
-        "unit": "steps/s" if T == 1 else "calls/s", "tokens_per_call": T,
-        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32 state, bf16 q/k/v", "data": "synthetic",
-        "config": {"workload": f"decode7b: H={H} d={d} batch {B}, state from an {n}-token prefill"
-                               + ("" if T == 1 else f", {T} tokens per call"),
-                   "batch": B, "tokens_per_call": T, "l2": "state larger than L2" if bytes_step > 126e6 else
-                   "state fits in L2 (L2-resident)"},
-        "timing": "one replay of a CUDA graph holding all timed steps (one kernel per step); "
-                  "the roofline divides by the replay's time per step",
-        "eager": {"steps_per_s": args.steps / (eager_ms / 1e3), "ms_per_step": eager_ms / args.steps,
-                  "kernel_event_us": eager_avg_s * 1e6, "clocks": clock_info,
-                  "gpu_launches": launches_eager},
-        "tokens_per_s": B * T * args.steps / (ms / 1e3),
+    res = {
+        "batch": B, "tokens_per_call": T, "steps": steps,
+        "steps_per_s": world * steps / (ms / 1e3) if T == 1 else None,
+        "calls_per_s": world * steps / (ms / 1e3) if T > 1 else None,
+        "tokens_per_s": world * B * T * steps / (ms / 1e3),
+        "us_per_step": avg_s * 1e6,
+        "l2": "state larger than L2" if bytes_step > 126e6 else "state fits in L2 (L2-resident)",
         "roofline": {"kernel": "retention_step", "bound": "hbm",
                      "state_l2_resident": bytes_step <= 126e6,
                      "achieved": bytes_step / avg_s / 1e9,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": bytes_step / avg_s / 1e9 / peaks["hbm_gbs"], "traffic": None,
                      "peak_source": src, "work_per_launch": bytes_step},
-        "kernel_avg_us": avg_s * 1e6,
         "gpu_launches": graph_launches, "clocks": clock_info2,
-        "launch_overlap": not args.no_overlap,
+        "eager": {"ms_per_step": eager_ms / steps, "kernel_event_us": eager_avg_s * 1e6,
+                  "clocks": clock_info, "gpu_launches": launches_eager},
+        "timing": "one replay of a CUDA graph holding all timed steps (one kernel per step); "
+                  "the roofline divides the algorithmic bytes by the replay's time per step",
     }
     if T > 1:
         # the state update and the output cost 4 dk dv flops per head-token
         # (float32 FMA on CUDA cores: 148 SMs x 128 lanes x 2 flop x clock)
         flops = B * H * T * 4 * d * d
         alu_peak = 148 * 128 * 2 * (peaks.get("sm_max_mhz", 1965.0) * 1e6) / 1e12
-        line["roofline_alu"] = {"bound": "alu", "achieved": flops / avg_s / 1e12,
-                                "peak": alu_peak, "unit": "TFLOP/s",
-                                "frac": flops / avg_s / 1e12 / alu_peak,
-                                "work_per_launch": flops}
+        res["roofline_alu"] = {"bound": "alu", "achieved": flops / avg_s / 1e12,
+                               "peak": alu_peak, "unit": "TFLOP/s",
+                               "frac": flops / avg_s / 1e12 / alu_peak, "work_per_launch": flops}
+    del state, qd, kd, vd, o
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_decode(args, w):
+    """Decode-only line: one timed step = one recurrent step for every
+    sequence of the batch (state seeded by an 8192-token GPU prefill)."""
+    import torch
+
+    import linear_recurrent_sequence_02_b200 as rn
+    from linear_recurrent_sequence_02_b200.build import build
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    build()
+    rn.load_library()
+    rn.retnet_set_launch_overlap(not args.no_overlap)
+    B, T = args.batch, args.tokens
+    r = measure_decode(args, w, B, T, dev)
+    H, d, n = w.heads, w.d, w.seqlen
+    line = {
+        "metric": "decode steps/s (all sequences advance one token)" if T == 1 else
+                  f"multi-token decode calls/s (all sequences advance {T} tokens per call)",
+        "value": r["steps_per_s"] if T == 1 else r["calls_per_s"],
+        "unit": "steps/s" if T == 1 else "calls/s", "tokens_per_call": T,
+        "n_gpus": 1, "steps": r["steps"], "warmup": args.warmup,
+        "ms_per_step": r["us_per_step"] / 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 state, bf16 q/k/v", "data": "synthetic",
+        "config": {"workload": f"decode7b: H={H} d={d} batch {B}, state from an {n}-token prefill"
+                               + ("" if T == 1 else f", {T} tokens per call"),
+                   "batch": B, "tokens_per_call": T, "l2": r["l2"]},
+        "timing": r["timing"], "eager": r["eager"], "tokens_per_s": r["tokens_per_s"],
+        "roofline": r["roofline"], "kernel_avg_us": r["us_per_step"],
+        "gpu_launches": r["gpu_launches"], "clocks": r["clocks"],
+        "launch_overlap": not args.no_overlap,
+    }
+    if "roofline_alu" in r:
+        line["roofline_alu"] = r["roofline_alu"]
     print(json.dumps(line), flush=True)
 
 
@@ -826,7 +899,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["layer200m", "layer3b", "long7b", "decode7b"],
-                    default="layer200m")
+                    default="long7b")
     ap.add_argument("--batch", type=int, default=128, help="decode7b batch")
     ap.add_argument("--tokens", type=int, default=1,
                     help="decode7b: tokens per call (above 1: the recurrent form)")
@@ -836,6 +909,8 @@ def main():
     ap.add_argument("--algo", choices=["auto", "simt", "tensor"], default="auto")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-legs", action="store_true",
+                    help="skip the decode legs (batch 32, 128) and the secondary prefill shape")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward pass of the prefill (no epilogue) instead")
     ap.add_argument("--no-overlap", action="store_true",

@@ -62,7 +62,8 @@ typedef enum retnet_status {
     RETNET_ERR_UNSUPPORTED = 2,  /* well-formed request this build does not implement */
     RETNET_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
     RETNET_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up */
-    RETNET_ERR_WORKSPACE = 5     /* workspace missing or smaller than required */
+    RETNET_ERR_WORKSPACE = 5,    /* workspace missing or smaller than required */
+    RETNET_ERR_BOUNDS = 6        /* an index check of the debug build failed */
 } retnet_status;
 
 typedef enum retnet_dtype {
@@ -142,7 +143,10 @@ RETNET_API retnet_status retnet_chunkwise_workspace_size(const retnet_shape *sha
  *   gammas     HOST float array [heads]: the per-head decay, each in [0, 1].
  *   chunk      chunk length b, 1..1024; seqlen need not be a multiple
  *              (the last chunk is then shorter).  The tensor path takes
- *              chunk in {128, 256, 512, 1024}.
+ *              chunk in {128, 256, 512, 1024} as given, and any chunk below
+ *              128 by computing with 128-token chunks: the outputs and the
+ *              final state of the chunkwise form do not depend on the chunk
+ *              length, so this changes the rounding order only.
  *   out        device output [batch, seqlen, heads, dv]: O, or Y when `gate`
  *              is given.  Must not overlap q, k, v, the gate input, the
  *              states or the workspace.
@@ -201,7 +205,8 @@ RETNET_API retnet_status retnet_retention_parallel(const void *q, const void *k,
  *   - every GPU that loads the library holds that array until exit;
  *   - it calls no cudaMalloc, cudaFree or other allocating routine;
  *   - it works on the current device (`stream` must belong to it).  Its
- *     first call on a device looks up the array's device address there
+ *     first call in a CUDA context (the first on each device, and the first
+ *     after a cudaDeviceReset) looks up the array's device address there
  *     (cudaGetSymbolAddress); make that first call before any stream
  *     capture on that device;
  *   - all calls on a device share the one array and it keeps the last
@@ -293,9 +298,25 @@ RETNET_API retnet_status retnet_groupnorm_swish(const void *o, const void *g, co
 /* Reads and clears the library's device-side error word on the current
  * device after synchronising `stream`.  Returns RETNET_OK when no kernel
  * reported a problem, RETNET_ERR_TIMEOUT when a bounded wait inside a
- * kernel gave up (its results are then invalid), RETNET_ERR_CUDA when the
- * read itself failed. */
+ * kernel gave up (its results are then invalid; the kernel let its own
+ * copies and MMAs finish, freed its tensor memory and returned, so the
+ * context stays usable), RETNET_ERR_BOUNDS when an index check of the debug
+ * build (RETNET_CHECK_BOUNDS) failed and the access was skipped, and
+ * RETNET_ERR_CUDA when the read itself failed. */
 RETNET_API retnet_status retnet_check_device_errors(retnet_stream_t stream);
+
+#ifdef RETNET_TEST_HOOKS
+/* Debug build only (compiled with RETNET_TEST_HOOKS; absent from the
+ * default library).  No counterpart on the pages: a way to exercise the
+ * timeout path without a GPU fault.  Sets, for the tensor-core prefill
+ * kernels on the current device, the wall-time limit of every pipeline
+ * wait (wait_limit_ns > 0; the default build uses about 2 s), and whether
+ * the state pass's first CTA skips its first TMA load (skip = 1), so that
+ * its MMA warp's wait runs out and the CTA takes the timeout path.
+ * Errors: INVALID_ARG, CUDA. */
+RETNET_API retnet_status retnet_test_set_hooks(unsigned long long wait_limit_ns,
+                                               int skip_first_state_load);
+#endif
 
 /* ---- Kernel timer (diagnostics; off by default) ----------------------
  * While enabled, every kernel this library launches is bracketed by CUDA

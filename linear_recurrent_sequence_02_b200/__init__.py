@@ -12,6 +12,7 @@ Tensors use the C ABI's layouts (see include/retnet.h):
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 from typing import Optional, Sequence
@@ -29,9 +30,12 @@ __all__ = [
     "retnet_check_device_errors", "retnet_profiler_enable", "retnet_profiler_select",
     "retnet_profiler_reset",
     "retnet_profiler_read", "ALGO_AUTO", "ALGO_SIMT", "ALGO_TENSOR", "LIB_PATH",
+    "DEBUG_LIB_PATH", "using_library", "retnet_test_set_hooks",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libretnet.so")
+# Same sources built with index checks and test hooks (build(variant="debug")).
+DEBUG_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libretnet_debug.so")
 
 RETNET_OK = 0
 F32, BF16 = 0, 1
@@ -56,14 +60,17 @@ class _Gate(ctypes.Structure):
                 ("bias", ctypes.c_void_p), ("eps", ctypes.c_float)]
 
 
-_lib = None
+_libs = {}
+_active = None           # path of the library the functions below call (None: LIB_PATH)
 
 
-def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
-    """Loads libretnet.so once; raises if it has not been built."""
-    global _lib
-    if _lib is not None:
-        return _lib
+def load_library(path: Optional[str] = None) -> ctypes.CDLL:
+    """Loads a build of the library once (default: the one the functions of
+    this module currently call, libretnet.so unless `using_library` says
+    otherwise); raises if it has not been built."""
+    path = path or _active or LIB_PATH
+    if path in _libs:
+        return _libs[path]
     if not os.path.exists(path):
         raise RuntimeError(
             f"{path} not found: build it with `python -m linear_recurrent_sequence_02_b200.build`")
@@ -95,12 +102,38 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "retnet_profiler_read": (i, [i, ctypes.c_char_p, sz, ctypes.POINTER(ctypes.c_double),
                                      ctypes.POINTER(ctypes.c_ulonglong)]),
     }
+    if hasattr(lib, "retnet_test_set_hooks"):            # debug build only
+        sigs["retnet_test_set_hooks"] = (i, [ctypes.c_ulonglong, i])
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
         fn.restype = res
         fn.argtypes = args
-    _lib = lib
+    _libs[path] = lib
     return lib
+
+
+@contextlib.contextmanager
+def using_library(path: str):
+    """Inside the with-block every function of this module calls the library
+    at `path` (for example DEBUG_LIB_PATH) instead of libretnet.so."""
+    global _active
+    prev = _active
+    lib = load_library(path)
+    _active = path
+    try:
+        yield lib
+    finally:
+        _active = prev
+
+
+def retnet_test_set_hooks(wait_limit_ns: int, skip_first_state_load: bool) -> None:
+    """Debug build only: the pipeline waits' time limit and the state pass's
+    skipped first load (see retnet_test_set_hooks in include/retnet.h)."""
+    lib = load_library()
+    if not hasattr(lib, "retnet_test_set_hooks"):
+        raise RuntimeError("retnet_test_set_hooks exists only in the debug build")
+    _check("retnet_test_set_hooks",
+           lib.retnet_test_set_hooks(int(wait_limit_ns), int(bool(skip_first_state_load))))
 
 
 def _check(fn: str, status: int):

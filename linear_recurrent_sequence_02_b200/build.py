@@ -1,10 +1,16 @@
 """Builds libretnet.so (all CUDA sources of the package) for sm_100a in-tree.
 
-    python -m linear_recurrent_sequence_02_b200.build [--force] [--verbose]
+    python -m linear_recurrent_sequence_02_b200.build [--force] [--verbose] [--debug]
 
 Each csrc/*.cu is compiled to an object under _build/ (skipped when the
 object is newer than its source and every header), then linked into
 libretnet.so beside this file.  nvcc cross-compiles, so no GPU is needed.
+
+`--debug` (build(variant="debug")) builds libretnet_debug.so from the same
+sources with RETNET_CHECK_BOUNDS (index checks that report through the
+device error word instead of trapping) and RETNET_TEST_HOOKS (the
+retnet_test_set_hooks entry point that lets a test make a pipeline wait run
+out); its objects go to _build/debug/.  The default library has neither.
 """
 from __future__ import annotations
 
@@ -21,6 +27,12 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libretnet.so")
+DEBUG_LIB = os.path.join(PKG, "libretnet_debug.so")
+VARIANTS = {
+    "default": (BUILD, LIB, []),
+    "debug": (os.path.join(BUILD, "debug"), DEBUG_LIB,
+              ["-DRETNET_CHECK_BOUNDS", "-DRETNET_TEST_HOOKS"]),
+}
 INCLUDE = os.path.join(ROOT, "include")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -47,16 +59,18 @@ def _stale(obj: str, src: str, headers) -> bool:
     return any(os.path.getmtime(p) > t for p in [src, *headers, __file__])
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False,
+          variant: str = "default") -> str:
+    build_dir, lib_path, defines = VARIANTS[variant]
+    os.makedirs(build_dir, exist_ok=True)
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     headers = _headers()
     cc = nvcc()
     jobs = []
     for src in sources:
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
         if force or _stale(obj, src, headers):
-            cmd = [cc, *ARCH, *FLAGS, "-c", src, "-o", obj]
+            cmd = [cc, *ARCH, *FLAGS, *defines, "-c", src, "-o", obj]
             if ptxas_verbose:
                 cmd.insert(1, "-Xptxas=-v")
             jobs.append((src, cmd))
@@ -78,19 +92,19 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
     if failed:
         raise RuntimeError(f"nvcc failed for: {', '.join(failed)}")
 
-    objs = [os.path.join(BUILD, os.path.basename(s)[:-3] + ".o") for s in sources]
-    if jobs or force or not os.path.exists(LIB) or \
-            any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
-        tmp = LIB + ".tmp"
+    objs = [os.path.join(build_dir, os.path.basename(s)[:-3] + ".o") for s in sources]
+    if jobs or force or not os.path.exists(lib_path) or \
+            any(os.path.getmtime(o) > os.path.getmtime(lib_path) for o in objs):
+        tmp = lib_path + ".tmp"
         cmd = [cc, *ARCH, "-shared", "-o", tmp, *objs]
         if verbose:
             print(" ".join(cmd), flush=True)
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode:
             sys.stderr.write(r.stdout + r.stderr)
-            raise RuntimeError("linking libretnet.so failed")
-        os.replace(tmp, LIB)
-    return LIB
+            raise RuntimeError(f"linking {os.path.basename(lib_path)} failed")
+        os.replace(tmp, lib_path)
+    return lib_path
 
 
 def main():
@@ -98,8 +112,10 @@ def main():
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
     ap.add_argument("--ptxas-verbose", action="store_true")
+    ap.add_argument("--debug", action="store_true",
+                    help="build libretnet_debug.so (bounds checks and test hooks)")
     a = ap.parse_args()
-    print(build(a.force, a.verbose, a.ptxas_verbose))
+    print(build(a.force, a.verbose, a.ptxas_verbose, "debug" if a.debug else "default"))
 
 
 if __name__ == "__main__":

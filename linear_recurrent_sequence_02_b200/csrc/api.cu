@@ -17,9 +17,26 @@ bool launch_overlap_enabled() { return g_overlap.load(std::memory_order_relaxed)
 
 __device__ unsigned g_device_error = 0u;
 
+void *current_context() {
+    typedef int (*CtxGetCurrentFn)(void **);
+    static CtxGetCurrentFn fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return (CtxGetCurrentFn) nullptr;
+        return (CtxGetCurrentFn)p;
+    }();
+    void *ctx = nullptr;
+    if (!fn || fn(&ctx) != 0) return nullptr;
+    return ctx;
+}
+
+static SymbolAddressCache g_error_word_cache;
+
 unsigned *device_error_word() {
     void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    if (g_error_word_cache.get(g_device_error, &p) != cudaSuccess) return nullptr;
     return (unsigned *)p;
 }
 
@@ -132,6 +149,7 @@ const char *retnet_status_string(retnet_status status) {
         case RETNET_ERR_CUDA: return "CUDA error";
         case RETNET_ERR_TIMEOUT: return "device-side wait timed out";
         case RETNET_ERR_WORKSPACE: return "workspace missing or too small";
+        case RETNET_ERR_BOUNDS: return "device-side index check failed (debug build)";
     }
     return "unknown status";
 }
@@ -438,7 +456,8 @@ retnet_status retnet_check_device_errors(retnet_stream_t stream) {
     if (word == 0) return RETNET_OK;
     if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess)
         return RETNET_ERR_CUDA;
-    return (word & kDevErrTimeout) ? RETNET_ERR_TIMEOUT : RETNET_ERR_CUDA;
+    if (word & kDevErrTimeout) return RETNET_ERR_TIMEOUT;
+    return (word & kDevErrBounds) ? RETNET_ERR_BOUNDS : RETNET_ERR_CUDA;
 }
 
 }  // extern "C"

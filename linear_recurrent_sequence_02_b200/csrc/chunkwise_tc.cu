@@ -60,7 +60,9 @@ struct TcPrepParams {
 __global__ void __launch_bounds__(256, 4)
 tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                TcPrepParams pp, __nv_bfloat16 *__restrict__ qt, __nv_bfloat16 *__restrict__ kt,
-               int batch, int heads, int n, int chunk, long long pos0, int rotate) {
+               int batch, int heads, int n, int chunk, long long pos0, int rotate,
+               unsigned *err) {
+    const long long elems = (long long)batch * n * heads * kD;   // of q, k, Qt and Kt
     __shared__ float2 cs[kD / 2];
     const int t = blockIdx.x;
     const int i = t % chunk;                        // index inside the chunk
@@ -79,6 +81,7 @@ tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
                 const int bhi = task / (kD / 8);
                 const int h = bhi % heads, b = bhi / heads;
                 const size_t src = (((size_t)b * n + t) * heads + h) * kD + part * 8;
+                if (!in_bounds((long long)src + 7, elems, err)) continue;
                 rq[u] = *reinterpret_cast<const uint4 *>(q + src);
                 rk[u] = *reinterpret_cast<const uint4 *>(k + src);
             }
@@ -117,6 +120,7 @@ tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
                     ok[2 * p + 1] = xk.x * sk2 + xk.y * ck;
                 }
                 const size_t dst = (((size_t)b * heads + h) * n + t) * kD + part * 8;
+                if (!in_bounds((long long)dst + 7, elems, err)) continue;
                 store8(qt + dst, oq);
                 store8(kt + dst, ok);
             }
@@ -150,6 +154,13 @@ __device__ __forceinline__ void store_bf16_row(__nv_bfloat16 *dst, const float *
                        sm100::pack_bf16x2(v[i + 4], v[i + 5]), sm100::pack_bf16x2(v[i + 6], v[i + 7]));
 }
 
+#ifdef RETNET_TEST_HOOKS
+// Test hook (debug build only): when set, the state pass's first CTA never
+// issues its first TMA load, so its MMA warp's wait runs out and the CTA
+// takes the timeout path.  Set by retnet_test_set_hooks.
+static __device__ int g_hook_skip_first_load = 0;
+#endif
+
 template <int DVC>
 __global__ void __launch_bounds__(kTcThreads, 1)
 tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -161,12 +172,13 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     constexpr int kParts = 2 * (kD / DVC);             // CTAs per sequence-head
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    __shared__ uint64_t full[S], empty[S], acc_full[2], acc_free[2];
+    __shared__ uint64_t full[S], empty[S], acc_full[2], acc_free[2], drain;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int bh = blockIdx.x / kParts;
+    const long long nbh = gridDim.x / kParts;               // sequence-heads of the launch
     const int part = blockIdx.x % kParts;
     const int mh = part / (kD / DVC), nv = part % (kD / DVC);   // d_k half, d_v block
     const int b = bh / heads, h = bh % heads;
@@ -180,6 +192,7 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             mbar_init(&acc_full[x], 1);
             mbar_init(&acc_free[x], 128);
         }
+        mbar_init(&drain, 1);
         abort_flag = 0;
         fence_barrier_init();
     }
@@ -197,9 +210,9 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const uint32_t tmem = tmem_slot;
     grid_dependency_wait();                             // Kt from the prep kernel
 
+    int it = 0, skipped = -1;              // producer: ring items issued, one never issued
     if (warp == 0) {
         if (lane == 0) {
-            int it = 0;
             for (int c = 0; c < nchunks && !abort_flag; ++c) {
                 const int c0 = c * chunk;
                 const int L = min(chunk, n - c0);
@@ -207,6 +220,13 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     const int s = it % S;
                     if (it >= S && !mbar_wait(&empty[s], ((it / S) - 1) & 1, &abort_flag, err))
                         break;
+#ifdef RETNET_TEST_HOOKS
+                    if (it == 0 && blockIdx.x == 0 &&
+                        *(volatile int *)&g_hook_skip_first_load) {
+                        skipped = 0;                       // never issued: its wait runs out
+                        continue;
+                    }
+#endif
                     uint8_t *kb = smem + s * Smem::kStage;
                     uint8_t *vb = kb + 2 * kBox;
                     mbar_expect_tx(&full[s], Smem::kStage);
@@ -256,8 +276,10 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const int krow = 128 * mh + row;                     // row of S
         const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
         const size_t sbase = ((size_t)bh * kD + krow) * kD + DVC * nv;
+        const long long state_elems = nbh * kD * kD;
+        const long long sprev_elems = nbh * nchunks * kD * kD;
         float st[DVC];
-        if (state_in) {
+        if (state_in && in_bounds((long long)sbase + DVC - 1, state_elems, err)) {
             const float4 *src = reinterpret_cast<const float4 *>(state_in + sbase);
 #pragma unroll
             for (int v4 = 0; v4 < DVC / 4; ++v4) {
@@ -268,7 +290,11 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 #pragma unroll
             for (int e = 0; e < DVC; ++e) st[e] = 0.f;
         }
-        store_bf16_row(s_prev + ((size_t)bh * nchunks * kD + krow) * kD + DVC * nv, st, DVC);
+        {
+            const size_t o0 = ((size_t)bh * nchunks * kD + krow) * kD + DVC * nv;
+            if (in_bounds((long long)o0 + DVC - 1, sprev_elems, err))
+                store_bf16_row(s_prev + o0, st, DVC);
+        }
         for (int c = 0; c < nchunks; ++c) {
             const int buf = c & 1;
             if (!warp_wait(&acc_full[buf], (c >> 1) & 1, &abort_flag, err)) break;
@@ -287,9 +313,10 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             tc_fence_before();
             mbar_arrive(&acc_free[buf]);                     // buffer free for chunk c + 2
             if (!last) {
-                store_bf16_row(s_prev + (((size_t)bh * nchunks + c + 1) * kD + krow) * kD + DVC * nv,
-                               st, DVC);
-            } else if (state_out) {
+                const size_t o1 = (((size_t)bh * nchunks + c + 1) * kD + krow) * kD + DVC * nv;
+                if (in_bounds((long long)o1 + DVC - 1, sprev_elems, err))
+                    store_bf16_row(s_prev + o1, st, DVC);
+            } else if (state_out && in_bounds((long long)sbase + DVC - 1, state_elems, err)) {
                 float4 *o = reinterpret_cast<float4 *>(state_out + sbase);
 #pragma unroll
                 for (int v4 = 0; v4 < DVC / 4; ++v4)
@@ -299,7 +326,19 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     }
     tc_fence_before();
     __syncthreads();
+    // Every role has finished, so abort_flag is final.  After an abort, wait
+    // (bounded) for what this CTA still has in flight: the TMA loads (at most
+    // the last S issued) before shared memory goes away, the MMAs before
+    // tensor memory is freed.
+    if (abort_flag && warp == 0 && lane == 0)
+        for (int j = max(0, it - S); j < it; ++j)
+            if (j != skipped) mbar_drain(&full[j % S], (j / S) & 1, err);
     if (warp == 1) {
+        if (abort_flag && lane == 0) {
+            mma_commit(&drain);
+            mbar_drain(&drain, 0, err);
+        }
+        __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, 256);
     }
@@ -386,12 +425,13 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     __shared__ uint64_t rfull[kSlots], rempty[kSlots];
-    __shared__ uint64_t s_full, s_read, p_full[2], p_free[2], o_full, o_free;
+    __shared__ uint64_t s_full, s_read, p_full[2], p_free[2], o_full, o_free, drain;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     unsigned *err = a.err;
+    const long long nbh = a.items / (a.nchunks * a.rblocks);   // sequence-heads
     auto slot_ptr = [smem](int it) -> uint8_t * { return smem + (it % kSlots) * kSlot; };
     uint8_t *pbuf = smem + TcOutSmem::kP;
 
@@ -405,6 +445,7 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         mbar_init(&o_full, 1);
         mbar_init(&o_free, kEpiThreads);
+        mbar_init(&drain, 1);
         abort_flag = 0;
         fence_barrier_init();
     }
@@ -424,9 +465,10 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t tO = tmem, tQ = tmem + 256, tS = tmem + 384;
     grid_dependency_wait();                             // Qt, Kt, S_prev from the kernels before
 
+    int pit = 0;                           // producer: ring items issued
     if (warp == 0) {
         if (lane == 0) {
-            int it = 0;
+            int &it = pit;
             bool ok = true;
             auto acquire = [&]() -> bool {
                 if (it < kSlots) return true;
@@ -447,6 +489,13 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const TcItem m = tc_item(a, w);
                 if (!m.valid) continue;
                 const int srow = (m.bh * a.nchunks + m.c) * kD;
+                // debug build: the item's tile coordinates lie inside its tensors
+                if (!in_bounds(m.t0row, a.n, err) || !in_bounds(m.bh, nbh, err) ||
+                    !in_bounds(srow + kD - 1, nbh * a.nchunks * kD, err)) {
+                    abort_flag = 1;
+                    ok = false;
+                    break;
+                }
                 if (!(ok = acquire())) break;
                 issue(&tm_q, 3, m.t0row, m.bh, 0);
                 if (!(ok = acquire())) break;
@@ -499,8 +548,13 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     if (o_written || li == 0) return true;
                     return mbar_wait(&o_free, (li - 1) & 1, &abort_flag, err);
                 };
-                // Qt (K-major, 128-byte swizzle) -> TMEM, 16 columns of K per copy;
-                // ordered after the previous item's MMAs that read Qt.
+                // Qt (K-major, 128-byte swizzle) -> TMEM, 16 columns of K per copy.
+                // The PTX ISA orders tcgen05.cp before later tcgen05.mma of the
+                // same thread, but not after earlier ones: the previous item's
+                // MMAs, the last readers of Qt, must have completed (o_full)
+                // before the copy may overwrite it.
+                if (li > 0 && !(ok = mbar_wait(&o_full, (li - 1) & 1, &abort_flag, err))) break;
+                tc_fence_after();
                 if (!(ok = take())) break;
                 {
                     const uint32_t base = sbase + (it % kSlots) * kSlot;
@@ -568,6 +622,7 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     ++npv;
                 }
                 for (int p = m.nk; ok && p < m.nsp; ++p) ok = qs_half(p);
+                if (!ok) break;
                 mma_commit(&o_full);
                 ++it;                                          // skip the gate/output item
             }
@@ -742,7 +797,19 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     tc_fence_before();
     __syncthreads();
+    // Every role has finished, so abort_flag is final.  After an abort, wait
+    // (bounded) for what this CTA still has in flight: the TMA loads (at most
+    // the last kSlots issued) before shared memory goes away, the MMAs before
+    // tensor memory is freed.
+    if (abort_flag && warp == 0 && lane == 0)
+        for (int j = max(0, pit - kSlots); j < pit; ++j)
+            mbar_drain(&rfull[j % kSlots], (j / kSlots) & 1, err);
     if (warp == 1) {
+        if (abort_flag && lane == 0) {
+            mma_commit(&drain);
+            mbar_drain(&drain, 0, err);
+        }
+        __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
@@ -798,12 +865,20 @@ static TcLayout tc_layout(int batch, int heads, int n, int chunk) {
     return l;
 }
 
+// Chunk length the kernels compute with.  The chunkwise form's outputs and
+// final state do not depend on the chunk length (every length gives the
+// recurrence's result), so a chunk shorter than one 128-row tile is computed
+// with 128-token chunks; longer chunks run as given.
+static int effective_chunk(int chunk) { return chunk < kBlk ? kBlk : chunk; }
+
 bool tc_shape_ok(int dk, int dv, retnet_dtype dtype, int chunk) {
     if (dk != kD || dv != kD || dtype != RETNET_BF16) return false;
-    return chunk == 128 || chunk == 256 || chunk == 512 || chunk == 1024;
+    return (chunk >= 1 && chunk < kBlk) || chunk == 128 || chunk == 256 || chunk == 512 ||
+           chunk == 1024;
 }
 
 bool tc_gammas_ok(int chunk, const float *gammas, int heads) {
+    chunk = effective_chunk(chunk);
     for (int h = 0; h < heads; ++h) {
         const double g = gammas[h];
         if (!(g > 0.0)) return false;
@@ -813,7 +888,7 @@ bool tc_gammas_ok(int chunk, const float *gammas, int heads) {
 }
 
 size_t tc_workspace_bytes(int batch, int heads, int seqlen, int chunk) {
-    return tc_layout(batch, heads, seqlen, chunk).total;
+    return tc_layout(batch, heads, seqlen, effective_chunk(chunk)).total;
 }
 
 // The parallel form runs the output pass over the whole sequence as one
@@ -828,8 +903,8 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
                                 bool parallel) {
     const int n = a.seqlen, H = a.heads, B = a.batch;
     // parallel form: one chunk spanning the sequence, decay folded per 128-row block
-    const int C = parallel ? parallel_span(n) : a.chunk;
-    const int fold = parallel ? kBlk : a.chunk;
+    const int C = parallel ? parallel_span(n) : effective_chunk(a.chunk);
+    const int fold = parallel ? kBlk : C;
     const int BH = B * H;
     if (BH == 0 || (parallel && n == 0)) return cudaSuccess;
     if (n == 0) {                                   // nothing to scan: state passes through
@@ -902,7 +977,7 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
         KernelTimer timer("tc_prep", stream);
         e = launch_overlapped(tc_prep_kernel, dim3(n), dim3(256), 0, stream,
                               (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, pp, qt, kt,
-                              B, H, n, fold, a.pos0, a.rotate);
+                              B, H, n, fold, a.pos0, a.rotate, err);
         count_launch();
         if (e != cudaSuccess) return e;
     }
@@ -964,3 +1039,19 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
 }
 
 }  // namespace retnet
+
+#ifdef RETNET_TEST_HOOKS
+// Debug build only: lowers the wall-time limit of the pipeline waits in this
+// file's kernels, and makes the state pass's first CTA skip its first load.
+extern "C" RETNET_API retnet_status retnet_test_set_hooks(unsigned long long wait_limit_ns,
+                                                          int skip_first_state_load) {
+    if (wait_limit_ns == 0 || (skip_first_state_load != 0 && skip_first_state_load != 1))
+        return RETNET_ERR_INVALID_ARG;
+    if (cudaMemcpyToSymbol(retnet::sm100::g_hook_wait_limit_ns, &wait_limit_ns,
+                           sizeof(wait_limit_ns)) != cudaSuccess ||
+        cudaMemcpyToSymbol(retnet::g_hook_skip_first_load, &skip_first_state_load,
+                           sizeof(int)) != cudaSuccess)
+        return RETNET_ERR_CUDA;
+    return RETNET_OK;
+}
+#endif

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/retnet.h"
 
 namespace retnet {
@@ -19,8 +21,75 @@ struct HeadGammas {
 // Device-side error word (bit flags), read by retnet_check_device_errors.
 enum DeviceError : unsigned {
     kDevErrTimeout = 1u,
+    kDevErrBounds = 2u,          // an index check of a RETNET_CHECK_BOUNDS build failed
 };
-unsigned *device_error_word();   // device address of this device's error word
+unsigned *device_error_word();   // device address of the current context's error word
+
+// The current CUDA context (a CUcontext), or null if none is current.
+void *current_context();
+
+// Device address of a __device__ variable in the current context, looked up
+// once per context (cudaGetSymbolAddress, with that context current) and
+// cached.  Keyed by context, not device ordinal, so an address never outlives
+// the context it belongs to (after cudaDeviceReset the primary context is a
+// new one).  Use it in the translation unit that defines the variable.
+class SymbolAddressCache {
+  public:
+    template <typename T>
+    cudaError_t get(const T &symbol, void **out) {
+        void *ctx = current_context();
+        if (!ctx) {                        // no context yet: the runtime creates it
+            cudaError_t e = cudaFree(nullptr);
+            if (e != cudaSuccess) return e;
+            ctx = current_context();
+            if (!ctx) return cudaErrorDeviceUninitialized;
+        }
+        Lock lk(this);
+        for (int i = 0; i < n_; ++i)
+            if (ctx_[i] == ctx) {
+                *out = ptr_[i];
+                return cudaSuccess;
+            }
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, symbol);
+        if (e != cudaSuccess) return e;
+        const int slot = n_ < kEntries ? n_++ : (next_++ % kEntries);
+        ctx_[slot] = ctx;
+        ptr_[slot] = p;
+        *out = p;
+        return cudaSuccess;
+    }
+
+  private:
+    static constexpr int kEntries = 64;
+    struct Lock {
+        explicit Lock(SymbolAddressCache *c) : c_(c) { c_->lock(); }
+        ~Lock() { c_->unlock(); }
+        SymbolAddressCache *c_;
+    };
+    void lock() { while (busy_.test_and_set(std::memory_order_acquire)) {} }
+    void unlock() { busy_.clear(std::memory_order_release); }
+    std::atomic_flag busy_ = ATOMIC_FLAG_INIT;
+    void *ctx_[kEntries] = {};
+    void *ptr_[kEntries] = {};
+    int n_ = 0, next_ = 0;
+};
+
+// Index checks of the debug build.  With RETNET_CHECK_BOUNDS defined,
+// in_bounds(i, n, err) tests 0 <= i < n; a failed test records kDevErrBounds
+// in the error word and the caller skips the access.  Without it the test
+// is the constant true and compiles away.
+#ifdef RETNET_CHECK_BOUNDS
+__device__ __forceinline__ bool in_bounds(long long i, long long n, unsigned *err) {
+    if (i >= 0 && i < n) return true;
+    if (err) atomicOr(err, (unsigned)kDevErrBounds);
+    return false;
+}
+#else
+__device__ __forceinline__ constexpr bool in_bounds(long long, long long, unsigned *) {
+    return true;
+}
+#endif
 
 // Counts host-side kernel launches (see retnet_kernel_launch_count).
 void count_launch(unsigned n = 1);

@@ -9,41 +9,24 @@
 // scratch array compiled into this library (RETNET_NOALLOC_SCRATCH_BYTES per
 // device, held by every GPU that loads the library until the process exits)
 // and allocates nothing itself.
-#include <mutex>
-
 #include "kernels.h"
 
 // The scratch array: the stated maximum plus room to round its start up to
 // the 1024-byte boundary the tensor-core path's TMA buffers need.  In host
 // code this name is only a stand-in for the symbol, not a device address:
-// its address on a device comes from cudaGetSymbolAddress, taken once per
-// device below.
+// its address comes from cudaGetSymbolAddress, taken once per CUDA context
+// (per device, and again after a cudaDeviceReset) with that context current.
 static __device__ __align__(256) unsigned char
     g_noalloc_scratch[RETNET_NOALLOC_SCRATCH_BYTES + 1024];
 
 namespace retnet {
 namespace {
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mu;
-void *g_scratch_ptr[kMaxDevices] = {};
+SymbolAddressCache g_scratch_cache;
 
-// Device address of the scratch array on the current device; resolved once
-// per device, with that device current.
+// Device address of the scratch array in the current context.
 cudaError_t scratch_on_current_device(void **out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
-    return cudaSuccess;
+    return g_scratch_cache.get(g_noalloc_scratch, out);
 }
 
 }  // namespace

@@ -42,27 +42,58 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Wall-time limit of every pipeline wait: about 2 s.  A build with
+// RETNET_TEST_HOOKS lets a test lower it (retnet_test_set_hooks) so that
+// the timeout path can be exercised without a long stall.
+#ifdef RETNET_TEST_HOOKS
+static __device__ unsigned long long g_hook_wait_limit_ns = 2000000000ull;
+__device__ __forceinline__ uint64_t wait_limit_ns() {
+    return *(volatile unsigned long long *)&g_hook_wait_limit_ns;
+}
+#else
+__device__ __forceinline__ uint64_t wait_limit_ns() { return 2000000000ull; }
+#endif
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
 // Waits for the barrier phase with the given parity.  Gives up after
-// roughly `limit_ns` nanoseconds of wall time, or as soon as another thread
-// of the CTA has raised *abort; on giving up it records kDevErrTimeout in
-// the device error word, raises *abort and returns false.
+// wait_limit_ns() of wall time, or as soon as another thread of the CTA has
+// raised *abort; on giving up it records kDevErrTimeout in the device error
+// word, raises *abort and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
-                                          volatile int *abort, unsigned *err,
-                                          uint64_t limit_ns = 2000000000ull) {
+                                          volatile int *abort, unsigned *err) {
     if (mbar_try_wait(bar, parity)) return true;
-    uint64_t t0;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    const uint64_t t0 = global_ns();
+    const uint64_t limit_ns = wait_limit_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        uint64_t t;
-        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-        if (t - t0 > limit_ns) {
+        if (global_ns() - t0 > limit_ns) {
             if (err) atomicOr(err, (unsigned)kDevErrTimeout);
             *abort = 1;
             return false;
         }
     }
+}
+
+// Used on the way out of an aborted CTA: waits, ignoring the abort flag but
+// never longer than the pipeline limit, for a phase that this thread's own
+// asynchronous copies or MMAs will complete, so that nothing still writes
+// shared or tensor memory when the CTA frees it and exits.
+__device__ __forceinline__ bool mbar_drain(uint64_t *bar, uint32_t parity, unsigned *err) {
+    const uint64_t t0 = global_ns();
+    const uint64_t limit_ns = wait_limit_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_ns() - t0 > limit_ns) {
+            if (err) atomicOr(err, (unsigned)kDevErrTimeout);
+            return false;
+        }
+    }
+    return true;
 }
 
 // Warp-uniform wait: lane 0 polls, the result is broadcast, so every lane

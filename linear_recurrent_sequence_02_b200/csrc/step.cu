@@ -113,7 +113,7 @@ __global__ void __launch_bounds__(kStepThreads)
 retention_step_kernel(const T *__restrict__ q, const T *__restrict__ k,
                       const T *__restrict__ v, HeadGammas gam, StepRotation rot,
                       float *__restrict__ state, T *__restrict__ out, int bh0, int heads,
-                      int dv, int rotate) {
+                      int dv, int rotate, long long bh_total, unsigned *err) {
     constexpr int RPL = DK / kStepLanes;             // rows per thread: 2, 4 or 8
     const int bh = bh0 + blockIdx.y;                 // sequence * heads + head
     const int h = bh % heads;
@@ -126,6 +126,12 @@ retention_step_kernel(const T *__restrict__ q, const T *__restrict__ k,
     __shared__ float4 red[kStepThreads / 32][kStepCols / 4];
 
     grid_dependency_wait();          // the state may come from the kernel before
+#ifdef RETNET_CHECK_BOUNDS
+    // debug build: this CTA's (sequence, head) row and columns exist
+    if (!__syncthreads_and(in_bounds(bh, bh_total, err) &&
+                           in_bounds(col0 + cgi * 4 + 3, dv, err)))
+        return;
+#endif
     // Issue this thread's state loads first: they do not depend on q, k, v.
     float *S = state + (size_t)bh * DK * dv + col0 + cgi * 4;
     float4 s[RPL];
@@ -173,7 +179,8 @@ __global__ void __launch_bounds__(kStepThreads, 2)
 retention_tokens_kernel(const T *__restrict__ q, const T *__restrict__ k,
                         const T *__restrict__ v, HeadGammas gam, TokenRotation rot,
                         float *__restrict__ state, T *__restrict__ out, int bh0, int heads,
-                        int tokens, int tok0, int ntok, int dv, int rotate) {
+                        int tokens, int tok0, int ntok, int dv, int rotate, long long bh_total,
+                        unsigned *err) {
     constexpr int RPL = DK / kStepLanes;
     constexpr int kPairs = DK / 2;
     const int bh = bh0 + blockIdx.y;
@@ -188,6 +195,13 @@ retention_tokens_kernel(const T *__restrict__ q, const T *__restrict__ k,
     __shared__ float4 red[kGroup][kStepThreads / 32][kStepCols / 4];
 
     grid_dependency_wait();          // the state may come from the kernel before
+#ifdef RETNET_CHECK_BOUNDS
+    // debug build: this CTA's row, columns and tokens exist
+    if (!__syncthreads_and(in_bounds(bh, bh_total, err) &&
+                           in_bounds(col0 + cgi * 4 + 3, dv, err) &&
+                           in_bounds(tok0 + ntok - 1, tokens, err)))
+        return;
+#endif
     float *S = state + (size_t)bh * DK * dv + col0 + cgi * 4;
     float4 s[RPL];
 #pragma unroll
@@ -284,7 +298,8 @@ static cudaError_t launch_step_dk(const void *q, const void *k, const void *v,
         const dim3 grid((unsigned)(dv / kStepCols), (unsigned)std::min(65535LL, bh_total - bh0));
         const cudaError_t e = launch_overlapped(
             retention_step_kernel<T, DK>, grid, dim3(kStepThreads), 0, stream, (const T *)q,
-            (const T *)k, (const T *)v, gam, rot, state, (T *)out, (int)bh0, heads, dv, rotate);
+            (const T *)k, (const T *)v, gam, rot, state, (T *)out, (int)bh0, heads, dv, rotate,
+            bh_total, device_error_word());
         count_launch();
         if (e != cudaSuccess) return e;
     }
@@ -311,7 +326,7 @@ static cudaError_t launch_tokens_dk(const void *q, const void *k, const void *v,
             const cudaError_t e = launch_overlapped(
                 retention_tokens_kernel<T, DK>, grid, dim3(kStepThreads), 0, stream,
                 (const T *)q, (const T *)k, (const T *)v, gam, rot, state, (T *)out, (int)bh0,
-                heads, tokens, tok0, ntok, dv, rotate);
+                heads, tokens, tok0, ntok, dv, rotate, bh_total, device_error_word());
             count_launch();
             if (e != cudaSuccess) return e;
         }

@@ -21,6 +21,27 @@ def read_golden(name: str) -> dict:
     return out
 
 
+# Every parity error the tests compute, with the test and the line that
+# asked for it; conftest.py prints the worst per test at the end of the run
+# and, when RETNET_PARITY_LOG names a file, writes them all there as JSON.
+MEASURED = []
+
+
+def record(value: float, what: str = "") -> float:
+    """Keeps an achieved error (and what it measures) for the run's report."""
+    import inspect
+    caller = inspect.stack()[1]
+    frame = caller
+    for f in inspect.stack()[1:]:            # the test function's own line
+        if os.path.basename(f.filename).startswith("test_"):
+            frame = f
+            break
+    MEASURED.append({"test": os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0],
+                     "where": f"{os.path.basename(frame.filename)}:{frame.lineno}",
+                     "what": what, "err": float(value)})
+    return value
+
+
 def slice_rel_err(got, ref, head_axis: int = 2) -> float:
     """Norm-wise relative error, worst over (batch, head) slices.
 
@@ -40,5 +61,5 @@ def slice_rel_err(got, ref, head_axis: int = 2) -> float:
     den = np.abs(r).max(axis=-1)
     den = np.where(den == 0, 1.0, den)
     if not np.all(np.isfinite(g)):
-        return float("inf")
-    return float((num / den).max())
+        return record(float("inf"), "slice")
+    return record(float((num / den).max()), "slice")

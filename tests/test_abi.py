@@ -13,9 +13,20 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "retnet.h")
 
 
+_DECL = r"RETNET_API[^;(]*?\b(retnet_\w+)\s*\("
+_HOOKS_BLOCK = r"#ifdef RETNET_TEST_HOOKS(.*?)#endif"
+
+
 def declared_functions():
-    text = open(HEADER).read()
-    return sorted(set(re.findall(r"RETNET_API[^;(]*?\b(retnet_\w+)\s*\(", text)))
+    """Entry points the default library exports (the header minus the
+    debug-build-only block)."""
+    text = re.sub(_HOOKS_BLOCK, "", open(HEADER).read(), flags=re.S)
+    return sorted(set(re.findall(_DECL, text)))
+
+
+def debug_only_functions():
+    blocks = re.findall(_HOOKS_BLOCK, open(HEADER).read(), flags=re.S)
+    return sorted(set(re.findall(_DECL, "".join(blocks))))
 
 
 @pytest.fixture(scope="module")
@@ -41,6 +52,18 @@ def test_every_declared_symbol_is_exported(lib):
     out = os.popen(f"nm -D --defined-only {rn.LIB_PATH}").read()
     exported = sorted(set(re.findall(r"\b(retnet_\w+)\b", out)))
     assert exported == declared_functions()
+
+
+def test_debug_build_exports_the_test_hooks_and_nothing_else_differs(lib):
+    from linear_recurrent_sequence_02_b200.build import build
+    path = build(variant="debug")
+    hooks = debug_only_functions()
+    assert hooks == ["retnet_test_set_hooks"]
+    out = os.popen(f"nm -D --defined-only {path}").read()
+    exported = sorted(set(re.findall(r"\b(retnet_\w+)\b", out)))
+    assert exported == sorted(declared_functions() + hooks)
+    # the default library has no hook
+    assert not hasattr(lib, "retnet_test_set_hooks")
 
 
 def test_status_strings(lib):
@@ -75,6 +98,20 @@ def test_workspace_size_validation(lib):
     neg = _shape(B=-1)
     assert lib.retnet_chunkwise_workspace_size(ctypes.byref(neg), 64, 1, ctypes.byref(n)) == 1
     assert lib.retnet_chunkwise_workspace_size(None, 64, 1, ctypes.byref(n)) == 1
+
+
+def test_tensor_path_takes_short_chunks_as_128(lib):
+    # chunks below 128 run on the tensor path with 128-token chunks: the same
+    # workspace as chunk 128; 384 (not a tile multiple the path serves) does not
+    s = _shape(B=2, H=4, n=1000, dk=256, dv=256, dt=1)
+    sizes = {}
+    for chunk in (16, 64, 100, 128):
+        n = ctypes.c_size_t(0)
+        assert lib.retnet_chunkwise_workspace_size(ctypes.byref(s), chunk, 2, ctypes.byref(n)) == 0
+        sizes[chunk] = n.value
+    assert len(set(sizes.values())) == 1
+    n = ctypes.c_size_t(0)
+    assert lib.retnet_chunkwise_workspace_size(ctypes.byref(s), 384, 2, ctypes.byref(n)) == 2
 
 
 def _chunkwise(lib, q=16, k=16, v=16, out=16, gam=(0.9,) * 4, chunk=64, shape=None, pos0=0,

@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import workloads as wl
-from helpers import slice_rel_err
+from helpers import record, slice_rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -62,12 +62,13 @@ def check(rn, dtype, B, n, H, dk, dv, chunk, pos0=0, rotate=True, algo="auto", s
                                                    np.float32(gam), np.abs(do), rotate=False)
     for got, want, scale, name in ((dq, wq, scales[0], "dq"), (dk_, wk, scales[1], "dk"),
                                    (dv_, wv, scales[2], "dv")):
+        plain = slice_rel_err(host(got), want)      # recorded for the report either way
         if scale is None:
-            err = slice_rel_err(host(got), want)
+            err = plain
         else:
             diff = np.abs(host(got) - want).max(axis=(1, 3))
-            err = float((diff / np.abs(scale).max(axis=(1, 3))).max())
-        assert err < TOL[dtype], (name, err)
+            err = record(float((diff / np.abs(scale).max(axis=(1, 3))).max()), "term-scaled")
+        assert err < TOL[dtype], (name, err, plain)
 
 
 @pytest.mark.parametrize("n,chunk", [(128, 128), (700, 256), (1024, 512)])

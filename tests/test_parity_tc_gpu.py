@@ -61,7 +61,8 @@ def test_single_tile(rn):
 
 
 @pytest.mark.parametrize("n,chunk", [(256, 128), (512, 512), (300, 128), (1101, 256),
-                                     (640, 512), (2048, 1024), (77, 512)])
+                                     (640, 512), (2048, 1024), (77, 512), (300, 64),
+                                     (517, 16), (1000, 100)])
 def test_chunks_and_ragged_lengths(rn, n, chunk):
     B, H = 2, 3
     q, k, v, _ = inputs(B, n, H, 12 + n)
@@ -147,13 +148,16 @@ def test_layer_workloads_full(rn, name):
     assert slice_rel_err(st, ws, head_axis=1) < TOL
 
 
-def test_layer200m_chunk64_uses_simt(rn):
+@pytest.mark.parametrize("algo", ["tensor", "simt"])
+def test_layer200m_chunk64(rn, algo):
+    # chunk 64: the tensor path computes it with 128-token chunks (the result
+    # does not depend on the chunk length); the SIMT path uses 64 as given
     w = wl.WORKLOADS["layer200m"]
     q, k, v, g = wl.make_prefill_inputs(2, w.heads, w.seqlen, w.d, w.dtype, w.scale, w.seed,
                                         hidden=w.hidden)
     gam = rn.retnet_default_gammas(w.heads)
     want, ws = oracle.retention_prefill(q, k, v, np.float32(gam), 64, gate=g)
-    got, st = run(rn, q, k, v, gam, 64, algo="auto", gate=g)
+    got, st = run(rn, q, k, v, gam, 64, algo=algo, gate=g)
     assert slice_rel_err(got, want) < TOL
     assert slice_rel_err(st, ws, head_axis=1) < TOL
 

@@ -43,7 +43,7 @@ def _ptr(t):
 def _noalloc(lib, q, k, v, gam, chunk, out, state_out, gate, pos0=0):
     import linear_recurrent_sequence_02_b200 as rn
     B, n, H, d = q.shape
-    shape = rn._Shape(B, H, n, d, d, rn.BF16)
+    shape = rn._Shape(B, H, n, d, d, rn.BF16 if q.dtype == torch.bfloat16 else rn.F32)
     g = None if gate is None else rn._Gate(gate.data_ptr(), None, None, 1e-5)
     gbuf = (ctypes.c_float * H)(*gam)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
@@ -71,8 +71,58 @@ def test_noalloc_matches_regular_entry_point_twice(lib):
         assert _noalloc(lib, q, k, v, gam, chunk, out, state, g) == 0
         torch.cuda.synchronize()
         rn.retnet_check_device_errors()
-        assert slice_rel_err(out.float().cpu().numpy(), want.float().cpu().numpy()) < TOL
-        assert slice_rel_err(state.cpu().numpy(), want_state.cpu().numpy(), head_axis=1) < TOL
+        # the same kernels on the same inputs: the same bits
+        assert torch.equal(out, want)
+        assert torch.equal(state, want_state)
+
+
+def test_noalloc_float32_short_chunks_match_regular_entry_point(lib):
+    # the float32 CUDA-core path (chunk 64, the tiny configuration's shape)
+    # also takes its scratch from the built-in array
+    import linear_recurrent_sequence_02_b200 as rn
+    q, k, v = wl.make_prefill_inputs(1, 4, 256, 64, "f32", 1.0 / 8.0, 903)[:3]
+    q, k, v = (torch.from_numpy(x).cuda() for x in (q, k, v))
+    gam = rn.retnet_default_gammas(4)
+    want_state = torch.empty(1, 4, 64, 64, device="cuda")
+    want = rn.retnet_retention_chunkwise(q, k, v, gam, 64, state_out=want_state)
+    for _ in range(2):
+        out = torch.full_like(want, float("nan"))
+        state = torch.full_like(want_state, float("nan"))
+        assert _noalloc(lib, q, k, v, gam, 64, out, state, None) == 0
+        torch.cuda.synchronize()
+        rn.retnet_check_device_errors()
+        assert torch.equal(out, want)
+        assert torch.equal(state, want_state)
+
+
+def test_noalloc_near_its_scratch_limit(lib):
+    # the longest two-head bf16 prefill whose tensor-path scratch still fits
+    # the 32 MiB array, so the array's last bytes are in use
+    import oracle
+    import linear_recurrent_sequence_02_b200 as rn
+    B, H, d, chunk = 1, 2, 256, 512
+    limit = 32 * 1024 * 1024
+    n = 128
+    while rn.retnet_chunkwise_workspace_size(B, H, n + 128, d, d, torch.bfloat16, chunk,
+                                             "tensor") <= limit:
+        n += 128
+    need = rn.retnet_chunkwise_workspace_size(B, H, n, d, d, torch.bfloat16, chunk, "tensor")
+    assert limit - 2 * 1024 * 1024 < need <= limit
+    qn, kn, vn, gn = wl.make_prefill_inputs(B, H, n, d, "bf16", 1.0 / 16.0, 904, hidden=256)
+    q, k, v, g = (torch.from_numpy(x).to(torch.bfloat16).cuda() for x in (qn, kn, vn, gn))
+    gam = rn.retnet_default_gammas(H)
+    want_state = torch.empty(B, H, d, d, device="cuda")
+    want = rn.retnet_retention_chunkwise(q, k, v, gam, chunk, gate=g, state_out=want_state)
+    out = torch.full_like(want, float("nan"))
+    state = torch.full_like(want_state, float("nan"))
+    assert _noalloc(lib, q, k, v, gam, chunk, out, state, g) == 0
+    torch.cuda.synchronize()
+    rn.retnet_check_device_errors()
+    assert torch.equal(out, want)
+    assert torch.equal(state, want_state)
+    y_ref, s_ref = oracle.retention_prefill(qn, kn, vn, np.float32(gam), chunk, gate=gn)
+    assert slice_rel_err(out.float().cpu().numpy(), y_ref) < TOL
+    assert slice_rel_err(state.cpu().numpy(), s_ref, head_axis=1) < TOL
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(lib):
