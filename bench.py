@@ -36,6 +36,9 @@ Other modes print their own line with their own metric:
   --form parallel    the parallel form instead of the chunkwise prefill
                      (prefill only, no state, no decode step);
   --backward         the backward pass of the prefill (dq, dk, dv);
+  --layer            the multi-scale retention layer: Q/K/V/G projection
+                     GEMM, gated prefill, output projection GEMM (random
+                     weights; hidden = the workload's gate width, or H d);
   --workload decode7b [--batch B] [--tokens T]
                      decode steps (T = 1) or T-token recurrent calls from
                      states seeded by an 8192-token prefill;
@@ -892,6 +895,110 @@ def run_decode(args, w):
     print(json.dumps(line), flush=True)
 
 
+def run_layer(args, w, chunk):
+    """The multi-scale retention layer (retnet_msr_layer): Q/K/V/G projection
+    GEMM, the gated chunkwise prefill, and the output projection GEMM.  One
+    timed step = one layer pass over the workload's batch."""
+    import torch
+
+    import linear_recurrent_sequence_02_b200 as rn
+    from linear_recurrent_sequence_02_b200.build import build
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    build()
+    rn.load_library()
+    rn.retnet_set_launch_overlap(not args.no_overlap)
+    B, n, H, d = w.batch, w.seqlen, w.heads, w.d
+    hidden = w.hidden or H * d
+    gam = rn.retnet_default_gammas(H)
+    sets = []
+    for i in range(3):                                # rotating inputs
+        x, wqkvg, wo = wl.make_msr_inputs(B, n, hidden, H, d, w.seed + 17 * i)
+        sets.append(tuple(torch.from_numpy(a).to(torch.bfloat16).to(dev)
+                          for a in (x, wqkvg, wo)))
+    y = torch.empty(B, n, hidden, dtype=torch.bfloat16, device=dev)
+    st = torch.empty(B, H, d, d, device=dev)
+    ws = rn.retnet_workspace(rn.retnet_msr_workspace_size(B, H, n, d, hidden, chunk), dev)
+
+    def step(i):
+        x, wqkvg, wo = sets[i % 3]
+        rn.retnet_msr_layer(x, wqkvg, wo, gam, chunk, state_out=st, out=y, workspace=ws)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    rn.retnet_profiler_reset()
+    rn.retnet_profiler_select(None)
+    rn.retnet_profiler_enable(True)
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize()
+    rn.retnet_profiler_enable(False)
+    kern = rn.retnet_profiler_read()
+    rn.retnet_check_device_errors(dev)
+    launches0 = rn.retnet_kernel_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(args.steps):
+            step(i)
+    launches = rn.retnet_kernel_launch_count() - launches0
+    graph.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index or 0)
+    clocks.start()
+    ev0.record(stream)
+    graph.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    del graph
+    rn.retnet_check_device_errors(dev)
+    peaks, src = load_peaks()
+    rows = B * n
+    gemm_flops = {"gemm_qkvg": 2 * rows * 4 * H * d * hidden,
+                  "gemm_out": 2 * rows * hidden * H * d}
+    gemms = {}
+    for name, fl in gemm_flops.items():
+        if name in kern:
+            tot, cnt = kern[name]
+            avg_s = tot / cnt / 1e3
+            gemms[name] = {"avg_us": avg_s * 1e6, "achieved": fl / avg_s / 1e12,
+                           "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                           "frac": fl / avg_s / 1e12 / peaks["bf16_tflops"],
+                           "work_per_launch": fl}
+    step_s = ms / args.steps / 1e3
+    total_kern = sum(v[0] for v in kern.values())
+    alg = sum(gemm_flops.values()) + algorithmic_flops_per_token_head(d, chunk) * rows * H
+    line = {
+        "metric": "MSR layer tokens/s (Q/K/V/G projection, gated chunkwise retention, "
+                  "output projection)",
+        "value": rows / step_s, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{w.name} MSR layer: B={B} n={n} hidden={hidden} H={H} d={d} "
+                               f"chunk {chunk}, random weights",
+                   "batch": B, "seqlen": n, "hidden": hidden, "heads": H, "d": d,
+                   "chunk": chunk,
+                   "l2": "3 rotating input sets; the five [B n, H d] intermediates of a step "
+                         "exceed L2"},
+        "roofline": dict(gemms.get("gemm_qkvg", {}), kernel="gemm_qkvg", bound="tensor",
+                         peak_source=src, traffic=None),
+        "gemms": gemms,
+        "tflops_algorithmic": alg / step_s / 1e12,
+        "frac_of_bf16_peak": alg / step_s / 1e12 / peaks["bf16_tflops"],
+        "kernels": {k: {"avg_us": 1e3 * v[0] / v[1], "launches_per_step": v[1] / 3,
+                        "share": v[0] / max(total_kern, 1e-12)} for k, v in kern.items()},
+        "gpu_launches": launches, "clocks": clock_info, "peak_source": src,
+        "timing": "one replay of a CUDA graph holding the K timed steps; 'kernels' are 3 "
+                  "steps with every kernel bracketed by events",
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -915,6 +1022,8 @@ def main():
                     help="time the backward pass of the prefill (no epilogue) instead")
     ap.add_argument("--no-overlap", action="store_true",
                     help="launch kernels without programmatic launch overlap")
+    ap.add_argument("--layer", action="store_true",
+                    help="time the whole multi-scale retention layer (projections included)")
     ap.add_argument("--form", choices=["chunkwise", "parallel"], default="chunkwise",
                     help="prefill form; 'parallel' times the parallel form alone (no decode)")
     args = ap.parse_args()
@@ -931,6 +1040,8 @@ def main():
         run_decode(args, w)
     elif args.backward:
         run_backward(args, w, chunk)
+    elif args.layer:
+        run_layer(args, w, chunk)
     else:
         run_ours(args, w, chunk)
 

@@ -295,6 +295,50 @@ RETNET_API retnet_status retnet_groupnorm_swish(const void *o, const void *g, co
                                      int dv, retnet_dtype dtype, void *y,
                                      retnet_stream_t stream);
 
+/* ---- The multi-scale retention layer ----------------------------------
+ * Retention replaces multi-head attention, with a swish gate and GroupNorm
+ * added on its output ("Summary"); around the operator the layer projects
+ * its input and output with dense weights.  Both projections run on a
+ * tcgen05 GEMM of this library (TMA-fed, bf16 operands, float32
+ * accumulation, bf16 result).
+ *
+ * retnet_linear: y[r, :] = x[r, :] W^T for r < rows.
+ *   x  device bf16 [rows, in_features]; w device bf16 [out_features,
+ *      in_features] (a linear layer's weight layout); y device bf16
+ *      [rows, out_features], not overlapping x or w.
+ *   in_features must be a multiple of 64 and out_features of 256, else
+ *   UNSUPPORTED.  Errors: INVALID_ARG (null or misaligned pointers,
+ *   negative sizes), UNSUPPORTED, CUDA. */
+RETNET_API retnet_status retnet_linear(const void *x, const void *w, void *y, long long rows,
+                                       int in_features, int out_features,
+                                       retnet_stream_t stream);
+
+/* retnet_msr_layer: for x [batch, seqlen, hidden] (bf16, shape->dtype must
+ * be RETNET_BF16 and dk = dv = d):
+ *     q, k, v, g = x W_Q^T, x W_K^T, x W_V^T, x W_G^T      ([B, n, H, d] each)
+ *     o = swish(g) (.) GroupNorm(retention(R q, R k, v))     (as
+ *         retnet_retention_chunkwise with this gate, chunk, pos0, rotate = 1,
+ *         state_in, state_out and algo AUTO)
+ *     y = o W_O^T                                          ([B, n, hidden])
+ *   w_qkvg  device bf16 [4 H d, hidden]: the rows of W_Q, then W_K, W_V, W_G.
+ *   w_o     device bf16 [hidden, H d].
+ *   gn_weight, gn_bias  device float32 [H d] GroupNorm affine, or NULL.
+ *   workspace  retnet_msr_workspace_size() bytes, 1024-byte aligned.
+ *   hidden must be a multiple of 256 and H d a multiple of 256, else
+ *   UNSUPPORTED.  y must not overlap x, the weights, the states or the
+ *   workspace.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+RETNET_API retnet_status retnet_msr_workspace_size(const retnet_shape *shape, int hidden,
+                                                   int chunk, size_t *bytes);
+RETNET_API retnet_status retnet_msr_layer(const void *x, const void *w_qkvg, const void *w_o,
+                                          const float *gammas, int chunk, void *y,
+                                          const retnet_shape *shape, int hidden,
+                                          long long pos0, const float *gn_weight,
+                                          const float *gn_bias, float eps,
+                                          const float *state_in, float *state_out,
+                                          void *workspace, size_t workspace_bytes,
+                                          retnet_stream_t stream);
+
 /* Reads and clears the library's device-side error word on the current
  * device after synchronising `stream`.  Returns RETNET_OK when no kernel
  * reported a problem, RETNET_ERR_TIMEOUT when a bounded wait inside a

@@ -31,6 +31,7 @@ __all__ = [
     "retnet_profiler_reset",
     "retnet_profiler_read", "ALGO_AUTO", "ALGO_SIMT", "ALGO_TENSOR", "LIB_PATH",
     "DEBUG_LIB_PATH", "using_library", "retnet_test_set_hooks",
+    "retnet_linear", "retnet_msr_workspace_size", "retnet_msr_layer",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libretnet.so")
@@ -95,6 +96,10 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "retnet_retention_backward": (i, [vp, vp, vp, vp, vp, i, vp, vp, vp,
                                           ctypes.POINTER(_Shape), ll, i, i, vp, sz, vp]),
         "retnet_groupnorm_swish": (i, [vp, vp, vp, vp, f, ll, i, i, i, vp, vp]),
+        "retnet_linear": (i, [vp, vp, vp, ll, i, i, vp]),
+        "retnet_msr_workspace_size": (i, [ctypes.POINTER(_Shape), i, i, ctypes.POINTER(sz)]),
+        "retnet_msr_layer": (i, [vp, vp, vp, vp, i, vp, ctypes.POINTER(_Shape), i, ll, vp, vp,
+                                 f, vp, vp, vp, sz, vp]),
         "retnet_check_device_errors": (i, [vp]),
         "retnet_profiler_enable": (i, [i]),
         "retnet_profiler_select": (i, [ctypes.c_char_p]),
@@ -449,6 +454,75 @@ def retnet_groupnorm_swish(o: torch.Tensor, g: torch.Tensor, weight: Optional[to
             _ptr(o), _ptr(g), _ptr(weight), _ptr(bias), float(eps), rows, H, dv, _dtype_code(o),
             _ptr(out), _stream(o))
     _check("retnet_groupnorm_swish", st)
+    return out
+
+
+def retnet_linear(x: torch.Tensor, w: torch.Tensor,
+                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y = x W^T on the tensor cores: x [..., in] bf16, w [out, in] bf16."""
+    _dev(x, "x", torch.bfloat16)
+    _dev(w, "w", torch.bfloat16)
+    if w.dim() != 2 or x.shape[-1] != w.shape[1]:
+        raise ValueError("need x [..., in] and w [out, in]")
+    rows = x.numel() // x.shape[-1] if x.numel() else 0
+    oshape = (*x.shape[:-1], w.shape[0])
+    out = torch.empty(oshape, dtype=torch.bfloat16, device=x.device) if out is None else \
+        _dev(out, "out", torch.bfloat16, oshape)
+    with torch.cuda.device(x.device):
+        st = load_library().retnet_linear(_ptr(x), _ptr(w), _ptr(out), rows, x.shape[-1],
+                                          w.shape[0], _stream(x))
+    _check("retnet_linear", st)
+    return out
+
+
+def retnet_msr_workspace_size(batch: int, heads: int, seqlen: int, d: int, hidden: int,
+                              chunk: int) -> int:
+    shape = _Shape(batch, heads, seqlen, d, d, BF16)
+    n = ctypes.c_size_t(0)
+    _check("retnet_msr_workspace_size",
+           load_library().retnet_msr_workspace_size(ctypes.byref(shape), int(hidden), int(chunk),
+                                                    ctypes.byref(n)))
+    return int(n.value)
+
+
+def retnet_msr_layer(x: torch.Tensor, w_qkvg: torch.Tensor, w_o: torch.Tensor,
+                     gammas: Sequence[float], chunk: int, *, pos0: int = 0,
+                     weight: Optional[torch.Tensor] = None, bias: Optional[torch.Tensor] = None,
+                     eps: float = 1e-5, state_in: Optional[torch.Tensor] = None,
+                     state_out: Optional[torch.Tensor] = None,
+                     out: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The multi-scale retention layer on x [batch, seqlen, hidden] (bf16):
+    projections by w_qkvg [4 H d, hidden] (rows of W_Q, W_K, W_V, W_G), the
+    gated chunkwise retention, and the output projection w_o [hidden, H d].
+    H = len(gammas).  Returns out [batch, seqlen, hidden]."""
+    _dev(x, "x", torch.bfloat16)
+    if x.dim() != 3:
+        raise ValueError("x must be [batch, seqlen, hidden]")
+    B, n, hidden = x.shape
+    H = len(gammas)
+    if w_qkvg.dim() != 2 or w_qkvg.shape[0] % (4 * H) or w_qkvg.shape[1] != hidden:
+        raise ValueError("w_qkvg must be [4 * heads * d, hidden]")
+    d = w_qkvg.shape[0] // (4 * H)
+    _dev(w_qkvg, "w_qkvg", torch.bfloat16)
+    _dev(w_o, "w_o", torch.bfloat16, (hidden, H * d))
+    _dev(weight, "weight", torch.float32, (H * d,))
+    _dev(bias, "bias", torch.float32, (H * d,))
+    _dev(state_in, "state_in", torch.float32, (B, H, d, d))
+    _dev(state_out, "state_out", torch.float32, (B, H, d, d))
+    out = torch.empty_like(x) if out is None else _dev(out, "out", torch.bfloat16, x.shape)
+    need = retnet_msr_workspace_size(B, H, n, d, hidden, chunk)
+    if workspace is None:
+        workspace = retnet_workspace(need, x.device)
+    else:
+        _dev(workspace, "workspace", torch.uint8)
+    shape = _Shape(B, H, n, d, d, BF16)
+    with torch.cuda.device(x.device):
+        st = load_library().retnet_msr_layer(
+            _ptr(x), _ptr(w_qkvg), _ptr(w_o), _gammas(gammas, H), int(chunk), _ptr(out),
+            ctypes.byref(shape), int(hidden), int(pos0), _ptr(weight), _ptr(bias), float(eps),
+            _ptr(state_in), _ptr(state_out), _ptr(workspace), workspace.numel(), _stream(x))
+    _check("retnet_msr_layer", st)
     return out
 
 

@@ -835,8 +835,8 @@ static EncodeTiledFn encode_fn() {
 }
 
 // bf16 tensor map, 128-byte swizzle, innermost dimension first.
-static bool make_map(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims,
-                     const cuuint64_t *strides_bytes, const cuuint32_t *box) {
+bool make_tensor_map_bf16(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims,
+                          const cuuint64_t *strides_bytes, const cuuint32_t *box) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint32_t estr[5] = {1, 1, 1, 1, 1};
@@ -943,20 +943,20 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
         cuuint64_t dims[3] = {kD, (cuuint64_t)n, (cuuint64_t)BH};
         cuuint64_t str[2] = {kD * 2, (cuuint64_t)n * kD * 2};
         cuuint32_t box[3] = {64, kBlk, 1};
-        if (!make_map(&tm_k, kt, 3, dims, str, box) || !make_map(&tm_q, qt, 3, dims, str, box))
+        if (!make_tensor_map_bf16(&tm_k, kt, 3, dims, str, box) || !make_tensor_map_bf16(&tm_q, qt, 3, dims, str, box))
             return cudaErrorInvalidValue;
     }
     {
         cuuint64_t dims[4] = {kD, (cuuint64_t)H, (cuuint64_t)n, (cuuint64_t)B};
         cuuint64_t str[3] = {kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)n * H * kD * 2};
         cuuint32_t box[4] = {64, 1, kBlk, 1};
-        if (!make_map(&tm_v, a.v, 4, dims, str, box)) return cudaErrorInvalidValue;
+        if (!make_tensor_map_bf16(&tm_v, a.v, 4, dims, str, box)) return cudaErrorInvalidValue;
     }
     {
         cuuint64_t dims[2] = {kD, (cuuint64_t)BH * nchunks * kD};
         cuuint64_t str[1] = {kD * 2};
         cuuint32_t box[2] = {64, kBlk};
-        if (!make_map(&tm_s, sp, 2, dims, str, box)) return cudaErrorInvalidValue;
+        if (!make_tensor_map_bf16(&tm_s, sp, 2, dims, str, box)) return cudaErrorInvalidValue;
     }
     // output and gate tiles: 128 tokens x 64 channels of one head
     CUtensorMap tm_out, tm_g;
@@ -964,8 +964,8 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
         cuuint64_t dims[4] = {kD, (cuuint64_t)H, (cuuint64_t)n, (cuuint64_t)B};
         cuuint64_t str[3] = {kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)n * H * kD * 2};
         cuuint32_t box[4] = {64, 1, kBlk, 1};
-        if (!make_map(&tm_out, a.out, 4, dims, str, box)) return cudaErrorInvalidValue;
-        if (!make_map(&tm_g, a.gate ? a.gate->g : a.out, 4, dims, str, box))
+        if (!make_tensor_map_bf16(&tm_out, a.out, 4, dims, str, box)) return cudaErrorInvalidValue;
+        if (!make_tensor_map_bf16(&tm_g, a.gate ? a.gate->g : a.out, 4, dims, str, box))
             return cudaErrorInvalidValue;
     }
 

@@ -1,0 +1,270 @@
+// Dense projection GEMM on the sm_100a tensor cores: Y = X W^T.
+//
+// Multi-scale retention replaces multi-head attention inside the RetNet
+// block, with the swish gate and GroupNorm on its output (RetNet research
+// summary, "Summary"); the layer around the retention operator projects the
+// input X to Q, K, V and the gate G, and projects the gated output back with
+// W_O.  Those projections are plain GEMMs: this kernel serves them.
+//
+//   X [M, K] bf16 row-major (K contiguous), W [N, K] bf16 row-major (the
+//   [out_features, in_features] layout of a linear layer's weight), Y bf16
+//   [M, N] with f32 accumulation.  The N columns may be split into up to
+//   four outputs of `n_split` columns each (the fused Q/K/V/G projection
+//   writes four dense [M, H*d] tensors).
+//
+// Persistent: one CTA per SM walks 128 x 256 output tiles in a grouped
+// raster (16 row blocks at a time, so neighbouring CTAs share X and W tiles
+// through L2).  Warp 0 streams 128 x 64 X and 256 x 64 W sub-tiles by TMA
+// (128-byte swizzle) through a four-stage ring; warp 1 issues
+// tcgen05.mma (M = 128, N = 256, K = 16, both operands K-major) into one of
+// two TMEM accumulators (2 x 256 columns); warps 2-5 read the finished
+// accumulator, round to bf16 and store, while the MMAs of the next tile run
+// into the other accumulator.  Every wait is bounded (about 2 s); on
+// timeout the CTA records kDevErrTimeout, lets its own loads and MMAs
+// finish, frees its tensor memory and returns.
+#include <algorithm>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace retnet {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kGemmM = 128;                 // rows of X per tile (TMEM lanes)
+constexpr int kGemmN = 256;                 // columns of Y per tile (TMEM columns)
+constexpr int kGemmK = 64;                  // K per stage: one 128-byte swizzle row
+constexpr int kGemmStages = 4;
+constexpr uint32_t kGemmABytes = kGemmM * kGemmK * 2;        // 16 KB
+constexpr uint32_t kGemmBBytes = kGemmN * kGemmK * 2;        // 32 KB
+constexpr uint32_t kGemmStage = kGemmABytes + kGemmBBytes;   // 48 KB
+constexpr uint32_t kGemmSmem = kGemmStages * kGemmStage + 1024;
+constexpr int kGemmThreads = 192;           // 6 warps
+constexpr int kGemmGroup = 16;              // row blocks per raster group
+
+struct GemmArgs {
+    __nv_bfloat16 *out[4];
+    long long m;                            // rows
+    int n, k;                               // columns of Y, reduction length
+    int n_split;                            // columns per output
+    int tiles_m, tiles_n;
+    unsigned *err;
+};
+
+__device__ __forceinline__ void gemm_tile(const GemmArgs &a, int t, int &mb, int &nb) {
+    const int per_group = kGemmGroup * a.tiles_n;
+    const int g = t / per_group, r = t % per_group;
+    const int m0 = g * kGemmGroup;
+    const int gm = min(kGemmGroup, a.tiles_m - m0);
+    mb = m0 + r % gm;
+    nb = r / gm;
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+gemm_bf16_tn_kernel(const __grid_constant__ CUtensorMap tm_x,
+                    const __grid_constant__ CUtensorMap tm_w, GemmArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    __shared__ uint64_t full[kGemmStages], empty[kGemmStages], acc_full[2], acc_free[2], drain;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int abort_flag;
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    unsigned *err = a.err;
+    const int tiles = a.tiles_m * a.tiles_n;
+    const int ksteps = (a.k + kGemmK - 1) / kGemmK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kGemmStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&acc_full[x], 1);
+            mbar_init(&acc_free[x], 128);
+        }
+        mbar_init(&drain, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_slot, 512);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_w);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+    grid_dependency_wait();                         // X may come from the kernel before
+
+    int pit = 0;                                    // producer: stages issued
+    if (warp == 0) {
+        if (lane == 0) {
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
+                int mb, nb;
+                gemm_tile(a, t, mb, nb);
+                for (int ks = 0; ks < ksteps; ++ks, ++pit) {
+                    const int s = pit % kGemmStages;
+                    if (pit >= kGemmStages &&
+                        !mbar_wait(&empty[s], ((pit / kGemmStages) - 1) & 1, &abort_flag, err)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *ab = smem + s * kGemmStage;
+                    mbar_expect_tx(&full[s], kGemmStage);
+                    tma_load_2d(ab, &tm_x, &full[s], ks * kGemmK, mb * kGemmM);
+                    tma_load_2d(ab + kGemmABytes, &tm_w, &full[s], ks * kGemmK, nb * kGemmN);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(kGemmM, kGemmN, 0, 0);
+            int it = 0, lt = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++lt) {
+                const int buf = lt & 1;
+                if (lt >= 2 && !mbar_wait(&acc_free[buf], ((lt - 2) >> 1) & 1, &abort_flag, err))
+                    break;
+                tc_fence_after();
+                for (int ks = 0; ks < ksteps; ++ks, ++it) {
+                    const int s = it % kGemmStages;
+                    if (!mbar_wait(&full[s], (it / kGemmStages) & 1, &abort_flag, err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t ab = smem_u32(smem + s * kGemmStage);
+                    const uint32_t bb = ab + kGemmABytes;
+#pragma unroll
+                    for (int kk = 0; kk < kGemmK / 16; ++kk)
+                        mma_bf16(tmem + kGemmN * buf, smem_desc_sw128(ab + kk * 32, 16, 1024),
+                                 smem_desc_sw128(bb + kk * 32, 16, 1024), idesc,
+                                 (ks > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(&empty[s]);
+                }
+                if (ok) mma_commit(&acc_full[buf]);
+            }
+        }
+    } else {
+        // epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 = rows of the tile
+        const int q4 = warp % 4;
+        const int row = 32 * q4 + lane;
+        const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
+        int lt = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++lt) {
+            const int buf = lt & 1;
+            if (!warp_wait(&acc_full[buf], (lt >> 1) & 1, &abort_flag, err)) break;
+            tc_fence_after();
+            int mb, nb;
+            gemm_tile(a, t, mb, nb);
+            const long long grow = (long long)mb * kGemmM + row;
+            const int col0 = nb * kGemmN;
+            const int which = col0 / a.n_split;
+            const int c_in = col0 % a.n_split;
+            const bool live = grow < a.m && in_bounds(which, 4, err);
+            // (a select chain, not a dynamic index, keeps a.out out of local memory)
+            __nv_bfloat16 *base = which == 0   ? a.out[0]
+                                  : which == 1 ? a.out[1]
+                                  : which == 2 ? a.out[2]
+                                               : a.out[3];
+            __nv_bfloat16 *dst = live ? base + grow * a.n_split + c_in : nullptr;
+#pragma unroll 1
+            for (int cb = 0; cb < kGemmN / 32; ++cb) {
+                uint32_t v[32];
+                tmem_ld32(tmem + kGemmN * buf + lane_off + 32 * cb, v);
+                tmem_wait_ld();
+                if (cb == kGemmN / 32 - 1) {             // accumulator fully read
+                    tc_fence_before();
+                    mbar_arrive(&acc_free[buf]);
+                }
+                if (live) {
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * cb);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        d4[q] = make_uint4(
+                            pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                            pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                            pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                            pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    // Every role has finished, so abort_flag is final.  After an abort, wait
+    // (bounded) for the loads still in flight (at most the last kGemmStages
+    // issued) and for the MMAs before freeing shared and tensor memory.
+    if (abort_flag && warp == 0 && lane == 0)
+        for (int j = max(0, pit - kGemmStages); j < pit; ++j)
+            mbar_drain(&full[j % kGemmStages], (j / kGemmStages) & 1, err);
+    if (warp == 1) {
+        if (abort_flag && lane == 0) {
+            mma_commit(&drain);
+            mbar_drain(&drain, 0, err);
+        }
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace
+
+bool gemm_shape_ok(long long m, int n, int k, int n_split) {
+    if (m < 0 || n <= 0 || k <= 0 || k % kGemmK != 0 || n % kGemmN != 0) return false;
+    if (n_split <= 0 || n_split % kGemmN != 0 || n % n_split != 0 || n / n_split > 4) return false;
+    const long long tiles = (m + kGemmM - 1) / kGemmM * (long long)(n / kGemmN);
+    return tiles < (1LL << 31);
+}
+
+cudaError_t launch_gemm_bf16(const void *x, const void *w, void *const *outs, long long m, int n,
+                             int k, int n_split, cudaStream_t stream, const char *timer_name) {
+    if (m == 0) return cudaSuccess;
+    CUtensorMap tm_x, tm_w;
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)k, (cuuint64_t)m};
+        cuuint64_t str[1] = {(cuuint64_t)k * 2};
+        cuuint32_t box[2] = {kGemmK, kGemmM};
+        if (!make_tensor_map_bf16(&tm_x, x, 2, dims, str, box)) return cudaErrorInvalidValue;
+    }
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)k, (cuuint64_t)n};
+        cuuint64_t str[1] = {(cuuint64_t)k * 2};
+        cuuint32_t box[2] = {kGemmK, kGemmN};
+        if (!make_tensor_map_bf16(&tm_w, w, 2, dims, str, box)) return cudaErrorInvalidValue;
+    }
+    GemmArgs a;
+    for (int i = 0; i < 4; ++i) a.out[i] = i < n / n_split ? (__nv_bfloat16 *)outs[i] : nullptr;
+    a.m = m;
+    a.n = n;
+    a.k = k;
+    a.n_split = n_split;
+    a.tiles_m = (int)((m + kGemmM - 1) / kGemmM);
+    a.tiles_n = n / kGemmN;
+    a.err = device_error_word();
+    if (!a.err) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tn_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long tiles = (long long)a.tiles_m * a.tiles_n;
+    const unsigned grid = (unsigned)std::min<long long>(tiles, sms);
+    KernelTimer timer(timer_name, stream);
+    e = launch_overlapped(gemm_bf16_tn_kernel, dim3(grid), dim3(kGemmThreads), kGemmSmem, stream,
+                          tm_x, tm_w, a);
+    count_launch();
+    return e;
+}
+
+}  // namespace retnet

@@ -1,6 +1,8 @@
 // Internal launcher declarations shared between api.cu and the kernel files.
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace retnet {
@@ -72,5 +74,18 @@ size_t tc_workspace_bytes(int batch, int heads, int seqlen, int chunk);
 cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cudaStream_t stream,
                                 bool parallel = false);
 size_t tc_parallel_workspace_bytes(int batch, int heads, int seqlen);
+// Tensor map of a bf16 tensor for TMA (128-byte swizzle), innermost
+// dimension first; false if the driver rejects it.
+bool make_tensor_map_bf16(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims,
+                          const cuuint64_t *strides_bytes, const cuuint32_t *box);
+
+// gemm_tc.cu ---------------------------------------------------------------
+// Y = X W^T on the tensor cores: X [m, k], W [n, k], bf16, f32 accumulation.
+// Columns [j n_split, (j+1) n_split) of Y go to outs[j] ([m, n_split], dense).
+// timer_name: the kernel timer's name for this launch (a string literal).
+bool gemm_shape_ok(long long m, int n, int k, int n_split);
+cudaError_t launch_gemm_bf16(const void *x, const void *w, void *const *outs, long long m, int n,
+                             int k, int n_split, cudaStream_t stream,
+                             const char *timer_name = "gemm");
 
 }  // namespace retnet

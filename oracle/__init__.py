@@ -18,4 +18,6 @@ from .retention import (  # noqa: F401
     retention_parallel_backward,
     xpos_rotate_backward,
     retention_prefill_backward,
+    linear,
+    msr_layer,
 )

@@ -312,3 +312,33 @@ def retention_prefill(q, k, v, gammas, chunk: int, pos0: int = 0, rotate: bool =
     if gate is not None:
         o = groupnorm_swish(o, gate, weight, bias, eps)
     return o, state
+
+
+# --------------------------------------------------------------------------
+# The multi-scale retention layer  ([SUM] "Summary": retention replaces
+# multi-head attention; a swish gate and GroupNorm are added.  "Key points":
+# the 200M models have hidden size 1024.)  The input is projected to the
+# queries, keys, values and the gate input by dense weights, and the gated,
+# normalised retention output is projected back.
+# --------------------------------------------------------------------------
+def linear(x, w):
+    """y = x W^T: x [..., in], w [out, in] (a linear layer's weight)."""
+    return _f64(x) @ _f64(w).T
+
+
+def msr_layer(x, w_q, w_k, w_v, w_g, w_o, gammas, chunk: int, pos0: int = 0,
+              state_in=None, weight=None, bias=None, eps: float = 1e-5):
+    """x [B, n, hidden]; w_q, w_k, w_v, w_g [H d, hidden]; w_o [hidden, H d].
+
+    q, k, v, g = x W_q^T, x W_k^T, x W_v^T, x W_g^T (reshaped [B, n, H, d]);
+    y = swish(g) (.) GroupNorm(retention(R q, R k, v)) as retention_prefill
+    computes it; returns (y W_o^T [B, n, hidden], final state).
+    """
+    x = _f64(x)
+    B, n, _ = x.shape
+    H = len(gammas)
+    d = w_q.shape[0] // H
+    q, k, v, g = (linear(x, w).reshape(B, n, H, d) for w in (w_q, w_k, w_v, w_g))
+    y, state = retention_prefill(q, k, v, gammas, chunk, pos0=pos0, state_in=state_in, gate=g,
+                                 weight=weight, bias=bias, eps=eps)
+    return linear(y.reshape(B, n, H * d), w_o), state

@@ -297,3 +297,41 @@ def test_bench_work_counts_match_the_formulas():
     assert bench.output_kernel_flops_per_token_head(d, C) == 2 * d * (C + 1) + 2 * d * d
     assert bench.state_kernel_flops_per_token_head(d) == 2 * d * d
     assert bench.parallel_flops_per_token_head(d, 2047) == 2 * d * 2048
+
+
+def test_linear_and_msr_layer_reject_before_launch(lib):
+    P = ctypes.c_void_p
+    # retnet_linear(x, w, y, rows, in, out, stream)
+    assert lib.retnet_linear(None, P(1024), P(1024), 100, 1024, 512, None) == 1
+    assert lib.retnet_linear(P(1024), P(1024), P(24), 100, 1024, 512, None) == 1   # misaligned
+    assert lib.retnet_linear(P(1024), P(1024), P(1024), -1, 1024, 512, None) == 1
+    assert lib.retnet_linear(P(1024), P(1024), P(1024), 100, 1000, 512, None) == 2  # K % 64
+    assert lib.retnet_linear(P(1024), P(1024), P(1024), 100, 1024, 300, None) == 2  # N % 256
+    assert lib.retnet_linear(None, None, None, 0, 1024, 512, None) == 0             # no rows
+    n = ctypes.c_size_t(0)
+    s = _shape(B=2, H=4, n=300, dk=256, dv=256, dt=1)
+    assert lib.retnet_msr_workspace_size(ctypes.byref(s), 1024, 512, ctypes.byref(n)) == 0
+    assert n.value >= 5 * 600 * 1024 * 2
+    assert lib.retnet_msr_workspace_size(ctypes.byref(s), 1000, 512, ctypes.byref(n)) == 2
+    f32 = _shape(B=2, H=4, n=300, dk=256, dv=256, dt=0)
+    assert lib.retnet_msr_workspace_size(ctypes.byref(f32), 1024, 512, ctypes.byref(n)) == 2
+    uneq = _shape(B=2, H=4, n=300, dk=256, dv=128, dt=1)
+    assert lib.retnet_msr_workspace_size(ctypes.byref(uneq), 1024, 512, ctypes.byref(n)) == 2
+    assert lib.retnet_msr_workspace_size(ctypes.byref(s), 1024, 512, None) == 1
+    g4 = (ctypes.c_float * 4)(0.9, 0.9, 0.9, 0.9)
+    bad = (ctypes.c_float * 4)(0.9, 1.5, 0.9, 0.9)
+
+    def call(x=1024, y=1024, gam=g4, pos0=0, eps=1e-5, ws=1024, wsb=1 << 40, hidden=1024):
+        return lib.retnet_msr_layer(P(x), P(1024), P(1024), gam, 512, P(y), ctypes.byref(s),
+                                    hidden, pos0, None, None, eps, None, None, P(ws), wsb, None)
+
+    assert call(x=None) == 1
+    assert call(y=8) == 1
+    assert call(gam=None) == 1
+    assert call(gam=bad) == 1
+    assert call(pos0=-1) == 1
+    assert call(eps=-1.0) == 1
+    assert call(hidden=100) == 2
+    assert call(ws=None) == 5
+    assert call(wsb=1024) == 5
+    assert call(ws=1024 + 256) == 5

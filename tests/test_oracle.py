@@ -369,3 +369,71 @@ def test_backward_matches_finite_differences_on_random_cases(n, d, seed, g, pos0
     got = oracle.retention_prefill_backward(q, k, v, [g], w, pos0=pos0)
     for g_fd, g_an in zip(fd, got):
         assert np.allclose(g_an, g_fd, rtol=1e-5, atol=1e-6)
+
+
+# ------------------------------------------------------------ the MSR layer
+def test_linear_hand_worked_example():
+    g = read_golden("linear_2x3x2.txt")
+    y = oracle.linear(g["x"].reshape(2, 3), g["w"].reshape(2, 3))
+    np.testing.assert_array_equal(y, g["y"].reshape(2, 2))
+
+
+def test_linear_against_scalar_loops_and_identity():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((3, 4, 5))
+    w = rng.standard_normal((6, 5))
+    y = oracle.linear(x, w)
+    want = np.zeros((3, 4, 6))
+    for a in range(3):
+        for b in range(4):
+            for o in range(6):
+                for i in range(5):
+                    want[a, b, o] += x[a, b, i] * w[o, i]
+    np.testing.assert_allclose(y, want, rtol=1e-13, atol=1e-13)
+    np.testing.assert_array_equal(oracle.linear(x, np.eye(5)), x)
+
+
+def test_msr_layer_wiring_against_per_head_loops():
+    # every projection written out per token and head by scalar loops, then the
+    # already pinned prefill and a per-token output projection
+    rng = np.random.default_rng(6)
+    B, n, H, d, hidden = 2, 5, 2, 4, 6
+    x = rng.standard_normal((B, n, hidden))
+    ws = [rng.standard_normal((H * d, hidden)) * 0.3 for _ in range(4)]
+    w_o = rng.standard_normal((hidden, H * d)) * 0.3
+    gam = np.array([0.9, 0.6])
+    got, st = oracle.msr_layer(x, *ws, w_o, gam, chunk=2, pos0=3)
+
+    proj = []
+    for w in ws:
+        p = np.zeros((B, n, H, d))
+        for b in range(B):
+            for t in range(n):
+                for h in range(H):
+                    for j in range(d):
+                        p[b, t, h, j] = sum(x[b, t, i] * w[h * d + j, i] for i in range(hidden))
+        proj.append(p)
+    q, k, v, g = proj
+    o = oracle.retention_recurrent(oracle.xpos_rotate(q, 3), oracle.xpos_rotate(k, 3), v, gam)[0]
+    y = oracle.groupnorm_swish(o, g)
+    want = np.zeros((B, n, hidden))
+    for b in range(B):
+        for t in range(n):
+            for c in range(hidden):
+                want[b, t, c] = sum(y[b, t, h, j] * w_o[c, h * d + j]
+                                    for h in range(H) for j in range(d))
+    np.testing.assert_allclose(got, want, rtol=1e-10, atol=1e-12)
+    _, want_state = oracle.retention_prefill(q, k, v, gam, 2, pos0=3, gate=g)
+    np.testing.assert_allclose(st, want_state, rtol=1e-12, atol=1e-14)
+
+
+def test_msr_layer_with_identity_weights_is_the_gated_prefill():
+    rng = np.random.default_rng(7)
+    B, n, H, d = 1, 6, 2, 4
+    x = rng.standard_normal((B, n, H * d))
+    eye = np.eye(H * d)
+    gam = np.array([0.8, 0.95])
+    got, _ = oracle.msr_layer(x, eye, eye, eye, eye, eye, gam, chunk=4)
+    xs = x.reshape(B, n, H, d)
+    want, _ = oracle.retention_prefill(xs, xs, xs, gam, 4, gate=xs)
+    np.testing.assert_allclose(got, want.reshape(B, n, H * d), rtol=1e-12, atol=1e-14)

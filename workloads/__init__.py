@@ -28,7 +28,7 @@ from dataclasses import dataclass, field
 import numpy as np
 
 __all__ = ["Workload", "WORKLOADS", "round_to_bf16", "make_prefill_inputs",
-           "make_decode_inputs", "make_prefill_inputs_device", "normal"]
+           "make_decode_inputs", "make_prefill_inputs_device", "make_msr_inputs", "normal"]
 
 
 @dataclass(frozen=True)
@@ -107,6 +107,26 @@ def make_prefill_inputs(batch: int, heads: int, seqlen: int, d: int, dtype: str,
         w = rng.standard_normal((hidden, heads * dv), dtype=np.float32) * np.float32(0.02)
         g = to_dtype((x @ w).reshape(batch, seqlen, heads, dv), dtype)
     return q, k, v, g
+
+
+def make_msr_inputs(batch: int, seqlen: int, hidden: int, heads: int, d: int, seed: int):
+    """Input and weights of the multi-scale retention layer, bf16 values.
+
+    x [B, n, hidden] ~ N(0, 1); W_Q, W_K, W_V [H d, hidden] ~ N(0, s) with
+    s = 1 / (16 sqrt(hidden)), so that the projected q, k, v have the
+    prefill workloads' spread N(0, 1/16^2); W_G [H d, hidden] ~ N(0, 0.02),
+    the gate weight of the layer workloads; W_O [hidden, H d] ~ N(0, 1/sqrt(H d)).
+    Returns x, w_qkvg (the rows of W_Q, W_K, W_V, W_G stacked) and w_o.
+    Draw order: x, W_Q, W_K, W_V, W_G, W_O.
+    """
+    rng = np.random.default_rng(seed)
+    hd = heads * d
+    x = normal(rng, (batch, seqlen, hidden), 1.0, "bf16")
+    s = 1.0 / (16.0 * np.sqrt(hidden))
+    wq, wk, wv = (normal(rng, (hd, hidden), s, "bf16") for _ in range(3))
+    wg = normal(rng, (hd, hidden), 0.02, "bf16")
+    wo = normal(rng, (hidden, hd), 1.0 / np.sqrt(hd), "bf16")
+    return x, np.concatenate([wq, wk, wv, wg], axis=0), wo
 
 
 def make_decode_inputs(batch: int, heads: int, steps: int, d: int, dtype: str,
