@@ -333,8 +333,10 @@ def run_ours(args, w, chunk):
         dist.barrier()
     rn.load_library()
     rn.retnet_set_launch_overlap(not args.no_overlap)
+    rn.retnet_set_output_pairing(args.pairs)
 
     line = measure_prefill(args, w, chunk, rank, world, dev, full=True)
+    line["output_pairs"] = args.pairs
     if args.form == "chunkwise" and not args.no_legs:
         # the decode configuration at the batches whose state is beyond L2,
         # and the 200M-layer step as a second prefill shape
@@ -656,6 +658,7 @@ def run_backward(args, w, chunk):
     build()
     rn.load_library()
     rn.retnet_set_launch_overlap(not args.no_overlap)
+    rn.retnet_set_output_pairing(args.pairs)
     B, n, H, d = w.batch, w.seqlen, w.heads, w.d
     gam = rn.retnet_default_gammas(H)
     sets = []
@@ -909,6 +912,7 @@ def run_layer(args, w, chunk):
     build()
     rn.load_library()
     rn.retnet_set_launch_overlap(not args.no_overlap)
+    rn.retnet_set_output_pairing(args.pairs)
     B, n, H, d = w.batch, w.seqlen, w.heads, w.d
     hidden = w.hidden or H * d
     gam = rn.retnet_default_gammas(H)
@@ -1022,6 +1026,9 @@ def main():
                     help="time the backward pass of the prefill (no epilogue) instead")
     ap.add_argument("--no-overlap", action="store_true",
                     help="launch kernels without programmatic launch overlap")
+    ap.add_argument("--pairs", type=int, choices=[0, 1, 2], default=1,
+                    help="output pass: 1 CTA pairs folding q (default), 2 CTA pairs with q "
+                         "folded by the prep pass, 0 single CTAs")
     ap.add_argument("--layer", action="store_true",
                     help="time the whole multi-scale retention layer (projections included)")
     ap.add_argument("--form", choices=["chunkwise", "parallel"], default="chunkwise",

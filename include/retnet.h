@@ -115,6 +115,18 @@ RETNET_API unsigned long long retnet_kernel_launch_count(void);
  * enable: 0 or 1, else INVALID_ARG. */
 RETNET_API retnet_status retnet_set_launch_overlap(int enable);
 
+/* How the tensor-core prefill's output pass runs (process-wide).
+ *   1 (default): chunks of 256 tokens or more run on pairs of CTAs whose
+ *     tensor cores act as one (each CTA loads half of every key, value and
+ *     state tile), and the pair rotates and decay-scales q itself, so the
+ *     prep pass writes only the folded keys;
+ *   2: CTA pairs as in 1, with q folded by the prep pass;
+ *   0: every CTA works alone.
+ * Chunk 128 (and the shorter chunks computed as 128) always runs on single
+ * CTAs.  Results agree to rounding; only the speed changes.
+ * mode: 0, 1 or 2, else INVALID_ARG. */
+RETNET_API retnet_status retnet_set_output_pairing(int mode);
+
 /* Per-head decay constants gamma_h = 1 - 2^(-5-h), h = 0..heads-1, written
  * to the HOST array gammas[heads] ("Key points": gamma = 1 - 2^(-5-i)).
  * Errors: INVALID_ARG if gammas is NULL or heads is outside 1..256. */

@@ -21,7 +21,7 @@ import torch
 
 __all__ = [
     "RetnetError", "load_library", "retnet_status_string", "retnet_kernel_launch_count",
-    "retnet_set_launch_overlap",
+    "retnet_set_launch_overlap", "retnet_set_output_pairing",
     "retnet_default_gammas", "retnet_xpos_rotate", "retnet_chunkwise_workspace_size",
     "retnet_retention_chunkwise", "retnet_parallel_workspace_size", "retnet_retention_parallel",
     "retnet_workspace",
@@ -81,6 +81,7 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         "retnet_status_string": (ctypes.c_char_p, [i]),
         "retnet_kernel_launch_count": (ctypes.c_ulonglong, []),
         "retnet_set_launch_overlap": (i, [i]),
+        "retnet_set_output_pairing": (i, [i]),
         "retnet_default_gammas": (i, [i, vp]),
         "retnet_xpos_rotate": (i, [vp, vp, i, i, i, i, i, ll, vp]),
         "retnet_chunkwise_workspace_size": (i, [ctypes.POINTER(_Shape), i, i, ctypes.POINTER(sz)]),
@@ -157,6 +158,13 @@ def retnet_kernel_launch_count() -> int:
 def retnet_set_launch_overlap(enable: bool) -> None:
     """Programmatic launch overlap of the hot kernels (on by default)."""
     _check("retnet_set_launch_overlap", load_library().retnet_set_launch_overlap(int(bool(enable))))
+
+
+def retnet_set_output_pairing(mode) -> None:
+    """How the tensor-core output pass runs: 1 (or True) CTA pairs folding q
+    themselves (default), 2 CTA pairs with q folded by the prep pass, 0 (or
+    False) single CTAs."""
+    _check("retnet_set_output_pairing", load_library().retnet_set_output_pairing(int(mode)))
 
 
 def retnet_default_gammas(heads: int) -> list:

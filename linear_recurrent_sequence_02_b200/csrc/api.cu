@@ -15,6 +15,9 @@ void count_launch(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxe
 static std::atomic<bool> g_overlap{true};
 bool launch_overlap_enabled() { return g_overlap.load(std::memory_order_relaxed); }
 
+static std::atomic<int> g_pairs{0};
+int output_pairing_mode() { return g_pairs.load(std::memory_order_relaxed); }
+
 __device__ unsigned g_device_error = 0u;
 
 void *current_context() {
@@ -161,6 +164,12 @@ unsigned long long retnet_kernel_launch_count(void) {
 retnet_status retnet_set_launch_overlap(int enable) {
     if (enable != 0 && enable != 1) return RETNET_ERR_INVALID_ARG;
     g_overlap.store(enable == 1, std::memory_order_relaxed);
+    return RETNET_OK;
+}
+
+retnet_status retnet_set_output_pairing(int mode) {
+    if (mode < 0 || mode > 2) return RETNET_ERR_INVALID_ARG;
+    g_pairs.store(mode, std::memory_order_relaxed);
     return RETNET_OK;
 }
 

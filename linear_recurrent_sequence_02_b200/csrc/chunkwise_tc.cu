@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(256, 4)
 tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                TcPrepParams pp, __nv_bfloat16 *__restrict__ qt, __nv_bfloat16 *__restrict__ kt,
                int batch, int heads, int n, int chunk, long long pos0, int rotate,
-               unsigned *err) {
+               int write_q, unsigned *err) {
     const long long elems = (long long)batch * n * heads * kD;   // of q, k, Qt and Kt
     __shared__ float2 cs[kD / 2];
     const int t = blockIdx.x;
@@ -71,7 +71,7 @@ tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
     // round's loads are issued before the (cos, sin) prologue so its latency
     // overlaps the memory traffic.
     constexpr int kPrepBatch = 4;
-    uint4 rq[kPrepBatch], rk[kPrepBatch];
+    uint4 rq[kPrepBatch] = {}, rk[kPrepBatch];
     auto load_round = [&](int base) {
 #pragma unroll
         for (int u = 0; u < kPrepBatch; ++u) {
@@ -82,7 +82,7 @@ tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
                 const int h = bhi % heads, b = bhi / heads;
                 const size_t src = (((size_t)b * n + t) * heads + h) * kD + part * 8;
                 if (!in_bounds((long long)src + 7, elems, err)) continue;
-                rq[u] = *reinterpret_cast<const uint4 *>(q + src);
+                if (write_q) rq[u] = *reinterpret_cast<const uint4 *>(q + src);
                 rk[u] = *reinterpret_cast<const uint4 *>(k + src);
             }
         }
@@ -121,7 +121,7 @@ tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
                 }
                 const size_t dst = (((size_t)b * heads + h) * n + t) * kD + part * 8;
                 if (!in_bounds((long long)dst + 7, elems, err)) continue;
-                store8(qt + dst, oq);
+                if (write_q) store8(qt + dst, oq);
                 store8(kt + dst, ok);
             }
         }
@@ -387,6 +387,13 @@ struct TcOutArgs {
     // g^(128 (r - t)), applied in the mask pass.
     int parallel;
     float log2g[kMaxHeads];
+    // Paired output pass only: fold_q = 1 loads raw q and applies the rotation
+    // and the decay fold in shared memory (the prep pass then writes only Kt);
+    // fold = the decay fold's block length (the chunk, or 128 in the parallel
+    // form); theta_j = 10000^(-2j/256); pos0 and rotate as for the call.
+    int fold_q, fold, rotate;
+    long long pos0;
+    double theta[kD / 2];
 };
 
 struct TcItem {
@@ -815,6 +822,635 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
 }
 
+// ------------------------------------------------------------------ paired output pass
+// The output pass on CTA pairs: the two CTAs of a cluster work as one
+// (tcgen05 cta_group::2, M = 256).  A pair-item is the row blocks (2p, 2p+1)
+// of one chunk; CTA k owns row block 2p + k in its own TMEM (same layout as
+// tc_output: O [0,256), Qt [256,384), S [384,512)).  The B operands are
+// split by N between the CTAs: for Qt Kt^T each CTA loads 64 of the tile's
+// 128 keys, for P V and Qt S_prev 128 of the 256 d_v columns, so a key tile
+// costs each CTA 64 KB of loads instead of 128 KB and a ring of six 32 KB
+// slots holds twice the tiles of tc_output's three 64 KB slots.  The pair
+// spends one 128 x 128 tile of wasted MMA work per pair-item where the
+// lower row block stops short of the upper one's last key tile.
+//
+// Roles as in tc_output, with the leader (rank 0) issuing every MMA:
+//   warp 0 (both CTAs): TMA loads into its own slots.  Operand loads count
+//     on the leader's rfull barrier of the slot (the leader arms it for both
+//     CTAs' bytes); the gate/output tile (two slots) counts on this CTA's
+//     own lfull barriers.  Each CTA completes one lfull phase, and the
+//     leader one rfull phase, for every ring item, so that both follow the
+//     ring order whatever the slot holds.
+//   warp 1: TMEM allocation (both CTAs, paired); the leader's lane 0
+//     issues the copies and MMAs, whose commits arrive on the barrier of
+//     the same offset in both CTAs (rempty, s_full, p_free, o_full).
+//   warps 2-9 (both CTAs): the mask pass and the epilogue on this CTA's
+//     rows; their arrivals (s_read, p_full, o_free) go to the leader.
+// A timeout in either CTA raises both CTAs' abort flags; at the end the
+// leader settles and drains the operand loads of both CTAs before the
+// cluster's last barrier, so neither CTA exits with loads still landing in
+// its shared memory.
+constexpr int kPairSlots = 6;
+constexpr uint32_t kPairSlot = 2 * kBox;           // 32 KB
+constexpr int kPairThreads = 448;                  // 14 warps: the 10 of tc_output + 4 fold warps
+constexpr int kFoldThreads = 128;
+
+struct TcPairSmem {
+    static constexpr uint32_t kP = kPairSlots * kPairSlot;   // P tile; the epilogue's row sums
+    static constexpr uint32_t kBytes = kP + 2 * kBox + 1024;
+};
+
+struct TcPairItem {
+    int p, c, bh, b, h, c0, nk, nsp, r, t0row;
+    bool valid;                                    // some row of the pair lies in the chunk
+};
+
+// Pair-item w: group g = w / np is one (sequence, head, chunk) with np row-
+// block pairs at consecutive w, rotated by the group index as in tc_item.
+__device__ __forceinline__ TcPairItem tc_pair_item(const TcOutArgs &a, int w, int rank) {
+    const int np = (a.rblocks + 1) / 2;
+    TcPairItem it;
+    const int g = w / np;
+    it.p = (w + g) % np;
+    it.c = g % a.nchunks;
+    it.bh = g / a.nchunks;
+    it.b = it.bh / a.heads;
+    it.h = it.bh % a.heads;
+    it.c0 = it.c * a.chunk;
+    const int L = min(a.chunk, a.n - it.c0);
+    it.valid = 2 * it.p * kBlk < L;
+    const int kend = min(kBlk * (2 * it.p + 2), L);   // keys the pair's rows see
+    it.nk = (kend + kKeyTile - 1) / kKeyTile;
+    it.nsp = (it.c > 0 || a.has_state_in) ? 2 : 0;
+    it.r = 2 * it.p + rank;
+    it.t0row = it.c0 + it.r * kBlk;
+    return it;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
+tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_kh,
+                      const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_s,
+                      const __grid_constant__ CUtensorMap tm_g,
+                      const __grid_constant__ CUtensorMap tm_out,
+                      const __grid_constant__ CUtensorMap tm_qraw, TcOutArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    __shared__ uint64_t rfull[kPairSlots], rempty[kPairSlots], lfull[kPairSlots];
+    __shared__ uint64_t s_full, s_read, p_full[2], p_free[2], o_full, o_free, drain, q_ready;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int abort_flag;
+    __shared__ int issued;                         // ring items this CTA issued
+    __shared__ uint32_t slot_op[kPairSlots];       // latest item of the slot: 1 operand, 0 gate
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    unsigned *err = a.err;
+    const int np = (a.rblocks + 1) / 2;
+    const long long nbh = a.items / (a.nchunks * np);
+    const int cluster = blockIdx.x / 2, nclusters = gridDim.x / 2;
+    auto slot_ptr = [smem](int it) -> uint8_t * { return smem + (it % kPairSlots) * kPairSlot; };
+    uint8_t *pbuf = smem + TcPairSmem::kP;
+    // the leader's copy of a barrier, as a shared::cluster address
+    auto at_leader = [](uint64_t *bar) -> uint32_t { return mapa_shared(smem_u32(bar), 0); };
+    const uint32_t peer_abort = mapa_shared(smem_u32(&abort_flag), rank ^ 1u);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPairSlots; ++s) {
+            mbar_init(&rfull[s], 1);
+            mbar_init(&rempty[s], 1);
+            mbar_init(&lfull[s], 1);
+        }
+        mbar_init(&s_full, 1);
+        mbar_init(&s_read, 2 * kEpiThreads);
+        for (int x = 0; x < 2; ++x) {                    // one P half per warpgroup, both CTAs
+            mbar_init(&p_full[x], kEpiThreads);
+            mbar_init(&p_free[x], 1);
+        }
+        mbar_init(&o_full, 1);
+        mbar_init(&o_free, 2 * kEpiThreads);
+        mbar_init(&drain, 1);
+        mbar_init(&q_ready, 2 * kFoldThreads);
+        abort_flag = 0;
+        issued = 0;
+        for (int s = 0; s < kPairSlots; ++s) slot_op[s] = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(&tmem_slot, 512);
+        tmem_relinquish_pair();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_kh);
+        tma_prefetch_desc(&tm_v); tma_prefetch_desc(&tm_s);
+        if (a.has_gate) tma_prefetch_desc(&tm_g);
+        if (a.fold_q) tma_prefetch_desc(&tm_qraw);
+    }
+    tc_fence_before();
+    cluster_sync();                                   // both CTAs' barriers and TMEM exist
+    tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+    const uint32_t tO = tmem, tQ = tmem + 256, tS = tmem + 384;
+    grid_dependency_wait();                           // Qt, Kt, S_prev from the kernels before
+
+    // Raises this CTA's and the peer's abort flags (after a failed wait).
+    auto abort_both = [&]() {
+        abort_flag = 1;
+        st_cluster_u32(peer_abort, 1u);
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int it = 0;
+            bool ok = true;
+            auto acquire = [&]() -> bool {
+                if (it < kPairSlots) return true;
+                return mbar_wait(&rempty[it % kPairSlots], ((it / kPairSlots) - 1) & 1,
+                                 &abort_flag, err);
+            };
+            // one operand item: `boxes` boxes of 16 KB (or 8 KB for Kt halves) into
+            // this CTA's slot, counted on the leader's rfull (armed for both CTAs)
+            auto issue_op = [&](int kind, int c1, int c2, int c3) {
+                uint8_t *d = slot_ptr(it);
+                uint64_t *bar = &rfull[it % kPairSlots];
+                const uint32_t lbar = at_leader(bar);
+                slot_op[it % kPairSlots] = 1;
+                mbar_arrive(&lfull[it % kPairSlots]);          // keeps lfull in ring order
+                if (leader) mbar_expect_tx(bar, 2 * kPairSlot);
+                if (kind == 0) {                               // Qt: two 64-col boxes
+                    for (int x = 0; x < 2; ++x)
+                        tma_load_3d_pair(d + x * kBox, &tm_q, lbar, 64 * (c3 + x), c1, c2);
+                } else if (kind == 1) {                        // Kt half: 64 keys x 256
+                    for (int x = 0; x < 4; ++x)
+                        tma_load_3d_pair(d + x * (kBox / 2), &tm_kh, lbar, 64 * x, c1, c2);
+                } else if (kind == 2) {                        // S_prev half: 128 d_v cols
+                    for (int x = 0; x < 2; ++x)
+                        tma_load_2d_pair(d + x * kBox, &tm_s, lbar, 128 * (int)rank + 64 * x, c1);
+                } else {                                       // V: 128 d_v cols x 128 keys
+                    for (int x = 0; x < 2; ++x)
+                        tma_load_4d_pair(d + x * kBox, &tm_v, lbar, 128 * (int)rank + 64 * x, c2,
+                                         c1, c3);
+                }
+                ++it;
+                *(volatile int *)&issued = it;
+            };
+            for (int w = cluster; ok && w < a.items; w += nclusters) {
+                const TcPairItem m = tc_pair_item(a, w, rank);
+                if (!m.valid) continue;
+                const int srow = (m.bh * a.nchunks + m.c) * kD;
+                if (!in_bounds(m.bh, nbh, err) ||
+                    !in_bounds(srow + kD - 1, nbh * a.nchunks * kD, err)) {
+                    ok = false;
+                    abort_both();
+                    break;
+                }
+                for (int half = 0; ok && half < 2; ++half) {
+                    if (!(ok = acquire())) break;
+                    if (a.fold_q) {
+                        // raw q rows of this CTA, folded in place by the fold
+                        // warps (counted on lfull; rfull only kept in order)
+                        uint8_t *d = slot_ptr(it);
+                        uint64_t *lb = &lfull[it % kPairSlots];
+                        slot_op[it % kPairSlots] = 0;
+                        if (leader) mbar_arrive(&rfull[it % kPairSlots]);
+                        mbar_expect_tx(lb, kPairSlot);
+                        for (int x = 0; x < 2; ++x)
+                            tma_load_4d(d + x * kBox, &tm_qraw, lb, 128 * half + 64 * x, m.h,
+                                        m.t0row, m.b);
+                        ++it;
+                        *(volatile int *)&issued = it;
+                    } else {
+                        issue_op(0, m.t0row, m.bh, 2 * half);
+                    }
+                }
+                if (!ok || !(ok = acquire())) break;
+                issue_op(1, m.c0 + 64 * (int)rank, m.bh, 0);
+                for (int t = 0; ok && t < m.nk; ++t) {
+                    if (t + 1 < m.nk) {
+                        if (!(ok = acquire())) break;
+                        issue_op(1, m.c0 + (t + 1) * kKeyTile + 64 * (int)rank, m.bh, 0);
+                    }
+                    if (t < m.nsp) {
+                        if (!(ok = acquire())) break;
+                        issue_op(2, srow + kBlk * t, 0, 0);
+                    }
+                    if (!(ok = acquire())) break;
+                    issue_op(3, m.c0 + t * kKeyTile, m.h, m.b);
+                }
+                for (int p = m.nk; ok && p < m.nsp; ++p) {
+                    if (!(ok = acquire())) break;
+                    issue_op(2, srow + kBlk * p, 0, 0);
+                }
+                // the gate/output tile: two slots of this CTA, each counted on
+                // its own lfull (or only reserved for the output rows)
+                for (int half = 0; ok && half < 2; ++half) {
+                    if (!(ok = acquire())) break;
+                    uint8_t *gs = slot_ptr(it);
+                    uint64_t *lb = &lfull[it % kPairSlots];
+                    slot_op[it % kPairSlots] = 0;
+                    if (leader) mbar_arrive(&rfull[it % kPairSlots]);   // keeps rfull in order
+                    if (a.has_gate) {
+                        mbar_expect_tx(lb, 2 * kBox);
+                        for (int x = 0; x < 2; ++x)
+                            tma_load_4d(gs + x * kBox, &tm_g, lb, 128 * half + 64 * x, m.h,
+                                        m.t0row, m.b);
+                    } else {
+                        mbar_arrive(lb);
+                    }
+                    ++it;
+                    *(volatile int *)&issued = it;
+                }
+            }
+            if (!ok) abort_both();
+        }
+    } else if (warp == 1) {
+        if (leader && lane == 0) {
+            const uint32_t id_qk = idesc_bf16(256, kKeyTile, 0, 0);
+            const uint32_t id_pv = idesc_bf16(256, 256, 0, 1);
+            const uint32_t sP = smem_u32(pbuf);
+            int it = 0, nqk = 0, npv = 0, li = 0;
+            bool ok = true;
+            auto take = [&]() -> bool {
+                if (!mbar_wait(&rfull[it % kPairSlots], (it / kPairSlots) & 1, &abort_flag, err))
+                    return false;
+                tc_fence_after();
+                return true;
+            };
+            auto slot_addr = [&](int i) -> uint32_t { return smem_u32(slot_ptr(i)); };
+            for (int w = cluster; ok && w < a.items; w += nclusters, ++li) {
+                const TcPairItem m = tc_pair_item(a, w, 0);
+                if (!m.valid) { --li; continue; }
+                bool o_written = false;
+                auto claim_o = [&]() -> bool {
+                    if (o_written || li == 0) return true;
+                    return mbar_wait(&o_free, (li - 1) & 1, &abort_flag, err);
+                };
+                // the previous item's MMAs read Qt from TMEM: they must be
+                // complete before the copy below overwrites it (cp is ordered
+                // before later MMAs of this thread, not after earlier ones)
+                if (li > 0 && !(ok = mbar_wait(&o_full, (li - 1) & 1, &abort_flag, err))) break;
+                tc_fence_after();
+                // Qt of both CTAs -> their TMEM, 16 columns of K per copy: as
+                // loaded, or once the fold warps of both CTAs have folded it
+                if (a.fold_q) {
+                    if (!(ok = mbar_wait(&q_ready, li & 1, &abort_flag, err))) break;
+                    tc_fence_after();
+                } else if (!(ok = take())) {
+                    break;
+                }
+                const uint32_t qa = slot_addr(it);
+                const int sa = it % kPairSlots;
+                ++it;
+                if (!a.fold_q && !(ok = take())) break;
+                const uint32_t qb = slot_addr(it);
+                const int sb = it % kPairSlots;
+                ++it;
+#pragma unroll
+                for (int ks = 0; ks < kD / 16; ++ks) {
+                    const uint32_t base = (ks < 8 ? qa : qb) + ((ks / 4) % 2) * kBox + (ks % 4) * 32;
+                    tmem_cp_128x256b_pair(tQ + 8 * ks, smem_desc_sw128(base, 16, 1024));
+                }
+                mma_commit_pair(&rempty[sa], 3);
+                mma_commit_pair(&rempty[sb], 3);
+                // S = Qt Kt^T for key tile t: each CTA holds 64 of its keys
+                auto qk = [&]() -> bool {
+                    if (nqk >= 1 && !mbar_wait(&s_read, (nqk - 1) & 1, &abort_flag, err)) return false;
+                    if (!take()) return false;
+                    const uint32_t base = slot_addr(it);
+#pragma unroll
+                    for (int ks = 0; ks < kD / 16; ++ks)
+                        mma_bf16_ts_pair(tS, tQ + 8 * ks,
+                                         smem_desc_sw128(base + (ks / 4) * (kBox / 2) + (ks % 4) * 32,
+                                                         16, 1024),
+                                         id_qk, ks > 0 ? 1u : 0u);
+                    mma_commit_pair(&rempty[it % kPairSlots], 3);
+                    mma_commit_pair(&s_full, 3);
+                    ++it;
+                    ++nqk;
+                    return true;
+                };
+                // O += Qt[:, 128p .. 128p+128) S_prev[128p .. 128p+128, :]
+                auto qs_half = [&](int p) -> bool {
+                    if (!take() || !claim_o()) return false;
+                    const uint32_t base = slot_addr(it);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ts_pair(tO, tQ + 8 * (8 * p + kk),
+                                         smem_desc_sw128(base + kk * 2048, kBox, 1024), id_pv,
+                                         (o_written || kk > 0) ? 1u : 0u);
+                    o_written = true;
+                    mma_commit_pair(&rempty[it % kPairSlots], 3);
+                    ++it;
+                    return true;
+                };
+                ok = qk();
+                for (int t = 0; ok && t < m.nk; ++t) {
+                    if (t + 1 < m.nk && !(ok = qk())) break;
+                    if (t < m.nsp && !(ok = qs_half(t))) break;
+                    if (!(ok = take() && claim_o())) break;
+                    const uint32_t base = slot_addr(it);
+                    for (int hx = 0; ok && hx < 2; ++hx) {
+                        if (!mbar_wait(&p_full[hx], npv & 1, &abort_flag, err)) { ok = false; break; }
+                        tc_fence_after();
+#pragma unroll
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            const int kk = 4 * hx + k4;
+                            mma_bf16_pair(tO, smem_desc_sw128(sP + hx * kBox + k4 * 32, 16, 1024),
+                                          smem_desc_sw128(base + kk * 2048, kBox, 1024), id_pv,
+                                          (o_written || kk > 0) ? 1u : 0u);
+                        }
+                        mma_commit_pair(&p_free[hx], 3);
+                    }
+                    if (!ok) break;
+                    o_written = true;
+                    mma_commit_pair(&rempty[it % kPairSlots], 3);
+                    ++it;
+                    ++npv;
+                }
+                for (int p = m.nk; ok && p < m.nsp; ++p) ok = qs_half(p);
+                if (!ok) break;
+                mma_commit_pair(&o_full, 3);
+                it += 2;                                       // skip the gate/output slots
+            }
+            if (!ok) abort_both();
+        }
+    } else if (warp >= 10) {
+        // Fold warps: rotate and decay-scale this CTA's raw q rows in place,
+        // Qt_i = g^(lf+1) R q_i (lf: the row's index in its fold block).
+        // Thread j owns the pair (2j, 2j+1) and walks the 128 rows in eight
+        // interleaved runs of 16; each run starts from an exact (cos, sin)
+        // and steps the complex factor g e^{i theta_j} per row.
+        if (a.fold_q) {
+            const int j = threadIdx.x - 10 * 32;               // pair column 0..127
+            const uint32_t l_q_ready = at_leader(&q_ready);
+            const double theta = a.theta[j];
+            float st_c = 1.f, st_s = 0.f;                      // e^{i theta_j}
+            if (a.rotate) {
+                const float2 r = rotation_cs(1, theta);
+                st_c = r.x;
+                st_s = r.y;
+            }
+            const int bx = j / 32;                             // 64-column box
+            const uint32_t in_row = (uint32_t)((j % 4) * 4);
+            const int ch = (j % 32) / 4;                       // 16-byte chunk in the row
+            int it_base = 0;
+            bool ok = true;
+            for (int w = cluster; ok && w < a.items; w += nclusters) {
+                const TcPairItem m = tc_pair_item(a, w, rank);
+                if (!m.valid) continue;
+                const int qi = it_base;
+                it_base += 2 + 2 * m.nk + m.nsp + 2;
+                const int qs = qi + bx / 2;                    // this column's slot
+                if (!mbar_wait(&lfull[qs % kPairSlots], (qs / kPairSlots) & 1, &abort_flag, err)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t *box = slot_ptr(qs) + (bx % 2) * kBox;
+                const float lg = a.log2g[m.h];
+                const float gc = exp2f(lg) * st_c, gs = exp2f(lg) * st_s;   // g e^{i theta}
+                const int lf0 = a.fold == kBlk ? 0 : m.r * kBlk;            // fold index of row 0
+                float zc[8], zs[8];
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    const float2 r = a.rotate ? rotation_cs(a.pos0 + m.t0row + 16 * g, theta)
+                                              : make_float2(1.f, 0.f);
+                    const float sc = exp2f((float)(lf0 + 16 * g + 1) * lg);
+                    zc[g] = r.x * sc;
+                    zs[g] = r.y * sc;
+                }
+#pragma unroll 2
+                for (int i = 0; i < 16; ++i) {
+#pragma unroll
+                    for (int g = 0; g < 8; ++g) {
+                        const int row = 16 * g + i;
+                        uint32_t *pw = reinterpret_cast<uint32_t *>(
+                            box + row * 128 + ((ch ^ (row & 7)) * 16) + in_row);
+                        const uint32_t raw = *pw;
+                        const float2 x =
+                            __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw));
+                        const float c = zc[g], sn = zs[g];
+                        *pw = pack_bf16x2(x.x * c - x.y * sn, x.x * sn + x.y * c);
+                        zc[g] = c * gc - sn * gs;
+                        zs[g] = c * gs + sn * gc;
+                    }
+                }
+                fence_async_shared();
+                mbar_arrive_cluster(l_q_ready);
+            }
+            if (!ok && lane == 0) abort_both();
+        }
+    } else {
+        const int wg = (warp - 2) / 4;
+        const int q4 = warp % 4;
+        const int row = 32 * q4 + lane;
+        const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
+        const uint32_t l_s_read = at_leader(&s_read), l_o_free = at_leader(&o_free);
+        const uint32_t l_p_full = at_leader(&p_full[wg]);
+        uint8_t *prow = pbuf + wg * kBox + row * 128;
+        int it_base = 0, ntile = 0, li = 0;
+        bool ok = true;
+        for (int w = cluster; ok && w < a.items; w += nclusters, ++li) {
+            const TcPairItem m = tc_pair_item(a, w, rank);
+            if (!m.valid) { --li; continue; }
+            const int lrow = m.r * kBlk + row;                  // row within the chunk
+            for (int t = 0; t < m.nk; ++t, ++ntile) {
+                if (!warp_wait(&s_full, ntile & 1, &abort_flag, err)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t v0[32], v1[32];
+                const uint32_t col = tS + lane_off + 64 * wg;
+                tmem_ld32(col, v0);
+                tmem_ld32(col + 32, v1);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive_cluster(l_s_read);                  // S may be overwritten now
+                const int j0 = t * kKeyTile + 64 * wg;
+                uint32_t wv[32];
+                if (a.parallel && t < m.r) {
+                    const float tf = exp2f((float)(kKeyTile * (m.r - t)) * a.log2g[m.h]);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        wv[e] = pack_bf16x2(tf * __uint_as_float(v0[2 * e]), tf * __uint_as_float(v0[2 * e + 1]));
+                        wv[16 + e] = pack_bf16x2(tf * __uint_as_float(v1[2 * e]), tf * __uint_as_float(v1[2 * e + 1]));
+                    }
+                } else if (j0 + 63 <= lrow) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        wv[e] = pack_bf16x2(__uint_as_float(v0[2 * e]), __uint_as_float(v0[2 * e + 1]));
+                        wv[16 + e] = pack_bf16x2(__uint_as_float(v1[2 * e]), __uint_as_float(v1[2 * e + 1]));
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int j = j0 + 2 * e;
+                        const float x0 = (lrow >= j) ? __uint_as_float(v0[2 * e]) : 0.f;
+                        const float x1 = (lrow >= j + 1) ? __uint_as_float(v0[2 * e + 1]) : 0.f;
+                        const float y0 = (lrow >= j + 32) ? __uint_as_float(v1[2 * e]) : 0.f;
+                        const float y1 = (lrow >= j + 33) ? __uint_as_float(v1[2 * e + 1]) : 0.f;
+                        wv[e] = pack_bf16x2(x0, x1);
+                        wv[16 + e] = pack_bf16x2(y0, y1);
+                    }
+                }
+                if (ntile >= 1 && !warp_wait(&p_free[wg], (ntile - 1) & 1, &abort_flag, err)) { ok = false; break; }
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    *reinterpret_cast<uint4 *>(prow + ((ch ^ (row & 7)) * 16)) =
+                        make_uint4(wv[4 * ch], wv[4 * ch + 1], wv[4 * ch + 2], wv[4 * ch + 3]);
+                fence_async_shared();
+                tc_fence_before();
+                mbar_arrive_cluster(l_p_full);
+            }
+            // ring items of this pair-item: Qt (2), nk Kt halves, nsp S_prev
+            // halves, nk V halves, then the gate/output tile (2 slots)
+            const int ig = it_base + 2 + 2 * m.nk + m.nsp;
+            it_base = ig + 2;
+            uint8_t *ya = slot_ptr(ig), *yb = slot_ptr(ig + 1);
+            const bool go =
+                ok && warp_wait(&o_full, li & 1, &abort_flag, err) &&
+                warp_wait(&lfull[ig % kPairSlots], (ig / kPairSlots) & 1, &abort_flag, err) &&
+                warp_wait(&lfull[(ig + 1) % kPairSlots], ((ig + 1) / kPairSlots) & 1, &abort_flag,
+                          err);
+            float (*red)[kBlk] = reinterpret_cast<float (*)[kBlk]>(pbuf);   // [4][128]
+            float mean = 0.f, rstd = 1.f;
+            if (go) tc_fence_after();
+            if (a.has_gate) {
+                float sum = 0.f, sq = 0.f, shift = 0.f;
+                if (go) {
+                    uint32_t v0[32];
+                    tmem_ld32(tO + lane_off, v0);
+                    tmem_wait_ld();
+                    shift = __uint_as_float(v0[0]);
+#pragma unroll 1
+                    for (int cb = 0; cb < 4; ++cb) {
+                        uint32_t v[32];
+                        tmem_ld32(tO + lane_off + 128 * wg + 32 * cb, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const float d = __uint_as_float(v[e]) - shift;
+                            sum += d;
+                            sq = fmaf(d, d, sq);
+                        }
+                    }
+                }
+                red[2 * wg][row] = sum;
+                red[2 * wg + 1][row] = sq;
+                named_barrier(1, kEpiThreads);
+                const float ms = (red[0][row] + red[2][row]) * (1.f / kD);
+                const float m2 = (red[1][row] + red[3][row]) * (1.f / kD);
+                mean = shift + ms;
+                rstd = rsqrtf(fmaxf(m2 - ms * ms, 0.f) + a.eps);
+                named_barrier(1, kEpiThreads);
+            }
+            if (go) {
+                const int sw = row & 7;
+                const float *gw = a.gn_weight ? a.gn_weight + m.h * kD : nullptr;
+                const float *gb = a.gn_bias ? a.gn_bias + m.h * kD : nullptr;
+#pragma unroll 1
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const int cb = 4 * wg + k4;
+                    uint32_t v[32];
+                    tmem_ld32(tO + lane_off + 32 * cb, v);
+                    tmem_wait_ld();
+                    if (k4 == 3) {
+                        tc_fence_before();
+                        mbar_arrive_cluster(l_o_free);
+                    }
+                    const int bx = cb >> 1;                       // 64-column box
+                    uint8_t *box = (bx < 2 ? ya : yb) + (bx % 2) * kBox + row * 128;
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8) {
+                        uint4 *slot = reinterpret_cast<uint4 *>(box + ((((cb & 1) * 4 + q8) ^ sw) * 16));
+                        float y[8];
+                        if (a.has_gate) {
+                            uint4 graw = *slot;
+                            const __nv_bfloat162 *g2 = reinterpret_cast<const __nv_bfloat162 *>(&graw);
+#pragma unroll
+                            for (int e2 = 0; e2 < 4; ++e2) {
+                                const float2 gg = __bfloat1622float2(g2[e2]);
+#pragma unroll
+                                for (int hh = 0; hh < 2; ++hh) {
+                                    const int e = 2 * e2 + hh;
+                                    const int ch = 32 * cb + 8 * q8 + e;
+                                    float yh = (__uint_as_float(v[8 * q8 + e]) - mean) * rstd;
+                                    if (gw) yh *= gw[ch];
+                                    if (gb) yh += gb[ch];
+                                    y[e] = swish_fast(hh ? gg.y : gg.x) * yh;
+                                }
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) y[e] = __uint_as_float(v[8 * q8 + e]);
+                        }
+                        *slot = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
+                                           pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
+                    }
+                }
+                fence_async_shared();
+            } else {
+                mbar_arrive_cluster(l_o_free);
+            }
+            named_barrier(1, kEpiThreads);
+            if (wg == 0 && row == 0) {
+                if (!abort_flag && m.t0row < a.n) {           // rows past the sequence: nothing
+                    for (int x = 0; x < 4; ++x)
+                        tma_store_4d(&tm_out, (x < 2 ? ya : yb) + (x % 2) * kBox, 64 * x, m.h,
+                                     m.t0row, m.b);
+                    tma_store_commit();
+                    tma_store_wait_read();
+                }
+                mbar_arrive(&rempty[ig % kPairSlots]);        // both slots may be refilled
+                mbar_arrive(&rempty[(ig + 1) % kPairSlots]);
+            }
+            if (!go) ok = false;
+        }
+        if (!ok && lane == 0) abort_both();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();                                   // both CTAs' roles are done
+    // After an abort in either CTA, wait (bounded) for everything still in
+    // flight: the leader settles and drains the operand loads of both CTAs
+    // (they count on its barriers) and its MMAs; each CTA its own gate loads.
+    const bool aborted = abort_flag != 0;
+    if (aborted && warp == 0 && lane == 0) {
+        for (int j = max(0, issued - kPairSlots); j < issued; ++j)
+            mbar_drain(&lfull[j % kPairSlots], (j / kPairSlots) & 1, err);
+        if (leader) {
+            // Both CTAs walk the same ring order, at most kPairSlots items past
+            // the MMAs' progress, so the items still open are the last
+            // kPairSlots of the further producer; gate items never count on
+            // rfull beyond the leader's own arrival.
+            const int own = issued;
+            const int peer = (int)ld_cluster_u32(mapa_shared(smem_u32(&issued), 1));
+            const int last = max(own, peer);
+            for (int j = max(0, last - kPairSlots); j < last; ++j) {
+                uint64_t *bar = &rfull[j % kPairSlots];
+                if (j >= own) {                                // only the peer reached it
+                    const uint32_t op =
+                        ld_cluster_u32(mapa_shared(smem_u32(&slot_op[j % kPairSlots]), 1));
+                    if (!op) continue;
+                    mbar_expect_tx(bar, kPairSlot);
+                } else if (j >= peer && slot_op[j % kPairSlots]) {
+                    mbar_complete_tx(bar, kPairSlot);          // the peer never loaded its half
+                }
+                mbar_drain(bar, (j / kPairSlots) & 1, err);
+            }
+        }
+    }
+    if (aborted && warp == 1 && leader && lane == 0) {
+        mma_commit_pair(&drain, 1);
+        mbar_drain(&drain, 0, err);
+    }
+    tc_fence_before();
+    cluster_sync();                                   // the pair's loads and MMAs have landed
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, 512);
+    }
+}
+
 // ------------------------------------------------------------------ host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
@@ -970,14 +1606,22 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
     }
 
     cudaError_t e;
+    // The output pass runs on CTA pairs for two or more row blocks per chunk
+    // (a 128-token chunk would leave half of every pair idle); in mode 1 it
+    // also folds q itself, and the prep pass writes only Kt.
+    const int pair_mode = output_pairing_mode();
+    const bool pairs = pair_mode != 0 && C / kBlk >= 2;
+    const bool fold_q = pairs && pair_mode == 1;
+    double pp_theta[kD / 2];
+    for (int j = 0; j < kD / 2; ++j) pp_theta[j] = std::pow(10000.0, -2.0 * j / kD);
     {
         TcPrepParams pp;
-        for (int j = 0; j < kD / 2; ++j) pp.theta[j] = std::pow(10000.0, -2.0 * j / kD);
+        for (int j = 0; j < kD / 2; ++j) pp.theta[j] = pp_theta[j];
         for (int h = 0; h < kMaxHeads; ++h) pp.log2g[h] = hp.log2g[h];
         KernelTimer timer("tc_prep", stream);
         e = launch_overlapped(tc_prep_kernel, dim3(n), dim3(256), 0, stream,
                               (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, pp, qt, kt,
-                              B, H, n, fold, a.pos0, a.rotate, err);
+                              B, H, n, fold, a.pos0, a.rotate, fold_q ? 0 : 1, err);
         count_launch();
         if (e != cudaSuccess) return e;
     }
@@ -1018,22 +1662,70 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
         oa.gn_bias = a.gate ? a.gate->bias : nullptr;
         oa.eps = a.gate ? a.gate->eps : 0.f;
         oa.err = err;
-        oa.items = BH * nchunks * oa.rblocks;
         oa.parallel = parallel ? 1 : 0;
         for (int h = 0; h < kMaxHeads; ++h) oa.log2g[h] = hp.log2g[h];
-        const int smem = (int)TcOutSmem::kBytes;
-        e = cudaFuncSetAttribute(tc_output_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 smem);
-        if (e != cudaSuccess) return e;
+        oa.fold_q = fold_q ? 1 : 0;
+        oa.fold = fold;
+        oa.rotate = a.rotate;
+        oa.pos0 = a.pos0;
+        for (int j = 0; j < kD / 2; ++j) oa.theta[j] = pp_theta[j];
         int dev = 0, sms = 148;
         if (cudaGetDevice(&dev) == cudaSuccess)
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        const unsigned grid = (unsigned)std::min(oa.items, sms);
-        KernelTimer timer("tc_output", stream);
-        e = launch_overlapped(tc_output_kernel, dim3(grid), dim3(kOutThreads), smem, stream, tm_q,
-                              tm_k, tm_v, tm_s, tm_g, tm_out, oa);
-        count_launch();
-        if (e != cudaSuccess) return e;
+        // CTA pairs serve chunks of two or more row blocks; a chunk of one
+        // (128) would leave half of every pair idle.
+        if (pairs) {
+            oa.items = BH * nchunks * ((oa.rblocks + 1) / 2);
+            CUtensorMap tm_qraw;                  // raw q, folded inside the output pass
+            {
+                cuuint64_t dims[4] = {kD, (cuuint64_t)H, (cuuint64_t)n, (cuuint64_t)B};
+                cuuint64_t str[3] = {kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)n * H * kD * 2};
+                cuuint32_t box[4] = {64, 1, kBlk, 1};
+                if (!make_tensor_map_bf16(&tm_qraw, a.q, 4, dims, str, box))
+                    return cudaErrorInvalidValue;
+            }
+            CUtensorMap tm_kh;                    // Kt in halves of 64 keys
+            {
+                cuuint64_t dims[3] = {kD, (cuuint64_t)n, (cuuint64_t)BH};
+                cuuint64_t str[2] = {kD * 2, (cuuint64_t)n * kD * 2};
+                cuuint32_t box[3] = {64, kKeyTile / 2, 1};
+                if (!make_tensor_map_bf16(&tm_kh, kt, 3, dims, str, box))
+                    return cudaErrorInvalidValue;
+            }
+            const int smem = (int)TcPairSmem::kBytes;
+            e = cudaFuncSetAttribute(tc_output_pair_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (e != cudaSuccess) return e;
+            // as many pairs as fit on the GPU at once (whole clusters per GPC)
+            cudaLaunchConfig_t qc = {};
+            qc.gridDim = dim3(2 * (unsigned)std::max(1, sms / 2));
+            qc.blockDim = dim3(kPairThreads);
+            qc.dynamicSmemBytes = smem;
+            int clusters = 0;
+            if (cudaOccupancyMaxActiveClusters(&clusters, tc_output_pair_kernel, &qc) !=
+                    cudaSuccess ||
+                clusters < 1)
+                clusters = std::max(1, sms / 2);
+            clusters = std::min(clusters, oa.items);
+            KernelTimer timer("tc_output", stream);
+            e = launch_overlapped(tc_output_pair_kernel, dim3(2 * clusters), dim3(kPairThreads),
+                                  smem, stream, tm_q, tm_kh, tm_v, tm_s, tm_g, tm_out, tm_qraw,
+                                  oa);
+            count_launch();
+            if (e != cudaSuccess) return e;
+        } else {
+            oa.items = BH * nchunks * oa.rblocks;
+            const int smem = (int)TcOutSmem::kBytes;
+            e = cudaFuncSetAttribute(tc_output_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     smem);
+            if (e != cudaSuccess) return e;
+            const unsigned grid = (unsigned)std::min(oa.items, sms);
+            KernelTimer timer("tc_output", stream);
+            e = launch_overlapped(tc_output_kernel, dim3(grid), dim3(kOutThreads), smem, stream,
+                                  tm_q, tm_k, tm_v, tm_s, tm_g, tm_out, oa);
+            count_launch();
+            if (e != cudaSuccess) return e;
+        }
     }
     return cudaSuccess;
 }

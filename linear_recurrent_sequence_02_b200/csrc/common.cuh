@@ -132,6 +132,10 @@ __device__ __forceinline__ void grid_dependency_wait() {
 // Host: whether launches carry the programmatic-serialisation attribute
 // (retnet_set_launch_overlap; on by default).
 bool launch_overlap_enabled();
+// Host: how the tensor-core output pass runs (retnet_set_output_pairing):
+// 0 single CTAs, 1 CTA pairs folding q themselves (default), 2 CTA pairs
+// reading the prep pass's folded q.
+int output_pairing_mode();
 
 template <typename... KArgs, typename... Args>
 cudaError_t launch_overlapped(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,

@@ -78,3 +78,19 @@ def test_parallel_refuses_fast_decays(rn):
     q, k, v, _ = wl.make_prefill_inputs(1, 2, 128, 256, "bf16", 1.0 / 16.0, 92)
     with pytest.raises(rn.RetnetError):
         rn.retnet_retention_parallel(dev(q), dev(k), dev(v), [0.5, 0.9])
+
+
+@pytest.mark.parametrize("pairs", [1, 2, 0])
+@pytest.mark.parametrize("n", [300, 640, 129])
+def test_parallel_form_pairs_and_single(rn, pairs, n):
+    # an odd number of 128-row blocks leaves the last CTA pair half empty
+    B, H = 1, 2
+    q, k, v, g = wl.make_prefill_inputs(B, H, n, 256, "bf16", 1.0 / 16.0, 95 + n, hidden=256)
+    gam = rn.retnet_default_gammas(H)
+    rn.retnet_set_output_pairing(pairs)
+    try:
+        got = rn.retnet_retention_parallel(dev(q), dev(k), dev(v), gam, pos0=3, gate=dev(g))
+        rn.retnet_check_device_errors()
+    finally:
+        rn.retnet_set_output_pairing(0)
+    assert slice_rel_err(host(got), want_parallel(q, k, v, gam, 3, gate=g)) < TOL

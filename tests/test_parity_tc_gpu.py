@@ -209,3 +209,28 @@ def test_decode7b_after_long_prefill(rn):
         assert slice_rel_err(state.cpu().numpy()[sample], S, head_axis=1) < TOL
         del state
         torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("pairs", [1, 2, 0])
+@pytest.mark.parametrize("B,n,H,chunk", [(2, 1101, 3, 256), (1, 2048, 2, 1024), (2, 640, 2, 512),
+                                         (1, 77, 1, 512), (3, 1500, 2, 512)])
+def test_output_pass_on_pairs_and_single(rn, pairs, B, n, H, chunk):
+    # the same prefill through the paired and the single-CTA output pass:
+    # state in, gate with affine, ragged last chunk
+    q, k, v, g = inputs(B, n, H, 70 + n, gate_width=128)
+    rng = np.random.default_rng(n)
+    s0 = rng.standard_normal((B, H, 256, 256)) * 0.05
+    w = rng.standard_normal(H * 256).astype(np.float32)
+    b = rng.standard_normal(H * 256).astype(np.float32)
+    gam = rn.retnet_default_gammas(H)
+    want, ws = oracle.retention_prefill(q, k, v, np.float32(gam), chunk, pos0=7,
+                                        state_in=np.float32(s0), gate=g,
+                                        weight=w.reshape(H, 256), bias=b.reshape(H, 256))
+    rn.retnet_set_output_pairing(pairs)
+    try:
+        got, st = run(rn, q, k, v, gam, chunk, pos0=7, state_in=s0, gate=g,
+                      weight=torch.from_numpy(w).cuda(), bias=torch.from_numpy(b).cuda())
+    finally:
+        rn.retnet_set_output_pairing(0)
+    assert slice_rel_err(got, want) < TOL
+    assert slice_rel_err(st, ws, head_axis=1) < TOL
