@@ -49,68 +49,80 @@ struct TcHeadParams {
 };
 
 // ------------------------------------------------------------------ prep
-// One CTA per token t: its 128 (cos, sin) pairs are formed once
-// (rotation_cs of (pos0 + t) * theta_j) and applied to every (sequence,
-// head) row of q and k at that token, together with the decay fold.  Writes Qt, Kt in [b*H + h][t][:].
+// One CTA per TOK consecutive tokens: their TOK x 128 (cos, sin) pairs are
+// formed once (rotation_cs of (pos0 + t) * theta_j) and applied to every
+// (sequence, head) row of k (and of q when write_q) at those tokens,
+// together with the decay fold.  Writes Kt (Qt) in [b*H + h][t][:].  TOK
+// grows when there are few sequence-heads, so that each thread still has
+// four 16-byte loads in flight.
 struct TcPrepParams {
     double theta[kD / 2];          // 10000^(-2j/256), formed on the host
     float log2g[kMaxHeads];        // log2(gamma_h)
 };
 
+template <int TOK>
 __global__ void __launch_bounds__(256, 4)
 tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                TcPrepParams pp, __nv_bfloat16 *__restrict__ qt, __nv_bfloat16 *__restrict__ kt,
                int batch, int heads, int n, int chunk, long long pos0, int rotate,
                int write_q, unsigned *err) {
     const long long elems = (long long)batch * n * heads * kD;   // of q, k, Qt and Kt
-    __shared__ float2 cs[kD / 2];
-    const int t = blockIdx.x;
-    const int i = t % chunk;                        // index inside the chunk
-    const int tasks = batch * heads * (kD / 8);
+    __shared__ float2 cs[TOK][kD / 2];
+    const int t0 = blockIdx.x * TOK;
+    const int per_token = batch * heads * (kD / 8);
+    const int tasks = TOK * per_token;
     // Up to kPrepBatch 8-element tasks per thread per round; the first
     // round's loads are issued before the (cos, sin) prologue so its latency
     // overlaps the memory traffic.
     constexpr int kPrepBatch = 4;
     uint4 rq[kPrepBatch] = {}, rk[kPrepBatch];
+    auto task_src = [&](int task, int &u, int &part, int &h, int &b) -> long long {
+        u = task / per_token;
+        const int r = task % per_token;
+        part = r % (kD / 8);
+        const int bhi = r / (kD / 8);
+        h = bhi % heads;
+        b = bhi / heads;
+        return (((long long)b * n + t0 + u) * heads + h) * kD + part * 8;
+    };
     auto load_round = [&](int base) {
 #pragma unroll
-        for (int u = 0; u < kPrepBatch; ++u) {
-            const int task = base + u * blockDim.x;
-            if (task < tasks) {
-                const int part = task % (kD / 8);
-                const int bhi = task / (kD / 8);
-                const int h = bhi % heads, b = bhi / heads;
-                const size_t src = (((size_t)b * n + t) * heads + h) * kD + part * 8;
-                if (!in_bounds((long long)src + 7, elems, err)) continue;
-                if (write_q) rq[u] = *reinterpret_cast<const uint4 *>(q + src);
-                rk[u] = *reinterpret_cast<const uint4 *>(k + src);
+        for (int x = 0; x < kPrepBatch; ++x) {
+            const int task = base + x * blockDim.x;
+            int u, part, h, b;
+            const long long src = task_src(task, u, part, h, b);
+            if (task < tasks && t0 + u < n) {
+                if (!in_bounds(src + 7, elems, err)) continue;
+                if (write_q) rq[x] = *reinterpret_cast<const uint4 *>(q + src);
+                rk[x] = *reinterpret_cast<const uint4 *>(k + src);
             }
         }
     };
     grid_dependency_wait();                         // q, k may come from the kernel before
     load_round(threadIdx.x);
-    if (threadIdx.x < kD / 2) {
-        cs[threadIdx.x] = rotate ? rotation_cs(pos0 + t, pp.theta[threadIdx.x])
-                                 : make_float2(1.f, 0.f);
+    for (int c = threadIdx.x; c < TOK * (kD / 2); c += blockDim.x) {
+        const int u = c / (kD / 2), j = c % (kD / 2);
+        cs[u][j] = rotate ? rotation_cs(pos0 + t0 + u, pp.theta[j]) : make_float2(1.f, 0.f);
     }
     __syncthreads();
     for (int base = threadIdx.x; base < tasks; base += kPrepBatch * blockDim.x) {
         if (base != (int)threadIdx.x) load_round(base);
 #pragma unroll
-        for (int u = 0; u < kPrepBatch; ++u) {
-            const int task = base + u * blockDim.x;
-            if (task < tasks) {
-                const int part = task % (kD / 8);
-                const int bhi = task / (kD / 8);
-                const int h = bhi % heads, b = bhi / heads;
+        for (int x = 0; x < kPrepBatch; ++x) {
+            const int task = base + x * blockDim.x;
+            int u, part, h, b;
+            task_src(task, u, part, h, b);
+            const int t = t0 + u;
+            if (task < tasks && t < n) {
+                const int i = t % chunk;                    // index inside the chunk
                 const float e = (float)(i + 1) * pp.log2g[h];
                 const float sq = exp2f(e), sk = exp2f(-e);
-                const __nv_bfloat162 *hq = reinterpret_cast<const __nv_bfloat162 *>(&rq[u]);
-                const __nv_bfloat162 *hk = reinterpret_cast<const __nv_bfloat162 *>(&rk[u]);
+                const __nv_bfloat162 *hq = reinterpret_cast<const __nv_bfloat162 *>(&rq[x]);
+                const __nv_bfloat162 *hk = reinterpret_cast<const __nv_bfloat162 *>(&rk[x]);
                 float oq[8], ok[8];
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
-                    const float2 r = cs[part * 4 + p];
+                    const float2 r = cs[u][part * 4 + p];
                     const float cq = r.x * sq, sq2 = r.y * sq, ck = r.x * sk, sk2 = r.y * sk;
                     const float2 xq = __bfloat1622float2(hq[p]);
                     const float2 xk = __bfloat1622float2(hk[p]);
@@ -119,8 +131,8 @@ tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
                     ok[2 * p] = xk.x * ck - xk.y * sk2;
                     ok[2 * p + 1] = xk.x * sk2 + xk.y * ck;
                 }
-                const size_t dst = (((size_t)b * heads + h) * n + t) * kD + part * 8;
-                if (!in_bounds((long long)dst + 7, elems, err)) continue;
+                const long long dst = (((long long)b * heads + h) * n + t) * kD + part * 8;
+                if (!in_bounds(dst + 7, elems, err)) continue;
                 if (write_q) store8(qt + dst, oq);
                 store8(kt + dst, ok);
             }
@@ -1618,10 +1630,21 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
         TcPrepParams pp;
         for (int j = 0; j < kD / 2; ++j) pp.theta[j] = pp_theta[j];
         for (int h = 0; h < kMaxHeads; ++h) pp.log2g[h] = hp.log2g[h];
+        // tokens per CTA: enough (sequence, head) rows for 1024 tasks of 8 elements
+        const int per_token = BH * (kD / 8);
+        const int tok = per_token >= 1024 ? 1 : per_token >= 512 ? 2 : 4;
         KernelTimer timer("tc_prep", stream);
-        e = launch_overlapped(tc_prep_kernel, dim3(n), dim3(256), 0, stream,
-                              (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, pp, qt, kt,
-                              B, H, n, fold, a.pos0, a.rotate, fold_q ? 0 : 1, err);
+        const __nv_bfloat16 *qq = (const __nv_bfloat16 *)a.q, *kk = (const __nv_bfloat16 *)a.k;
+        const int wq = fold_q ? 0 : 1;
+        if (tok == 1)
+            e = launch_overlapped(tc_prep_kernel<1>, dim3(n), dim3(256), 0, stream, qq, kk, pp,
+                                  qt, kt, B, H, n, fold, a.pos0, a.rotate, wq, err);
+        else if (tok == 2)
+            e = launch_overlapped(tc_prep_kernel<2>, dim3((n + 1) / 2), dim3(256), 0, stream, qq,
+                                  kk, pp, qt, kt, B, H, n, fold, a.pos0, a.rotate, wq, err);
+        else
+            e = launch_overlapped(tc_prep_kernel<4>, dim3((n + 3) / 4), dim3(256), 0, stream, qq,
+                                  kk, pp, qt, kt, B, H, n, fold, a.pos0, a.rotate, wq, err);
         count_launch();
         if (e != cudaSuccess) return e;
     }
