@@ -217,6 +217,206 @@ gemm_bf16_tn_kernel(const __grid_constant__ CUtensorMap tm_x,
     }
 }
 
+// Paired variant: a cluster of two CTAs computes a 256 x 256 tile with
+// tcgen05 cta_group::2 (M = 256).  CTA k loads rows [128k, 128k+128) of the
+// tile's X block and rows [128k, 128k+128) of its W block (half of N), so a
+// 64-wide K step costs each CTA 32 KB of loads instead of 48 KB; each CTA
+// keeps its 128 rows x 256 columns of the product in its own TMEM (two
+// accumulators).  The leader (rank 0) issues the MMAs; both CTAs' loads
+// count on the leader's full barrier, and its commits arrive on both CTAs'
+// empty and acc_full barriers.  On an abort the leader settles and drains
+// the loads of both CTAs before the pair's last cluster barrier.
+constexpr int kPairM = 256;                // rows per pair tile
+constexpr int kPairStages = 6;
+constexpr uint32_t kPairHalf = kGemmM * kGemmK * 2;          // 16 KB: 128 rows x 64
+constexpr uint32_t kPairStage = 2 * kPairHalf;               // 32 KB per CTA
+constexpr uint32_t kPairSmem = kPairStages * kPairStage + 1024;
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+gemm_bf16_tn_pair_kernel(const __grid_constant__ CUtensorMap tm_x,
+                         const __grid_constant__ CUtensorMap tm_w, GemmArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    __shared__ uint64_t full[kPairStages], empty[kPairStages], acc_full[2], acc_free[2], drain;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int abort_flag, issued;
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    unsigned *err = a.err;
+    const int tiles = a.tiles_m * a.tiles_n;        // tiles_m counts 256-row blocks here
+    const int ksteps = (a.k + kGemmK - 1) / kGemmK;
+    const int cluster = blockIdx.x / 2, nclusters = gridDim.x / 2;
+    const uint32_t peer_abort = mapa_shared(smem_u32(&abort_flag), rank ^ 1u);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPairStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&acc_full[x], 1);
+            mbar_init(&acc_free[x], 2 * 128);
+        }
+        mbar_init(&drain, 1);
+        abort_flag = 0;
+        issued = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(&tmem_slot, 512);
+        tmem_relinquish_pair();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_w);
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+    grid_dependency_wait();
+    auto abort_both = [&]() {
+        abort_flag = 1;
+        st_cluster_u32(peer_abort, 1u);
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            bool ok = true;
+            int it = 0;
+            for (int t = cluster; ok && t < tiles; t += nclusters) {
+                int mb, nb;
+                gemm_tile(a, t, mb, nb);
+                for (int ks = 0; ks < ksteps; ++ks) {
+                    const int s = it % kPairStages;
+                    if (it >= kPairStages &&
+                        !mbar_wait(&empty[s], ((it / kPairStages) - 1) & 1, &abort_flag, err)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *ab = smem + s * kPairStage;
+                    const uint32_t lbar = mapa_shared(smem_u32(&full[s]), 0);
+                    if (leader) mbar_expect_tx(&full[s], 2 * kPairStage);
+                    tma_load_2d_pair(ab, &tm_x, lbar, ks * kGemmK, mb * kPairM + kGemmM * (int)rank);
+                    tma_load_2d_pair(ab + kPairHalf, &tm_w, lbar, ks * kGemmK,
+                                     nb * kGemmN + kGemmM * (int)rank);
+                    ++it;
+                    *(volatile int *)&issued = it;
+                }
+            }
+            if (!ok) abort_both();
+        }
+    } else if (warp == 1) {
+        if (leader && lane == 0) {
+            const uint32_t idesc = idesc_bf16(kPairM, kGemmN, 0, 0);
+            int it = 0, lt = 0;
+            bool ok = true;
+            for (int t = cluster; ok && t < tiles; t += nclusters, ++lt) {
+                const int buf = lt & 1;
+                if (lt >= 2 && !mbar_wait(&acc_free[buf], ((lt - 2) >> 1) & 1, &abort_flag, err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (int ks = 0; ks < ksteps; ++ks, ++it) {
+                    const int s = it % kPairStages;
+                    if (!mbar_wait(&full[s], (it / kPairStages) & 1, &abort_flag, err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t ab = smem_u32(smem + s * kPairStage);
+                    const uint32_t bb = ab + kPairHalf;
+#pragma unroll
+                    for (int kk = 0; kk < kGemmK / 16; ++kk)
+                        mma_bf16_pair(tmem + kGemmN * buf, smem_desc_sw128(ab + kk * 32, 16, 1024),
+                                      smem_desc_sw128(bb + kk * 32, 16, 1024), idesc,
+                                      (ks > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit_pair(&empty[s], 3);
+                }
+                if (ok) mma_commit_pair(&acc_full[buf], 3);
+            }
+            if (!ok) abort_both();
+        }
+    } else {
+        const int q4 = warp % 4;
+        const int row = 32 * q4 + lane;
+        const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
+        int lt = 0;
+        bool ok = true;
+        for (int t = cluster; t < tiles; t += nclusters, ++lt) {
+            const int buf = lt & 1;
+            if (!warp_wait(&acc_full[buf], (lt >> 1) & 1, &abort_flag, err)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            int mb, nb;
+            gemm_tile(a, t, mb, nb);
+            const long long grow = (long long)mb * kPairM + kGemmM * (int)rank + row;
+            const int col0 = nb * kGemmN;
+            const int which = col0 / a.n_split;
+            const int c_in = col0 % a.n_split;
+            const bool live = grow < a.m && in_bounds(which, 4, err);
+            __nv_bfloat16 *base = which == 0   ? a.out[0]
+                                  : which == 1 ? a.out[1]
+                                  : which == 2 ? a.out[2]
+                                               : a.out[3];
+            __nv_bfloat16 *dst = live ? base + grow * a.n_split + c_in : nullptr;
+            const uint32_t l_free = mapa_shared(smem_u32(&acc_free[buf]), 0);
+#pragma unroll 1
+            for (int cb = 0; cb < kGemmN / 32; ++cb) {
+                uint32_t v[32];
+                tmem_ld32(tmem + kGemmN * buf + lane_off + 32 * cb, v);
+                tmem_wait_ld();
+                if (cb == kGemmN / 32 - 1) {
+                    tc_fence_before();
+                    mbar_arrive_cluster(l_free);
+                }
+                if (live) {
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * cb);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        d4[q] = make_uint4(
+                            pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                            pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                            pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                            pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+                }
+            }
+        }
+        if (!ok && lane == 0) abort_both();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    // After an abort: the leader settles the loads only one CTA issued and
+    // drains the last stages of both; then the MMAs.
+    if (abort_flag && leader && warp == 0 && lane == 0) {
+        const int own = issued;
+        const int peer = (int)ld_cluster_u32(mapa_shared(smem_u32(&issued), 1));
+        const int last = max(own, peer);
+        for (int j = max(0, last - kPairStages); j < last; ++j) {
+            uint64_t *bar = &full[j % kPairStages];
+            if (j >= own) mbar_expect_tx(bar, kPairStage);
+            else if (j >= peer) mbar_complete_tx(bar, kPairStage);
+            mbar_drain(bar, (j / kPairStages) & 1, err);
+        }
+    }
+    if (abort_flag && leader && warp == 1 && lane == 0) {
+        mma_commit_pair(&drain, 1);
+        mbar_drain(&drain, 0, err);
+    }
+    tc_fence_before();
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, 512);
+    }
+}
+
 }  // namespace
 
 bool gemm_shape_ok(long long m, int n, int k, int n_split) {
@@ -248,16 +448,48 @@ cudaError_t launch_gemm_bf16(const void *x, const void *w, void *const *outs, lo
     a.n = n;
     a.k = k;
     a.n_split = n_split;
-    a.tiles_m = (int)((m + kGemmM - 1) / kGemmM);
     a.tiles_n = n / kGemmN;
     a.err = device_error_word();
     if (!a.err) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tn_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
-    if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaError_t e;
+    // CTA pairs (256-row tiles) unless the rows fill no more than one
+    // 128-row block per tile column
+    if (output_pairing_mode() != 0 && m > kGemmM) {
+        a.tiles_m = (int)((m + kPairM - 1) / kPairM);
+        CUtensorMap tm_wh;                          // W in halves of 128 rows
+        {
+            cuuint64_t dims[2] = {(cuuint64_t)k, (cuuint64_t)n};
+            cuuint64_t str[1] = {(cuuint64_t)k * 2};
+            cuuint32_t box[2] = {kGemmK, kGemmM};
+            if (!make_tensor_map_bf16(&tm_wh, w, 2, dims, str, box)) return cudaErrorInvalidValue;
+        }
+        e = cudaFuncSetAttribute(gemm_bf16_tn_pair_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmem);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t qc = {};
+        qc.gridDim = dim3(2 * (unsigned)std::max(1, sms / 2));
+        qc.blockDim = dim3(kGemmThreads);
+        qc.dynamicSmemBytes = kPairSmem;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, gemm_bf16_tn_pair_kernel, &qc) !=
+                cudaSuccess ||
+            clusters < 1)
+            clusters = std::max(1, sms / 2);
+        const long long tiles = (long long)a.tiles_m * a.tiles_n;
+        clusters = (int)std::min<long long>(tiles, clusters);
+        KernelTimer timer(timer_name, stream);
+        e = launch_overlapped(gemm_bf16_tn_pair_kernel, dim3(2 * clusters), dim3(kGemmThreads),
+                              kPairSmem, stream, tm_x, tm_wh, a);
+        count_launch();
+        return e;
+    }
+    a.tiles_m = (int)((m + kGemmM - 1) / kGemmM);
+    e = cudaFuncSetAttribute(gemm_bf16_tn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kGemmSmem);
+    if (e != cudaSuccess) return e;
     const long long tiles = (long long)a.tiles_m * a.tiles_n;
     const unsigned grid = (unsigned)std::min<long long>(tiles, sms);
     KernelTimer timer(timer_name, stream);
