@@ -372,6 +372,12 @@ RETNET_API retnet_status retnet_check_device_errors(retnet_stream_t stream);
  * Errors: INVALID_ARG, CUDA. */
 RETNET_API retnet_status retnet_test_set_hooks(unsigned long long wait_limit_ns,
                                                int skip_first_state_load);
+/* Debug build only: synchronises `stream` and returns in *word the raw
+ * device error word (bit 0 timeout, bit 1 index check, and one bit per
+ * kernel whose index check failed: 1<<8 prep, 1<<9 state, 1<<10 output,
+ * 1<<11 paired output, 1<<12 decode, 1<<13 projection GEMM), clearing it.
+ * Errors: INVALID_ARG, CUDA. */
+RETNET_API retnet_status retnet_test_error_word(retnet_stream_t stream, unsigned *word);
 #endif
 
 /* ---- Kernel timer (diagnostics; off by default) ----------------------

@@ -457,6 +457,21 @@ retnet_status retnet_groupnorm_swish(const void *o, const void *g, const float *
     return RETNET_OK;
 }
 
+#ifdef RETNET_TEST_HOOKS
+// Debug build only: synchronises `stream`, returns the raw device error word
+// (timeout and bounds bits, with the kSite* bits of the kernels whose index
+// checks failed) in *word and clears it.
+RETNET_API retnet_status retnet_test_error_word(retnet_stream_t stream, unsigned *word) {
+    if (!word) return RETNET_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return RETNET_ERR_CUDA;
+    unsigned zero = 0;
+    if (cudaMemcpyFromSymbol(word, g_device_error, sizeof(*word)) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+        return RETNET_ERR_CUDA;
+    return RETNET_OK;
+}
+#endif
+
 retnet_status retnet_check_device_errors(retnet_stream_t stream) {
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return RETNET_ERR_CUDA;
     unsigned word = 0, zero = 0;

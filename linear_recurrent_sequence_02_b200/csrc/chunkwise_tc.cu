@@ -92,7 +92,7 @@ tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
             int u, part, h, b;
             const long long src = task_src(task, u, part, h, b);
             if (task < tasks && t0 + u < n) {
-                if (!in_bounds(src + 7, elems, err)) continue;
+                if (!in_bounds(src + 7, elems, err, kSitePrep)) continue;
                 if (write_q) rq[x] = *reinterpret_cast<const uint4 *>(q + src);
                 rk[x] = *reinterpret_cast<const uint4 *>(k + src);
             }
@@ -132,7 +132,7 @@ tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
                     ok[2 * p + 1] = xk.x * sk2 + xk.y * ck;
                 }
                 const long long dst = (((long long)b * heads + h) * n + t) * kD + part * 8;
-                if (!in_bounds(dst + 7, elems, err)) continue;
+                if (!in_bounds(dst + 7, elems, err, kSitePrep)) continue;
                 if (write_q) store8(qt + dst, oq);
                 store8(kt + dst, ok);
             }
@@ -291,7 +291,7 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const long long state_elems = nbh * kD * kD;
         const long long sprev_elems = nbh * nchunks * kD * kD;
         float st[DVC];
-        if (state_in && in_bounds((long long)sbase + DVC - 1, state_elems, err)) {
+        if (state_in && in_bounds((long long)sbase + DVC - 1, state_elems, err, kSiteState)) {
             const float4 *src = reinterpret_cast<const float4 *>(state_in + sbase);
 #pragma unroll
             for (int v4 = 0; v4 < DVC / 4; ++v4) {
@@ -304,7 +304,7 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
         {
             const size_t o0 = ((size_t)bh * nchunks * kD + krow) * kD + DVC * nv;
-            if (in_bounds((long long)o0 + DVC - 1, sprev_elems, err))
+            if (in_bounds((long long)o0 + DVC - 1, sprev_elems, err, kSiteState))
                 store_bf16_row(s_prev + o0, st, DVC);
         }
         for (int c = 0; c < nchunks; ++c) {
@@ -326,9 +326,9 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             mbar_arrive(&acc_free[buf]);                     // buffer free for chunk c + 2
             if (!last) {
                 const size_t o1 = (((size_t)bh * nchunks + c + 1) * kD + krow) * kD + DVC * nv;
-                if (in_bounds((long long)o1 + DVC - 1, sprev_elems, err))
+                if (in_bounds((long long)o1 + DVC - 1, sprev_elems, err, kSiteState))
                     store_bf16_row(s_prev + o1, st, DVC);
-            } else if (state_out && in_bounds((long long)sbase + DVC - 1, state_elems, err)) {
+            } else if (state_out && in_bounds((long long)sbase + DVC - 1, state_elems, err, kSiteState)) {
                 float4 *o = reinterpret_cast<float4 *>(state_out + sbase);
 #pragma unroll
                 for (int v4 = 0; v4 < DVC / 4; ++v4)
@@ -509,8 +509,8 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 if (!m.valid) continue;
                 const int srow = (m.bh * a.nchunks + m.c) * kD;
                 // debug build: the item's tile coordinates lie inside its tensors
-                if (!in_bounds(m.t0row, a.n, err) || !in_bounds(m.bh, nbh, err) ||
-                    !in_bounds(srow + kD - 1, nbh * a.nchunks * kD, err)) {
+                if (!in_bounds(m.t0row, a.n, err, kSiteOutput) || !in_bounds(m.bh, nbh, err, kSiteOutput) ||
+                    !in_bounds(srow + kD - 1, nbh * a.nchunks * kD, err, kSiteOutput)) {
                     abort_flag = 1;
                     ok = false;
                     break;
@@ -849,10 +849,15 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 // Roles as in tc_output, with the leader (rank 0) issuing every MMA:
 //   warp 0 (both CTAs): TMA loads into its own slots.  Operand loads count
 //     on the leader's rfull barrier of the slot (the leader arms it for both
-//     CTAs' bytes); the gate/output tile (two slots) counts on this CTA's
-//     own lfull barriers.  Each CTA completes one lfull phase, and the
-//     leader one rfull phase, for every ring item, so that both follow the
-//     ring order whatever the slot holds.
+//     CTAs' bytes); the gate/output tile (two slots), and raw q when the
+//     pair folds it, count on this CTA's own lfull barriers.  Each CTA
+//     completes one lfull phase for every ring item, so lfull follows the
+//     ring order; rfull[s] has one phase per operand item of slot s, and
+//     its users count those per slot.  A CTA can refill a gate slot as soon
+//     as its own epilogue is done, possibly before the other CTA reaches it;
+//     counting rfull phases per operand item keeps such a load in the phase
+//     of its own item (its slot's previous operand item was consumed before
+//     the slot could pass on).
 //   warp 1: TMEM allocation (both CTAs, paired); the leader's lane 0
 //     issues the copies and MMAs, whose commits arrive on the barrier of
 //     the same offset in both CTAs (rempty, s_full, p_free, o_full).
@@ -913,8 +918,8 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     __shared__ uint64_t s_full, s_read, p_full[2], p_free[2], o_full, o_free, drain, q_ready;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
-    __shared__ int issued;                         // ring items this CTA issued
-    __shared__ uint32_t slot_op[kPairSlots];       // latest item of the slot: 1 operand, 0 gate
+    __shared__ uint32_t op_n[kPairSlots];          // operand items this CTA issued per slot
+    __shared__ uint32_t lf_n[kPairSlots];          // lfull phases this CTA armed per slot
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const uint32_t rank = cluster_ctarank();
@@ -946,8 +951,7 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_init(&drain, 1);
         mbar_init(&q_ready, 2 * kFoldThreads);
         abort_flag = 0;
-        issued = 0;
-        for (int s = 0; s < kPairSlots; ++s) slot_op[s] = 0;
+        for (int s = 0; s < kPairSlots; ++s) op_n[s] = lf_n[s] = 0;
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -988,7 +992,8 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                 uint8_t *d = slot_ptr(it);
                 uint64_t *bar = &rfull[it % kPairSlots];
                 const uint32_t lbar = at_leader(bar);
-                slot_op[it % kPairSlots] = 1;
+                *(volatile uint32_t *)&op_n[it % kPairSlots] += 1;
+                *(volatile uint32_t *)&lf_n[it % kPairSlots] += 1;
                 mbar_arrive(&lfull[it % kPairSlots]);          // keeps lfull in ring order
                 if (leader) mbar_expect_tx(bar, 2 * kPairSlot);
                 if (kind == 0) {                               // Qt: two 64-col boxes
@@ -1006,14 +1011,13 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                                          c1, c3);
                 }
                 ++it;
-                *(volatile int *)&issued = it;
             };
             for (int w = cluster; ok && w < a.items; w += nclusters) {
                 const TcPairItem m = tc_pair_item(a, w, rank);
                 if (!m.valid) continue;
                 const int srow = (m.bh * a.nchunks + m.c) * kD;
-                if (!in_bounds(m.bh, nbh, err) ||
-                    !in_bounds(srow + kD - 1, nbh * a.nchunks * kD, err)) {
+                if (!in_bounds(m.bh, nbh, err, kSiteOutputPair) ||
+                    !in_bounds(srow + kD - 1, nbh * a.nchunks * kD, err, kSiteOutputPair)) {
                     ok = false;
                     abort_both();
                     break;
@@ -1025,14 +1029,12 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                         // warps (counted on lfull; rfull only kept in order)
                         uint8_t *d = slot_ptr(it);
                         uint64_t *lb = &lfull[it % kPairSlots];
-                        slot_op[it % kPairSlots] = 0;
-                        if (leader) mbar_arrive(&rfull[it % kPairSlots]);
+                        *(volatile uint32_t *)&lf_n[it % kPairSlots] += 1;
                         mbar_expect_tx(lb, kPairSlot);
                         for (int x = 0; x < 2; ++x)
                             tma_load_4d(d + x * kBox, &tm_qraw, lb, 128 * half + 64 * x, m.h,
                                         m.t0row, m.b);
                         ++it;
-                        *(volatile int *)&issued = it;
                     } else {
                         issue_op(0, m.t0row, m.bh, 2 * half);
                     }
@@ -1061,8 +1063,7 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                     if (!(ok = acquire())) break;
                     uint8_t *gs = slot_ptr(it);
                     uint64_t *lb = &lfull[it % kPairSlots];
-                    slot_op[it % kPairSlots] = 0;
-                    if (leader) mbar_arrive(&rfull[it % kPairSlots]);   // keeps rfull in order
+                    *(volatile uint32_t *)&lf_n[it % kPairSlots] += 1;
                     if (a.has_gate) {
                         mbar_expect_tx(lb, 2 * kBox);
                         for (int x = 0; x < 2; ++x)
@@ -1072,7 +1073,6 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                         mbar_arrive(lb);
                     }
                     ++it;
-                    *(volatile int *)&issued = it;
                 }
             }
             if (!ok) abort_both();
@@ -1083,10 +1083,12 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
             const uint32_t id_pv = idesc_bf16(256, 256, 0, 1);
             const uint32_t sP = smem_u32(pbuf);
             int it = 0, nqk = 0, npv = 0, li = 0;
+            uint32_t opar = 0;                         // per slot: parity of its next rfull phase
             bool ok = true;
             auto take = [&]() -> bool {
-                if (!mbar_wait(&rfull[it % kPairSlots], (it / kPairSlots) & 1, &abort_flag, err))
-                    return false;
+                const int s = it % kPairSlots;
+                if (!mbar_wait(&rfull[s], (opar >> s) & 1u, &abort_flag, err)) return false;
+                opar ^= 1u << s;
                 tc_fence_after();
                 return true;
             };
@@ -1427,27 +1429,20 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     // (they count on its barriers) and its MMAs; each CTA its own gate loads.
     const bool aborted = abort_flag != 0;
     if (aborted && warp == 0 && lane == 0) {
-        for (int j = max(0, issued - kPairSlots); j < issued; ++j)
-            mbar_drain(&lfull[j % kPairSlots], (j / kPairSlots) & 1, err);
+        // each CTA: the latest armed lfull phase of every slot (gate tiles, raw q)
+        for (int j = 0; j < kPairSlots; ++j)
+            if (lf_n[j] > 0) mbar_drain(&lfull[j], (lf_n[j] - 1) & 1, err);
         if (leader) {
-            // Both CTAs walk the same ring order, at most kPairSlots items past
-            // the MMAs' progress, so the items still open are the last
-            // kPairSlots of the further producer; gate items never count on
-            // rfull beyond the leader's own arrival.
-            const int own = issued;
-            const int peer = (int)ld_cluster_u32(mapa_shared(smem_u32(&issued), 1));
-            const int last = max(own, peer);
-            for (int j = max(0, last - kPairSlots); j < last; ++j) {
-                uint64_t *bar = &rfull[j % kPairSlots];
-                if (j >= own) {                                // only the peer reached it
-                    const uint32_t op =
-                        ld_cluster_u32(mapa_shared(smem_u32(&slot_op[j % kPairSlots]), 1));
-                    if (!op) continue;
-                    mbar_expect_tx(bar, kPairSlot);
-                } else if (j >= peer && slot_op[j % kPairSlots]) {
-                    mbar_complete_tx(bar, kPairSlot);          // the peer never loaded its half
-                }
-                mbar_drain(bar, (j / kPairSlots) & 1, err);
+            // Each producer runs at most kPairSlots ring items past the MMAs,
+            // so every slot has at most one operand phase still open, and the
+            // two CTAs' operand counts of a slot differ by at most one.
+            for (int j = 0; j < kPairSlots; ++j) {
+                const uint32_t own = op_n[j];
+                const uint32_t peer = ld_cluster_u32(mapa_shared(smem_u32(&op_n[j]), 1));
+                if (own == 0 && peer == 0) continue;
+                if (peer > own) mbar_expect_tx(&rfull[j], kPairSlot);       // only the peer loaded
+                else if (own > peer) mbar_complete_tx(&rfull[j], kPairSlot); // only the leader
+                mbar_drain(&rfull[j], ((own > peer ? own : peer) - 1) & 1, err);
             }
         }
     }

@@ -79,14 +79,22 @@ class SymbolAddressCache {
 // in_bounds(i, n, err) tests 0 <= i < n; a failed test records kDevErrBounds
 // in the error word and the caller skips the access.  Without it the test
 // is the constant true and compiles away.
+// `site` (one of the kSite* bits) also goes into the word, so a debug run
+// can tell which kernel's check failed (retnet_test_error_word).
+enum BoundsSite : unsigned {
+    kSitePrep = 1u << 8, kSiteState = 1u << 9, kSiteOutput = 1u << 10,
+    kSiteOutputPair = 1u << 11, kSiteStep = 1u << 12, kSiteGemm = 1u << 13,
+};
 #ifdef RETNET_CHECK_BOUNDS
-__device__ __forceinline__ bool in_bounds(long long i, long long n, unsigned *err) {
+__device__ __forceinline__ bool in_bounds(long long i, long long n, unsigned *err,
+                                          unsigned site = 0) {
     if (i >= 0 && i < n) return true;
-    if (err) atomicOr(err, (unsigned)kDevErrBounds);
+    if (err) atomicOr(err, (unsigned)kDevErrBounds | site);
     return false;
 }
 #else
-__device__ __forceinline__ constexpr bool in_bounds(long long, long long, unsigned *) {
+__device__ __forceinline__ constexpr bool in_bounds(long long, long long, unsigned *,
+                                                    unsigned = 0) {
     return true;
 }
 #endif

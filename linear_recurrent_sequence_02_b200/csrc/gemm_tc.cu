@@ -169,7 +169,7 @@ gemm_bf16_tn_kernel(const __grid_constant__ CUtensorMap tm_x,
             const int col0 = nb * kGemmN;
             const int which = col0 / a.n_split;
             const int c_in = col0 % a.n_split;
-            const bool live = grow < a.m && in_bounds(which, 4, err);
+            const bool live = grow < a.m && in_bounds(which, 4, err, kSiteGemm);
             // (a select chain, not a dynamic index, keeps a.out out of local memory)
             __nv_bfloat16 *base = which == 0   ? a.out[0]
                                   : which == 1 ? a.out[1]
@@ -359,7 +359,7 @@ gemm_bf16_tn_pair_kernel(const __grid_constant__ CUtensorMap tm_x,
             const int col0 = nb * kGemmN;
             const int which = col0 / a.n_split;
             const int c_in = col0 % a.n_split;
-            const bool live = grow < a.m && in_bounds(which, 4, err);
+            const bool live = grow < a.m && in_bounds(which, 4, err, kSiteGemm);
             __nv_bfloat16 *base = which == 0   ? a.out[0]
                                   : which == 1 ? a.out[1]
                                   : which == 2 ? a.out[2]

@@ -128,8 +128,8 @@ retention_step_kernel(const T *__restrict__ q, const T *__restrict__ k,
     grid_dependency_wait();          // the state may come from the kernel before
 #ifdef RETNET_CHECK_BOUNDS
     // debug build: this CTA's (sequence, head) row and columns exist
-    if (!__syncthreads_and(in_bounds(bh, bh_total, err) &&
-                           in_bounds(col0 + cgi * 4 + 3, dv, err)))
+    if (!__syncthreads_and(in_bounds(bh, bh_total, err, kSiteStep) &&
+                           in_bounds(col0 + cgi * 4 + 3, dv, err, kSiteStep)))
         return;
 #endif
     // Issue this thread's state loads first: they do not depend on q, k, v.
@@ -197,9 +197,9 @@ retention_tokens_kernel(const T *__restrict__ q, const T *__restrict__ k,
     grid_dependency_wait();          // the state may come from the kernel before
 #ifdef RETNET_CHECK_BOUNDS
     // debug build: this CTA's row, columns and tokens exist
-    if (!__syncthreads_and(in_bounds(bh, bh_total, err) &&
-                           in_bounds(col0 + cgi * 4 + 3, dv, err) &&
-                           in_bounds(tok0 + ntok - 1, tokens, err)))
+    if (!__syncthreads_and(in_bounds(bh, bh_total, err, kSiteStep) &&
+                           in_bounds(col0 + cgi * 4 + 3, dv, err, kSiteStep) &&
+                           in_bounds(tok0 + ntok - 1, tokens, err, kSiteStep)))
         return;
 #endif
     float *S = state + (size_t)bh * DK * dv + col0 + cgi * 4;
