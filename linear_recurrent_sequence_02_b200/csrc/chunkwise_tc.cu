@@ -941,15 +941,16 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
             mbar_init(&lfull[s], 1);
         }
         mbar_init(&s_full, 1);
-        mbar_init(&s_read, 2 * kEpiThreads);
+        // cross-CTA signals arrive once per warp (lane 0, after __syncwarp)
+        mbar_init(&s_read, 2 * kEpiThreads / 32);
         for (int x = 0; x < 2; ++x) {                    // one P half per warpgroup, both CTAs
-            mbar_init(&p_full[x], kEpiThreads);
+            mbar_init(&p_full[x], 2 * (kEpiThreads / 2) / 32);
             mbar_init(&p_free[x], 1);
         }
         mbar_init(&o_full, 1);
-        mbar_init(&o_free, 2 * kEpiThreads);
+        mbar_init(&o_free, 2 * kEpiThreads / 32);
         mbar_init(&drain, 1);
-        mbar_init(&q_ready, 2 * kFoldThreads);
+        mbar_init(&q_ready, 2 * kFoldThreads / 32);
         abort_flag = 0;
         for (int s = 0; s < kPairSlots; ++s) op_n[s] = lf_n[s] = 0;
         fence_barrier_init();
@@ -1216,8 +1217,8 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                 if (!m.valid) continue;
                 const int qi = it_base;
                 it_base += 2 + 2 * m.nk + m.nsp + 2;
-                const int qs = qi + bx / 2;                    // this column's slot
-                if (!mbar_wait(&lfull[qs % kPairSlots], (qs / kPairSlots) & 1, &abort_flag, err)) {
+                const int qs = qi + bx / 2;                    // this column's slot (warp-uniform)
+                if (!warp_wait(&lfull[qs % kPairSlots], (qs / kPairSlots) & 1, &abort_flag, err)) {
                     ok = false;
                     break;
                 }
@@ -1251,7 +1252,8 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                     }
                 }
                 fence_async_shared();
-                mbar_arrive_cluster(l_q_ready);
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(l_q_ready);
             }
             if (!ok && lane == 0) abort_both();
         }
@@ -1278,7 +1280,8 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                 tmem_ld32(col + 32, v1);
                 tmem_wait_ld();
                 tc_fence_before();
-                mbar_arrive_cluster(l_s_read);                  // S may be overwritten now
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(l_s_read);   // S may be overwritten now
                 const int j0 = t * kKeyTile + 64 * wg;
                 uint32_t wv[32];
                 if (a.parallel && t < m.r) {
@@ -1313,7 +1316,8 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                         make_uint4(wv[4 * ch], wv[4 * ch + 1], wv[4 * ch + 2], wv[4 * ch + 3]);
                 fence_async_shared();
                 tc_fence_before();
-                mbar_arrive_cluster(l_p_full);
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(l_p_full);
             }
             // ring items of this pair-item: Qt (2), nk Kt halves, nsp S_prev
             // halves, nk V halves, then the gate/output tile (2 slots)
@@ -1369,7 +1373,8 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                     tmem_wait_ld();
                     if (k4 == 3) {
                         tc_fence_before();
-                        mbar_arrive_cluster(l_o_free);
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_cluster(l_o_free);
                     }
                     const int bx = cb >> 1;                       // 64-column box
                     uint8_t *box = (bx < 2 ? ya : yb) + (bx % 2) * kBox + row * 128;
@@ -1403,7 +1408,8 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                 }
                 fence_async_shared();
             } else {
-                mbar_arrive_cluster(l_o_free);
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(l_o_free);
             }
             named_barrier(1, kEpiThreads);
             if (wg == 0 && row == 0) {
