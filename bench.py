@@ -333,7 +333,8 @@ def run_ours(args, w, chunk):
         dist.barrier()
     rn.load_library()
     rn.retnet_set_launch_overlap(not args.no_overlap)
-    rn.retnet_set_output_pairing(args.pairs)
+    if args.pairs is not None:
+        rn.retnet_set_output_pairing(args.pairs)
 
     line = measure_prefill(args, w, chunk, rank, world, dev, full=True)
     line["output_pairs"] = args.pairs
@@ -658,7 +659,8 @@ def run_backward(args, w, chunk):
     build()
     rn.load_library()
     rn.retnet_set_launch_overlap(not args.no_overlap)
-    rn.retnet_set_output_pairing(args.pairs)
+    if args.pairs is not None:
+        rn.retnet_set_output_pairing(args.pairs)
     B, n, H, d = w.batch, w.seqlen, w.heads, w.d
     gam = rn.retnet_default_gammas(H)
     sets = []
@@ -912,7 +914,8 @@ def run_layer(args, w, chunk):
     build()
     rn.load_library()
     rn.retnet_set_launch_overlap(not args.no_overlap)
-    rn.retnet_set_output_pairing(args.pairs)
+    if args.pairs is not None:
+        rn.retnet_set_output_pairing(args.pairs)
     B, n, H, d = w.batch, w.seqlen, w.heads, w.d
     hidden = w.hidden or H * d
     gam = rn.retnet_default_gammas(H)
@@ -1026,9 +1029,9 @@ def main():
                     help="time the backward pass of the prefill (no epilogue) instead")
     ap.add_argument("--no-overlap", action="store_true",
                     help="launch kernels without programmatic launch overlap")
-    ap.add_argument("--pairs", type=int, choices=[0, 1, 2], default=1,
-                    help="output pass: 1 CTA pairs folding q (default), 2 CTA pairs with q "
-                         "folded by the prep pass, 0 single CTAs")
+    ap.add_argument("--pairs", type=int, choices=[0, 1, 2], default=None,
+                    help="output pass: 1 CTA pairs folding q, 2 CTA pairs with q folded by the "
+                         "prep pass, 0 single CTAs (default: the library's own default)")
     ap.add_argument("--layer", action="store_true",
                     help="time the whole multi-scale retention layer (projections included)")
     ap.add_argument("--form", choices=["chunkwise", "parallel"], default="chunkwise",

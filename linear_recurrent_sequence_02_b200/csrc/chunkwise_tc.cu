@@ -49,93 +49,93 @@ struct TcHeadParams {
 };
 
 // ------------------------------------------------------------------ prep
-// One CTA per TOK consecutive tokens: their TOK x 128 (cos, sin) pairs are
-// formed once (rotation_cs of (pos0 + t) * theta_j) and applied to every
-// (sequence, head) row of k (and of q when write_q) at those tokens,
-// together with the decay fold.  Writes Kt (Qt) in [b*H + h][t][:].  TOK
-// grows when there are few sequence-heads, so that each thread still has
-// four 16-byte loads in flight.
+// Rotation and decay fold of k (and of q when write_q) into Kt (Qt), laid
+// out [b*H + h][t][256].  One CTA per TOK consecutive tokens: their
+// TOK x 128 (cos, sin) pairs are formed once (rotation_cs of
+// (pos0 + t) * theta_j) in shared memory.  Each warp then takes whole
+// (token, sequence, head) rows of 256 elements, one 16-byte part per lane
+// (fully coalesced), four rows per round with all their loads issued before
+// any arithmetic; the row's (token, sequence, head) indices advance by
+// additions, so no per-element division is left.  TOK is chosen so that a
+// CTA has about 64 rows.
 struct TcPrepParams {
     double theta[kD / 2];          // 10000^(-2j/256), formed on the host
     float log2g[kMaxHeads];        // log2(gamma_h)
 };
 
 template <int TOK>
-__global__ void __launch_bounds__(256, 4)
+__global__ void __launch_bounds__(256, 3)
 tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                TcPrepParams pp, __nv_bfloat16 *__restrict__ qt, __nv_bfloat16 *__restrict__ kt,
                int batch, int heads, int n, int chunk, long long pos0, int rotate,
                int write_q, unsigned *err) {
+    constexpr int kRound = 4;                       // rows per warp per round
     const long long elems = (long long)batch * n * heads * kD;   // of q, k, Qt and Kt
     __shared__ float2 cs[TOK][kD / 2];
     const int t0 = blockIdx.x * TOK;
-    const int per_token = batch * heads * (kD / 8);
-    const int tasks = TOK * per_token;
-    // Up to kPrepBatch 8-element tasks per thread per round; the first
-    // round's loads are issued before the (cos, sin) prologue so its latency
-    // overlaps the memory traffic.
-    constexpr int kPrepBatch = 4;
-    uint4 rq[kPrepBatch] = {}, rk[kPrepBatch];
-    auto task_src = [&](int task, int &u, int &part, int &h, int &b) -> long long {
-        u = task / per_token;
-        const int r = task % per_token;
-        part = r % (kD / 8);
-        const int bhi = r / (kD / 8);
-        h = bhi % heads;
-        b = bhi / heads;
-        return (((long long)b * n + t0 + u) * heads + h) * kD + part * 8;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int bhn = batch * heads;
+    const int rows = TOK * bhn;                      // row r: token t0 + r / bhn, (b, h) = r % bhn
+
+    // first row of this warp, in (u, b, h) form; later rows step by 8
+    int u = warp / bhn, b = (warp % bhn) / heads, h = warp % heads;
+    auto advance = [&](int step) {
+        h += step;
+        while (h >= heads) { h -= heads; ++b; }
+        while (b >= batch) { b -= batch; ++u; }
     };
-    auto load_round = [&](int base) {
+    uint4 rq[kRound] = {}, rk[kRound];
+    int ru[kRound], rb[kRound], rh[kRound];
+    auto load_round = [&](int r0) {
 #pragma unroll
-        for (int x = 0; x < kPrepBatch; ++x) {
-            const int task = base + x * blockDim.x;
-            int u, part, h, b;
-            const long long src = task_src(task, u, part, h, b);
-            if (task < tasks && t0 + u < n) {
-                if (!in_bounds(src + 7, elems, err, kSitePrep)) continue;
-                if (write_q) rq[x] = *reinterpret_cast<const uint4 *>(q + src);
-                rk[x] = *reinterpret_cast<const uint4 *>(k + src);
+        for (int x = 0; x < kRound; ++x) {
+            ru[x] = u; rb[x] = b; rh[x] = h;
+            const int r = r0 + 8 * x;
+            if (r < rows && t0 + u < n) {
+                const long long src = (((long long)b * n + t0 + u) * heads + h) * kD + 8 * lane;
+                if (in_bounds(src + 7, elems, err, kSitePrep)) {
+                    if (write_q) rq[x] = *reinterpret_cast<const uint4 *>(q + src);
+                    rk[x] = *reinterpret_cast<const uint4 *>(k + src);
+                }
             }
+            advance(8);
         }
     };
     grid_dependency_wait();                         // q, k may come from the kernel before
-    load_round(threadIdx.x);
+    load_round(warp);
     for (int c = threadIdx.x; c < TOK * (kD / 2); c += blockDim.x) {
-        const int u = c / (kD / 2), j = c % (kD / 2);
-        cs[u][j] = rotate ? rotation_cs(pos0 + t0 + u, pp.theta[j]) : make_float2(1.f, 0.f);
+        const int uu = c / (kD / 2), j = c % (kD / 2);
+        cs[uu][j] = rotate ? rotation_cs(pos0 + t0 + uu, pp.theta[j]) : make_float2(1.f, 0.f);
     }
     __syncthreads();
-    for (int base = threadIdx.x; base < tasks; base += kPrepBatch * blockDim.x) {
-        if (base != (int)threadIdx.x) load_round(base);
+    for (int r0 = warp; r0 < rows; r0 += 8 * kRound) {
+        if (r0 != warp) load_round(r0);
 #pragma unroll
-        for (int x = 0; x < kPrepBatch; ++x) {
-            const int task = base + x * blockDim.x;
-            int u, part, h, b;
-            task_src(task, u, part, h, b);
-            const int t = t0 + u;
-            if (task < tasks && t < n) {
-                const int i = t % chunk;                    // index inside the chunk
-                const float e = (float)(i + 1) * pp.log2g[h];
-                const float sq = exp2f(e), sk = exp2f(-e);
-                const __nv_bfloat162 *hq = reinterpret_cast<const __nv_bfloat162 *>(&rq[x]);
-                const __nv_bfloat162 *hk = reinterpret_cast<const __nv_bfloat162 *>(&rk[x]);
-                float oq[8], ok[8];
+        for (int x = 0; x < kRound; ++x) {
+            const int r = r0 + 8 * x;
+            const int t = t0 + ru[x];
+            if (r >= rows || t >= n) continue;
+            const int hh = rh[x];
+            const float e = (float)(t % chunk + 1) * pp.log2g[hh];
+            const float sq = exp2f(e), sk = exp2f(-e);
+            const __nv_bfloat162 *hq = reinterpret_cast<const __nv_bfloat162 *>(&rq[x]);
+            const __nv_bfloat162 *hk = reinterpret_cast<const __nv_bfloat162 *>(&rk[x]);
+            float oq[8], ok[8];
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    const float2 r = cs[u][part * 4 + p];
-                    const float cq = r.x * sq, sq2 = r.y * sq, ck = r.x * sk, sk2 = r.y * sk;
-                    const float2 xq = __bfloat1622float2(hq[p]);
-                    const float2 xk = __bfloat1622float2(hk[p]);
-                    oq[2 * p] = xq.x * cq - xq.y * sq2;
-                    oq[2 * p + 1] = xq.x * sq2 + xq.y * cq;
-                    ok[2 * p] = xk.x * ck - xk.y * sk2;
-                    ok[2 * p + 1] = xk.x * sk2 + xk.y * ck;
-                }
-                const long long dst = (((long long)b * heads + h) * n + t) * kD + part * 8;
-                if (!in_bounds(dst + 7, elems, err, kSitePrep)) continue;
-                if (write_q) store8(qt + dst, oq);
-                store8(kt + dst, ok);
+            for (int p = 0; p < 4; ++p) {
+                const float2 cw = cs[ru[x]][lane * 4 + p];
+                const float cq = cw.x * sq, sq2 = cw.y * sq, ck = cw.x * sk, sk2 = cw.y * sk;
+                const float2 xq = __bfloat1622float2(hq[p]);
+                const float2 xk = __bfloat1622float2(hk[p]);
+                oq[2 * p] = xq.x * cq - xq.y * sq2;
+                oq[2 * p + 1] = xq.x * sq2 + xq.y * cq;
+                ok[2 * p] = xk.x * ck - xk.y * sk2;
+                ok[2 * p + 1] = xk.x * sk2 + xk.y * ck;
             }
+            const long long dst = (((long long)rb[x] * heads + hh) * n + t) * kD + 8 * lane;
+            if (!in_bounds(dst + 7, elems, err, kSitePrep)) continue;
+            if (write_q) store8(qt + dst, oq);
+            store8(kt + dst, ok);
         }
     }
 }
@@ -870,6 +870,13 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 constexpr int kPairSlots = 6;
 constexpr uint32_t kPairSlot = 2 * kBox;           // 32 KB
 constexpr int kPairThreads = 448;                  // 14 warps: the 10 of tc_output + 4 fold warps
+// Bits naming the paired pass's waits in the error word (see mbar_wait).
+enum PairWaitSite : unsigned {
+    kWaitRempty = 1u << 16, kWaitRfull = 1u << 17, kWaitOFree = 1u << 18,
+    kWaitOFullMma = 1u << 19, kWaitQReady = 1u << 20, kWaitSRead = 1u << 21,
+    kWaitPFull = 1u << 22, kWaitLfullFold = 1u << 23, kWaitSFull = 1u << 24,
+    kWaitPFree = 1u << 25, kWaitOFullEpi = 1u << 26, kWaitLfullEpi = 1u << 27,
+};
 constexpr int kFoldThreads = 128;
 
 struct TcPairSmem {
@@ -985,7 +992,7 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
             auto acquire = [&]() -> bool {
                 if (it < kPairSlots) return true;
                 return mbar_wait(&rempty[it % kPairSlots], ((it / kPairSlots) - 1) & 1,
-                                 &abort_flag, err);
+                                 &abort_flag, err, kWaitRempty);
             };
             // one operand item: `boxes` boxes of 16 KB (or 8 KB for Kt halves) into
             // this CTA's slot, counted on the leader's rfull (armed for both CTAs)
@@ -1088,7 +1095,7 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
             bool ok = true;
             auto take = [&]() -> bool {
                 const int s = it % kPairSlots;
-                if (!mbar_wait(&rfull[s], (opar >> s) & 1u, &abort_flag, err)) return false;
+                if (!mbar_wait(&rfull[s], (opar >> s) & 1u, &abort_flag, err, kWaitRfull)) return false;
                 opar ^= 1u << s;
                 tc_fence_after();
                 return true;
@@ -1100,17 +1107,17 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                 bool o_written = false;
                 auto claim_o = [&]() -> bool {
                     if (o_written || li == 0) return true;
-                    return mbar_wait(&o_free, (li - 1) & 1, &abort_flag, err);
+                    return mbar_wait(&o_free, (li - 1) & 1, &abort_flag, err, kWaitOFree);
                 };
                 // the previous item's MMAs read Qt from TMEM: they must be
                 // complete before the copy below overwrites it (cp is ordered
                 // before later MMAs of this thread, not after earlier ones)
-                if (li > 0 && !(ok = mbar_wait(&o_full, (li - 1) & 1, &abort_flag, err))) break;
+                if (li > 0 && !(ok = mbar_wait(&o_full, (li - 1) & 1, &abort_flag, err, kWaitOFullMma))) break;
                 tc_fence_after();
                 // Qt of both CTAs -> their TMEM, 16 columns of K per copy: as
                 // loaded, or once the fold warps of both CTAs have folded it
                 if (a.fold_q) {
-                    if (!(ok = mbar_wait(&q_ready, li & 1, &abort_flag, err))) break;
+                    if (!(ok = mbar_wait(&q_ready, li & 1, &abort_flag, err, kWaitQReady))) break;
                     tc_fence_after();
                 } else if (!(ok = take())) {
                     break;
@@ -1131,7 +1138,7 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                 mma_commit_pair(&rempty[sb], 3);
                 // S = Qt Kt^T for key tile t: each CTA holds 64 of its keys
                 auto qk = [&]() -> bool {
-                    if (nqk >= 1 && !mbar_wait(&s_read, (nqk - 1) & 1, &abort_flag, err)) return false;
+                    if (nqk >= 1 && !mbar_wait(&s_read, (nqk - 1) & 1, &abort_flag, err, kWaitSRead)) return false;
                     if (!take()) return false;
                     const uint32_t base = slot_addr(it);
 #pragma unroll
@@ -1167,7 +1174,7 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                     if (!(ok = take() && claim_o())) break;
                     const uint32_t base = slot_addr(it);
                     for (int hx = 0; ok && hx < 2; ++hx) {
-                        if (!mbar_wait(&p_full[hx], npv & 1, &abort_flag, err)) { ok = false; break; }
+                        if (!mbar_wait(&p_full[hx], npv & 1, &abort_flag, err, kWaitPFull)) { ok = false; break; }
                         tc_fence_after();
 #pragma unroll
                         for (int k4 = 0; k4 < 4; ++k4) {
@@ -1218,7 +1225,7 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                 const int qi = it_base;
                 it_base += 2 + 2 * m.nk + m.nsp + 2;
                 const int qs = qi + bx / 2;                    // this column's slot (warp-uniform)
-                if (!warp_wait(&lfull[qs % kPairSlots], (qs / kPairSlots) & 1, &abort_flag, err)) {
+                if (!warp_wait(&lfull[qs % kPairSlots], (qs / kPairSlots) & 1, &abort_flag, err, kWaitLfullFold)) {
                     ok = false;
                     break;
                 }
@@ -1272,7 +1279,7 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
             if (!m.valid) { --li; continue; }
             const int lrow = m.r * kBlk + row;                  // row within the chunk
             for (int t = 0; t < m.nk; ++t, ++ntile) {
-                if (!warp_wait(&s_full, ntile & 1, &abort_flag, err)) { ok = false; break; }
+                if (!warp_wait(&s_full, ntile & 1, &abort_flag, err, kWaitSFull)) { ok = false; break; }
                 tc_fence_after();
                 uint32_t v0[32], v1[32];
                 const uint32_t col = tS + lane_off + 64 * wg;
@@ -1309,7 +1316,7 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                         wv[16 + e] = pack_bf16x2(y0, y1);
                     }
                 }
-                if (ntile >= 1 && !warp_wait(&p_free[wg], (ntile - 1) & 1, &abort_flag, err)) { ok = false; break; }
+                if (ntile >= 1 && !warp_wait(&p_free[wg], (ntile - 1) & 1, &abort_flag, err, kWaitPFree)) { ok = false; break; }
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch)
                     *reinterpret_cast<uint4 *>(prow + ((ch ^ (row & 7)) * 16)) =
@@ -1325,10 +1332,10 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
             it_base = ig + 2;
             uint8_t *ya = slot_ptr(ig), *yb = slot_ptr(ig + 1);
             const bool go =
-                ok && warp_wait(&o_full, li & 1, &abort_flag, err) &&
-                warp_wait(&lfull[ig % kPairSlots], (ig / kPairSlots) & 1, &abort_flag, err) &&
+                ok && warp_wait(&o_full, li & 1, &abort_flag, err, kWaitOFullEpi) &&
+                warp_wait(&lfull[ig % kPairSlots], (ig / kPairSlots) & 1, &abort_flag, err, kWaitLfullEpi) &&
                 warp_wait(&lfull[(ig + 1) % kPairSlots], ((ig + 1) / kPairSlots) & 1, &abort_flag,
-                          err);
+                          err, kWaitLfullEpi);
             float (*red)[kBlk] = reinterpret_cast<float (*)[kBlk]>(pbuf);   // [4][128]
             float mean = 0.f, rstd = 1.f;
             if (go) tc_fence_after();
@@ -1631,9 +1638,8 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
         TcPrepParams pp;
         for (int j = 0; j < kD / 2; ++j) pp.theta[j] = pp_theta[j];
         for (int h = 0; h < kMaxHeads; ++h) pp.log2g[h] = hp.log2g[h];
-        // tokens per CTA: enough (sequence, head) rows for 1024 tasks of 8 elements
-        const int per_token = BH * (kD / 8);
-        const int tok = per_token >= 1024 ? 1 : per_token >= 512 ? 2 : 4;
+        // tokens per CTA: about 64 (token, sequence, head) rows per CTA
+        const int tok = BH >= 64 ? 1 : BH >= 32 ? 2 : BH >= 16 ? 4 : 8;
         KernelTimer timer("tc_prep", stream);
         const __nv_bfloat16 *qq = (const __nv_bfloat16 *)a.q, *kk = (const __nv_bfloat16 *)a.k;
         const int wq = fold_q ? 0 : 1;
@@ -1643,8 +1649,11 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
         else if (tok == 2)
             e = launch_overlapped(tc_prep_kernel<2>, dim3((n + 1) / 2), dim3(256), 0, stream, qq,
                                   kk, pp, qt, kt, B, H, n, fold, a.pos0, a.rotate, wq, err);
-        else
+        else if (tok == 4)
             e = launch_overlapped(tc_prep_kernel<4>, dim3((n + 3) / 4), dim3(256), 0, stream, qq,
+                                  kk, pp, qt, kt, B, H, n, fold, a.pos0, a.rotate, wq, err);
+        else
+            e = launch_overlapped(tc_prep_kernel<8>, dim3((n + 7) / 8), dim3(256), 0, stream, qq,
                                   kk, pp, qt, kt, B, H, n, fold, a.pos0, a.rotate, wq, err);
         count_launch();
         if (e != cudaSuccess) return e;

@@ -64,8 +64,11 @@ __device__ __forceinline__ uint64_t global_ns() {
 // wait_limit_ns() of wall time, or as soon as another thread of the CTA has
 // raised *abort; on giving up it records kDevErrTimeout in the device error
 // word, raises *abort and returns false.
+// `site` (bits 16 and up, optional) names the wait in the error word, so a
+// debug run can tell which wait gave up first.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
-                                          volatile int *abort, unsigned *err) {
+                                          volatile int *abort, unsigned *err,
+                                          unsigned site = 0) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     const uint64_t limit_ns = wait_limit_ns();
@@ -73,7 +76,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
         if (global_ns() - t0 > limit_ns) {
-            if (err) atomicOr(err, (unsigned)kDevErrTimeout);
+            if (err) atomicOr(err, (unsigned)kDevErrTimeout | site);
             *abort = 1;
             return false;
         }
@@ -99,9 +102,9 @@ __device__ __forceinline__ bool mbar_drain(uint64_t *bar, uint32_t parity, unsig
 // Warp-uniform wait: lane 0 polls, the result is broadcast, so every lane
 // of the warp takes the same branch (needed around .sync.aligned tcgen05 ops).
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          unsigned *err) {
+                                          unsigned *err, unsigned site = 0) {
     int ok = 0;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, err) ? 1 : 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, err, site) ? 1 : 0;
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
