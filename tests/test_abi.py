@@ -58,7 +58,7 @@ def test_debug_build_exports_the_test_hooks_and_nothing_else_differs(lib):
     from linear_recurrent_sequence_02_b200.build import build
     path = build(variant="debug")
     hooks = debug_only_functions()
-    assert hooks == ["retnet_test_set_hooks"]
+    assert hooks == ["retnet_test_error_word", "retnet_test_set_hooks"]
     out = os.popen(f"nm -D --defined-only {path}").read()
     exported = sorted(set(re.findall(r"\b(retnet_\w+)\b", out)))
     assert exported == sorted(declared_functions() + hooks)
