@@ -443,10 +443,18 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                  TcOutArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    __shared__ uint64_t rfull[kSlots], rempty[kSlots];
+    // rfull[s]: one phase per operand tile loaded into slot s (the MMA
+    // thread counts them per slot).  The gate/output tile has its own
+    // barrier, g_full, one phase per item, waited in order by the epilogue.
+    // (Were the gate tile counted on its slot's rfull, the MMA thread, which
+    // never waits for it, could reach the next operand tile of that slot
+    // while the gate load is still landing and mistake the slot's phase two
+    // back for the one it needs: the same parity.)
+    __shared__ uint64_t rfull[kSlots], rempty[kSlots], g_full;
     __shared__ uint64_t s_full, s_read, p_full[2], p_free[2], o_full, o_free, drain;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
+    __shared__ uint32_t op_n[kSlots], g_n;            // operand tiles per slot, gate tiles
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     unsigned *err = a.err;
@@ -455,7 +463,13 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     uint8_t *pbuf = smem + TcOutSmem::kP;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kSlots; ++s) { mbar_init(&rfull[s], 1); mbar_init(&rempty[s], 1); }
+        for (int s = 0; s < kSlots; ++s) {
+            mbar_init(&rfull[s], 1);
+            mbar_init(&rempty[s], 1);
+            op_n[s] = 0;
+        }
+        mbar_init(&g_full, 1);
+        g_n = 0;
         mbar_init(&s_full, 1);
         mbar_init(&s_read, kEpiThreads);
         for (int x = 0; x < 2; ++x) {                    // one P half per warpgroup
@@ -493,9 +507,9 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 if (it < kSlots) return true;
                 return mbar_wait(&rempty[it % kSlots], ((it / kSlots) - 1) & 1, &abort_flag, err);
             };
-            auto issue = [&](const CUtensorMap *map, int rank, int c1, int c2, int c3) {
+            auto issue = [&](const CUtensorMap *map, int rank, int c1, int c2, int c3,
+                             uint64_t *bar) {
                 uint8_t *d = slot_ptr(it);
-                uint64_t *bar = &rfull[it % kSlots];
                 mbar_expect_tx(bar, kSlot);
                 for (int x = 0; x < 4; ++x) {
                     if (rank == 2) tma_load_2d(d + x * kBox, map, bar, 64 * x, c1);
@@ -515,31 +529,37 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     ok = false;
                     break;
                 }
+                // an operand tile: counted on its slot's rfull
+                auto op = [&](const CUtensorMap *map, int rank, int c1, int c2, int c3) {
+                    *(volatile uint32_t *)&op_n[it % kSlots] += 1;
+                    issue(map, rank, c1, c2, c3, &rfull[it % kSlots]);
+                };
                 if (!(ok = acquire())) break;
-                issue(&tm_q, 3, m.t0row, m.bh, 0);
+                op(&tm_q, 3, m.t0row, m.bh, 0);
                 if (!(ok = acquire())) break;
-                issue(&tm_k, 3, m.c0, m.bh, 0);
+                op(&tm_k, 3, m.c0, m.bh, 0);
                 for (int t = 0; ok && t < m.nk; ++t) {
                     if (t + 1 < m.nk) {
                         if (!(ok = acquire())) break;
-                        issue(&tm_k, 3, m.c0 + (t + 1) * kKeyTile, m.bh, 0);
+                        op(&tm_k, 3, m.c0 + (t + 1) * kKeyTile, m.bh, 0);
                     }
                     if (t < m.nsp) {
                         if (!(ok = acquire())) break;
-                        issue(&tm_s, 2, srow + kBlk * t, 0, 0);
+                        op(&tm_s, 2, srow + kBlk * t, 0, 0);
                     }
                     if (!(ok = acquire())) break;
-                    issue(&tm_v, 4, m.h, m.c0 + t * kKeyTile, m.b);
+                    op(&tm_v, 4, m.h, m.c0 + t * kKeyTile, m.b);
                 }
                 for (int p = m.nk; ok && p < m.nsp; ++p) {
                     if (!(ok = acquire())) break;
-                    issue(&tm_s, 2, srow + kBlk * p, 0, 0);
+                    op(&tm_s, 2, srow + kBlk * p, 0, 0);
                 }
                 if (ok && (ok = acquire())) {                // the gate/output tile
+                    *(volatile uint32_t *)&g_n += 1;
                     if (a.has_gate) {
-                        issue(&tm_g, 4, m.h, m.t0row, m.b);
+                        issue(&tm_g, 4, m.h, m.t0row, m.b, &g_full);
                     } else {
-                        mbar_arrive(&rfull[it % kSlots]);     // reserved for the output rows
+                        mbar_arrive(&g_full);                 // reserved for the output rows
                         ++it;
                     }
                 }
@@ -552,9 +572,12 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const uint32_t sbase = smem_u32(smem);
             const uint32_t sP = sbase + TcOutSmem::kP;
             int it = 0, nqk = 0, npv = 0, li = 0;
+            uint32_t opar = 0;                         // per slot: parity of its next rfull phase
             bool ok = true;
             auto take = [&]() -> bool {
-                if (!mbar_wait(&rfull[it % kSlots], (it / kSlots) & 1, &abort_flag, err)) return false;
+                const int s = it % kSlots;
+                if (!mbar_wait(&rfull[s], (opar >> s) & 1u, &abort_flag, err)) return false;
+                opar ^= 1u << s;
                 tc_fence_after();
                 return true;
             };
@@ -714,7 +737,7 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             it_base = ig + 1;
             uint8_t *ybuf = slot_ptr(ig);
             const bool go = ok && warp_wait(&o_full, li & 1, &abort_flag, err) &&
-                            warp_wait(&rfull[ig % kSlots], (ig / kSlots) & 1, &abort_flag, err);
+                            warp_wait(&g_full, li & 1, &abort_flag, err);
             // the P tile is idle between items: it holds the partial row sums
             float (*red)[kBlk] = reinterpret_cast<float (*)[kBlk]>(pbuf);   // [4][128]
             float mean = 0.f, rstd = 1.f;
@@ -820,9 +843,11 @@ tc_output_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // (bounded) for what this CTA still has in flight: the TMA loads (at most
     // the last kSlots issued) before shared memory goes away, the MMAs before
     // tensor memory is freed.
-    if (abort_flag && warp == 0 && lane == 0)
-        for (int j = max(0, pit - kSlots); j < pit; ++j)
-            mbar_drain(&rfull[j % kSlots], (j / kSlots) & 1, err);
+    if (abort_flag && warp == 0 && lane == 0) {
+        for (int j = 0; j < kSlots; ++j)
+            if (op_n[j] > 0) mbar_drain(&rfull[j], (op_n[j] - 1) & 1, err);
+        if (g_n > 0) mbar_drain(&g_full, (g_n - 1) & 1, err);
+    }
     if (warp == 1) {
         if (abort_flag && lane == 0) {
             mma_commit(&drain);
@@ -923,6 +948,10 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     __shared__ uint64_t rfull[kPairSlots], rempty[kPairSlots], lfull[kPairSlots];
     __shared__ uint64_t s_full, s_read, p_full[2], p_free[2], o_full, o_free, drain, q_ready;
+    // raw q halves (fold mode): one phase per item, waited in sequence by the
+    // fold warps (a slot's lfull would let them alias a phase two ahead)
+    __shared__ uint64_t qfull[2];
+    __shared__ uint32_t q_n[2];                    // raw-q halves this CTA issued
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
     __shared__ uint32_t op_n[kPairSlots];          // operand items this CTA issued per slot
@@ -958,6 +987,9 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_init(&o_free, 2 * kEpiThreads / 32);
         mbar_init(&drain, 1);
         mbar_init(&q_ready, 2 * kFoldThreads / 32);
+        mbar_init(&qfull[0], 1);
+        mbar_init(&qfull[1], 1);
+        q_n[0] = q_n[1] = 0;
         abort_flag = 0;
         for (int s = 0; s < kPairSlots; ++s) op_n[s] = lf_n[s] = 0;
         fence_barrier_init();
@@ -1036,11 +1068,13 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                         // raw q rows of this CTA, folded in place by the fold
                         // warps (counted on lfull; rfull only kept in order)
                         uint8_t *d = slot_ptr(it);
-                        uint64_t *lb = &lfull[it % kPairSlots];
                         *(volatile uint32_t *)&lf_n[it % kPairSlots] += 1;
-                        mbar_expect_tx(lb, kPairSlot);
+                        mbar_arrive(&lfull[it % kPairSlots]);      // keeps lfull in ring order
+                        uint64_t *qb = &qfull[half];
+                        *(volatile uint32_t *)&q_n[half] += 1;
+                        mbar_expect_tx(qb, kPairSlot);
                         for (int x = 0; x < 2; ++x)
-                            tma_load_4d(d + x * kBox, &tm_qraw, lb, 128 * half + 64 * x, m.h,
+                            tma_load_4d(d + x * kBox, &tm_qraw, qb, 128 * half + 64 * x, m.h,
                                         m.t0row, m.b);
                         ++it;
                     } else {
@@ -1217,15 +1251,15 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
             const int bx = j / 32;                             // 64-column box
             const uint32_t in_row = (uint32_t)((j % 4) * 4);
             const int ch = (j % 32) / 4;                       // 16-byte chunk in the row
-            int it_base = 0;
+            int it_base = 0, fi = 0;
             bool ok = true;
-            for (int w = cluster; ok && w < a.items; w += nclusters) {
+            for (int w = cluster; ok && w < a.items; w += nclusters, ++fi) {
                 const TcPairItem m = tc_pair_item(a, w, rank);
-                if (!m.valid) continue;
+                if (!m.valid) { --fi; continue; }
                 const int qi = it_base;
                 it_base += 2 + 2 * m.nk + m.nsp + 2;
                 const int qs = qi + bx / 2;                    // this column's slot (warp-uniform)
-                if (!warp_wait(&lfull[qs % kPairSlots], (qs / kPairSlots) & 1, &abort_flag, err, kWaitLfullFold)) {
+                if (!warp_wait(&qfull[bx / 2], fi & 1, &abort_flag, err, kWaitLfullFold)) {
                     ok = false;
                     break;
                 }
@@ -1442,9 +1476,12 @@ tc_output_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     // (they count on its barriers) and its MMAs; each CTA its own gate loads.
     const bool aborted = abort_flag != 0;
     if (aborted && warp == 0 && lane == 0) {
-        // each CTA: the latest armed lfull phase of every slot (gate tiles, raw q)
+        // each CTA: the latest armed lfull phase of every slot (gate tiles), and
+        // the raw q halves
         for (int j = 0; j < kPairSlots; ++j)
             if (lf_n[j] > 0) mbar_drain(&lfull[j], (lf_n[j] - 1) & 1, err);
+        for (int h2 = 0; h2 < 2; ++h2)
+            if (q_n[h2] > 0) mbar_drain(&qfull[h2], (q_n[h2] - 1) & 1, err);
         if (leader) {
             // Each producer runs at most kPairSlots ring items past the MMAs,
             // so every slot has at most one operand phase still open, and the
