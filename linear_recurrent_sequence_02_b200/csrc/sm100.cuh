@@ -315,10 +315,12 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
     return r;
 }
 // Arrives on an mbarrier given by its shared::cluster address (this CTA's
-// or the peer's), releasing this thread's earlier writes at cluster scope.
+// or the peer's).  The default (CTA-scope release) semantics: every signal
+// sent this way guards data that stays in the arriving CTA (its P tile, its
+// reads of its own tensor memory), read later by its own SM's tensor core,
+// so no cluster-wide fence is needed on the way out.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-                 : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 // Counts `bytes` of expected transactions as done on a barrier of this CTA
 // (the abort path settles the share of a load the peer never issued).
