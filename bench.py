@@ -95,28 +95,56 @@ def workload_config(w: wl.Workload, chunk: int, form: str = "chunkwise") -> dict
     }
 
 
-# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
-# one ncu capture of the layer200m workload, keyed by a hash of the kernel's
-# source file at capture time; reported only while the source is unchanged.
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of a
+# kernel on a workload, from one ncu capture.  Each figure is kept with the
+# SHA-256 of the kernel's source at capture time: its section of the .cu file
+# (from its banner line to the next) and the device headers it includes.
+# The figure is reported only while that source is unchanged.
 NCU_TRAFFIC = {
-    "tc_output": {"source": "chunkwise_tc.cu",
-                  "sha256": "cdc9c928156913a3a79892a46604b1b96884fb9158abaf38f1e3692f25bd6743",
-                  "bytes": 160.33e6},
+    ("tc_output", "long7b"): {
+        "source": "chunkwise_tc.cu", "section": "output pass",
+        "headers": ["sm100.cuh", "common.cuh"],
+        "sha256": "cf91a0d29ac40dd6cbee331e2e3db328b08fd927ce53106ddff7716dc18fba0f",
+        "bytes": 277.98e6,
+    },
 }
+SECTION_BANNER = "// " + "-" * 66 + " "
+
+
+def kernel_source_sha(source: str, section: str, headers) -> str | None:
+    """SHA-256 over one banner-delimited section of a .cu file and the headers."""
+    import hashlib
+    csrc = os.path.join(ROOT, "linear_recurrent_sequence_02_b200", "csrc")
+    try:
+        with open(os.path.join(csrc, source), encoding="utf-8") as f:
+            lines = f.read().split("\n")
+        start = lines.index(SECTION_BANNER + section)
+        end = next((i for i in range(start + 1, len(lines))
+                    if lines[i].startswith(SECTION_BANNER)), len(lines))
+        h = hashlib.sha256("\n".join(lines[start:end]).encode())
+        for name in headers:
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
+    except (OSError, ValueError):
+        return None
+    return h.hexdigest()
 
 
 def measured_traffic(kernel: str, workload: str):
-    import hashlib
-    rec = NCU_TRAFFIC.get(kernel)
-    if not rec or workload != "layer200m" or not rec["sha256"]:
+    rec = NCU_TRAFFIC.get((kernel, workload))
+    if not rec or not rec["sha256"] or rec["bytes"] is None:
         return None
-    path = os.path.join(ROOT, "linear_recurrent_sequence_02_b200", "csrc", rec["source"])
-    try:
-        with open(path, "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()
-    except OSError:
-        return None
+    sha = kernel_source_sha(rec["source"], rec["section"], rec["headers"])
     return rec["bytes"] if sha == rec["sha256"] else None
+
+
+def output_kernel_bytes(batch: int, heads: int, n: int, d: int, chunk: int, gate: bool) -> int:
+    """Algorithmic HBM bytes of one output-pass launch: Qt, Kt, V read and O
+    written once (bf16), G read once when gated, and S_prev (bf16 d x d) read
+    once for every chunk after the first."""
+    th = batch * heads * n
+    nchunks = (n + chunk - 1) // chunk
+    return th * 2 * d * (3 + (2 if gate else 1)) + batch * heads * (nchunks - 1) * d * d * 2
 
 
 def algorithmic_flops_per_token_head(d: int, chunk: int) -> int:
@@ -574,16 +602,31 @@ def measure_prefill(args, w, chunk, rank, world, dev, full=True):
             flops = (parallel_flops_per_token_head(d, n) if par else
                      output_kernel_flops_per_token_head(d, chunk)) * th
             achieved = flops / avg_s / 1e12
-            bound = "tensor" if dom.startswith("tc") else "alu"
-            if bound == "tensor":
-                peak = peaks["bf16_tflops"]
+            if dom.startswith("tc"):
+                # the binding roof of min(tensor peak, HBM bandwidth x intensity):
+                # the larger of the two floors, flops / peak and bytes / bandwidth
+                nbytes = None if par else output_kernel_bytes(B, H, n, d, chunk, bool(w.hidden))
+                tensor = {"achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                          "frac": achieved / peaks["bf16_tflops"], "work_per_launch": flops}
+                hbm = None
+                if nbytes:
+                    gbs = nbytes / avg_s / 1e9
+                    hbm = {"achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                           "frac": gbs / peaks["hbm_gbs"], "work_per_launch": nbytes}
+                binding = hbm if hbm and hbm["frac"] > tensor["frac"] else tensor
+                roof = {"kernel": dom, "bound": "hbm" if binding is hbm else "tensor",
+                        "achieved": binding["achieved"], "peak": binding["peak"],
+                        "unit": binding["unit"], "frac": binding["frac"],
+                        "traffic": None if par else measured_traffic(dom, w.name),
+                        "peak_source": peak_src, "work_per_launch": binding["work_per_launch"],
+                        "avg_us": avg_s * 1e6, "tensor": tensor, "hbm": hbm,
+                        "intensity_flop_per_byte": flops / nbytes if nbytes else None}
             else:   # float32 FFMA: 148 SMs x 128 lanes x 2 flop x max SM clock
                 peak = 148 * 128 * 2 * (peaks.get("sm_max_mhz", 1965.0) * 1e6) / 1e12
-            roof = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak,
-                    "unit": "TFLOP/s", "frac": achieved / peak,
-                    "traffic": None if par else measured_traffic(dom, w.name),
-                    "peak_source": peak_src, "work_per_launch": flops,
-                    "avg_us": avg_s * 1e6}
+                roof = {"kernel": dom, "bound": "alu", "achieved": achieved, "peak": peak,
+                        "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                        "peak_source": peak_src, "work_per_launch": flops,
+                        "avg_us": avg_s * 1e6}
         elif dom in ("tc_state", "simt_state"):
             flops = state_kernel_flops_per_token_head(d) * th
             achieved = flops / avg_s / 1e12

@@ -116,12 +116,12 @@ RETNET_API unsigned long long retnet_kernel_launch_count(void);
 RETNET_API retnet_status retnet_set_launch_overlap(int enable);
 
 /* How the tensor-core prefill's output pass runs (process-wide).
- *   1 (default): chunks of 256 tokens or more run on pairs of CTAs whose
- *     tensor cores act as one (each CTA loads half of every key, value and
- *     state tile), and the pair rotates and decay-scales q itself, so the
- *     prep pass writes only the folded keys;
- *   2: CTA pairs as in 1, with q folded by the prep pass;
- *   0: every CTA works alone.
+ *   0 (default): every CTA works alone;
+ *   1: chunks of 256 tokens or more run on pairs of CTAs whose tensor
+ *     cores act as one (each CTA loads half of every key, value and state
+ *     tile), and the pair rotates and decay-scales q itself, so the prep
+ *     pass writes only the folded keys;
+ *   2: CTA pairs as in 1, with q folded by the prep pass.
  * Chunk 128 (and the shorter chunks computed as 128) always runs on single
  * CTAs.  Results agree to rounding; only the speed changes.
  * mode: 0, 1 or 2, else INVALID_ARG. */

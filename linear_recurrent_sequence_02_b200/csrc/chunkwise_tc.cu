@@ -50,92 +50,92 @@ struct TcHeadParams {
 
 // ------------------------------------------------------------------ prep
 // Rotation and decay fold of k (and of q when write_q) into Kt (Qt), laid
-// out [b*H + h][t][256].  One CTA per TOK consecutive tokens: their
-// TOK x 128 (cos, sin) pairs are formed once (rotation_cs of
-// (pos0 + t) * theta_j) in shared memory.  Each warp then takes whole
-// (token, sequence, head) rows of 256 elements, one 16-byte part per lane
-// (fully coalesced), four rows per round with all their loads issued before
-// any arithmetic; the row's (token, sequence, head) indices advance by
-// additions, so no per-element division is left.  TOK is chosen so that a
-// CTA has about 64 rows.
+// out [b*H + h][t][256].  One warp per token t (grid-stride): every row of
+// that token, all B*H (sequence, head) pairs, rotates by the same angles, so
+// the lane's four (cos, sin) pairs, rotation pairs j = 4 lane .. 4 lane + 3
+// of (pos0 + t) * theta_j, are formed once in registers and serve all of
+// them.  A row of 256 elements is one 16-byte part per lane (coalesced);
+// rows go four at a time with all their loads issued before any arithmetic,
+// the first four before the angles are formed.  The fold exponent
+// (t mod fold) + 1 is also per token; only the head's log2(gamma) varies by row.
 struct TcPrepParams {
     double theta[kD / 2];          // 10000^(-2j/256), formed on the host
     float log2g[kMaxHeads];        // log2(gamma_h)
 };
 
-template <int TOK>
-__global__ void __launch_bounds__(256, 3)
+__global__ void __launch_bounds__(256)
 tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                TcPrepParams pp, __nv_bfloat16 *__restrict__ qt, __nv_bfloat16 *__restrict__ kt,
-               int batch, int heads, int n, int chunk, long long pos0, int rotate,
+               int batch, int heads, int n, int fold, long long pos0, int rotate,
                int write_q, unsigned *err) {
-    constexpr int kRound = 4;                       // rows per warp per round
+    constexpr int kRound = 4;                       // rows per round
     const long long elems = (long long)batch * n * heads * kD;   // of q, k, Qt and Kt
-    __shared__ float2 cs[TOK][kD / 2];
-    const int t0 = blockIdx.x * TOK;
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int bhn = batch * heads;
-    const int rows = TOK * bhn;                      // row r: token t0 + r / bhn, (b, h) = r % bhn
-
-    // first row of this warp, in (u, b, h) form; later rows step by 8
-    int u = warp / bhn, b = (warp % bhn) / heads, h = warp % heads;
-    auto advance = [&](int step) {
-        h += step;
-        while (h >= heads) { h -= heads; ++b; }
-        while (b >= batch) { b -= batch; ++u; }
-    };
-    uint4 rq[kRound] = {}, rk[kRound];
-    int ru[kRound], rb[kRound], rh[kRound];
-    auto load_round = [&](int r0) {
+    const int lane = threadIdx.x % 32;
+    const int warp0 = (int)((blockIdx.x * (long long)blockDim.x + threadIdx.x) / 32);
+    const int nwarps = (int)(gridDim.x * (long long)blockDim.x / 32);
+    const int rows = batch * heads;                 // row r = b * heads + h
+    const long long row_in = (long long)heads * kD;            // q/k: one token of all heads
+    const long long seq_in = (long long)n * row_in;            // q/k: one sequence
+    const long long row_out = (long long)n * kD;               // Qt/Kt: one (sequence, head)
+    double th[4];
 #pragma unroll
-        for (int x = 0; x < kRound; ++x) {
-            ru[x] = u; rb[x] = b; rh[x] = h;
-            const int r = r0 + 8 * x;
-            if (r < rows && t0 + u < n) {
-                const long long src = (((long long)b * n + t0 + u) * heads + h) * kD + 8 * lane;
-                if (in_bounds(src + 7, elems, err, kSitePrep)) {
-                    if (write_q) rq[x] = *reinterpret_cast<const uint4 *>(q + src);
-                    rk[x] = *reinterpret_cast<const uint4 *>(k + src);
-                }
-            }
-            advance(8);
-        }
-    };
+    for (int p = 0; p < 4; ++p) th[p] = pp.theta[4 * lane + p];
     grid_dependency_wait();                         // q, k may come from the kernel before
-    load_round(warp);
-    for (int c = threadIdx.x; c < TOK * (kD / 2); c += blockDim.x) {
-        const int uu = c / (kD / 2), j = c % (kD / 2);
-        cs[uu][j] = rotate ? rotation_cs(pos0 + t0 + uu, pp.theta[j]) : make_float2(1.f, 0.f);
-    }
-    __syncthreads();
-    for (int r0 = warp; r0 < rows; r0 += 8 * kRound) {
-        if (r0 != warp) load_round(r0);
+
+    uint4 rq[kRound] = {}, rk[kRound] = {};
+    int rb[kRound], rh[kRound];
+    for (int t = warp0; t < n; t += nwarps) {
+        int b = 0, h = 0;                           // (sequence, head) of the round's first row
+        auto load_round = [&](int r0) {
+            int bb = b, hh = h;
 #pragma unroll
-        for (int x = 0; x < kRound; ++x) {
-            const int r = r0 + 8 * x;
-            const int t = t0 + ru[x];
-            if (r >= rows || t >= n) continue;
-            const int hh = rh[x];
-            const float e = (float)(t % chunk + 1) * pp.log2g[hh];
-            const float sq = exp2f(e), sk = exp2f(-e);
-            const __nv_bfloat162 *hq = reinterpret_cast<const __nv_bfloat162 *>(&rq[x]);
-            const __nv_bfloat162 *hk = reinterpret_cast<const __nv_bfloat162 *>(&rk[x]);
-            float oq[8], ok[8];
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                const float2 cw = cs[ru[x]][lane * 4 + p];
-                const float cq = cw.x * sq, sq2 = cw.y * sq, ck = cw.x * sk, sk2 = cw.y * sk;
-                const float2 xq = __bfloat1622float2(hq[p]);
-                const float2 xk = __bfloat1622float2(hk[p]);
-                oq[2 * p] = xq.x * cq - xq.y * sq2;
-                oq[2 * p + 1] = xq.x * sq2 + xq.y * cq;
-                ok[2 * p] = xk.x * ck - xk.y * sk2;
-                ok[2 * p + 1] = xk.x * sk2 + xk.y * ck;
+            for (int x = 0; x < kRound; ++x) {
+                rb[x] = bb; rh[x] = hh;
+                if (r0 + x < rows) {
+                    const long long src = bb * seq_in + t * row_in + hh * kD + 8 * lane;
+                    if (in_bounds(src + 7, elems, err, kSitePrep)) {
+                        if (write_q) rq[x] = *reinterpret_cast<const uint4 *>(q + src);
+                        rk[x] = *reinterpret_cast<const uint4 *>(k + src);
+                    }
+                }
+                if (++hh == heads) { hh = 0; ++bb; }
             }
-            const long long dst = (((long long)rb[x] * heads + hh) * n + t) * kD + 8 * lane;
-            if (!in_bounds(dst + 7, elems, err, kSitePrep)) continue;
-            if (write_q) store8(qt + dst, oq);
-            store8(kt + dst, ok);
+            b = bb; h = hh;
+        };
+        load_round(0);
+        float2 cs[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+            cs[p] = rotate ? rotation_cs(pos0 + t, th[p]) : make_float2(1.f, 0.f);
+        const float ef = (float)(t % fold + 1);
+        const long long dst0 = (long long)t * kD + 8 * lane;
+        for (int r0 = 0; r0 < rows; r0 += kRound) {
+            if (r0 > 0) load_round(r0);
+#pragma unroll
+            for (int x = 0; x < kRound; ++x) {
+                const int r = r0 + x;
+                if (r >= rows) continue;
+                const float e = ef * pp.log2g[rh[x]];
+                const float sq = exp2f(e), sk = exp2f(-e);
+                const __nv_bfloat162 *hq = reinterpret_cast<const __nv_bfloat162 *>(&rq[x]);
+                const __nv_bfloat162 *hk = reinterpret_cast<const __nv_bfloat162 *>(&rk[x]);
+                float oq[8], ok[8];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const float cq = cs[p].x * sq, sq2 = cs[p].y * sq;
+                    const float ck = cs[p].x * sk, sk2 = cs[p].y * sk;
+                    const float2 xq = __bfloat1622float2(hq[p]);
+                    const float2 xk = __bfloat1622float2(hk[p]);
+                    oq[2 * p] = xq.x * cq - xq.y * sq2;
+                    oq[2 * p + 1] = xq.x * sq2 + xq.y * cq;
+                    ok[2 * p] = xk.x * ck - xk.y * sk2;
+                    ok[2 * p + 1] = xk.x * sk2 + xk.y * ck;
+                }
+                const long long dst = r * row_out + dst0;
+                if (!in_bounds(dst + 7, elems, err, kSitePrep)) continue;
+                if (write_q) store8(qt + dst, oq);
+                store8(kt + dst, ok);
+            }
         }
     }
 }
@@ -1675,23 +1675,16 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
         TcPrepParams pp;
         for (int j = 0; j < kD / 2; ++j) pp.theta[j] = pp_theta[j];
         for (int h = 0; h < kMaxHeads; ++h) pp.log2g[h] = hp.log2g[h];
-        // tokens per CTA: about 64 (token, sequence, head) rows per CTA
-        const int tok = BH >= 64 ? 1 : BH >= 32 ? 2 : BH >= 16 ? 4 : 8;
+        // one warp per token, eight per CTA, at most eight CTAs per SM
+        int dev = 0, sms = 148;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int blocks = std::max(1, std::min((n + 7) / 8, 8 * sms));
         KernelTimer timer("tc_prep", stream);
-        const __nv_bfloat16 *qq = (const __nv_bfloat16 *)a.q, *kk = (const __nv_bfloat16 *)a.k;
         const int wq = fold_q ? 0 : 1;
-        if (tok == 1)
-            e = launch_overlapped(tc_prep_kernel<1>, dim3(n), dim3(256), 0, stream, qq, kk, pp,
-                                  qt, kt, B, H, n, fold, a.pos0, a.rotate, wq, err);
-        else if (tok == 2)
-            e = launch_overlapped(tc_prep_kernel<2>, dim3((n + 1) / 2), dim3(256), 0, stream, qq,
-                                  kk, pp, qt, kt, B, H, n, fold, a.pos0, a.rotate, wq, err);
-        else if (tok == 4)
-            e = launch_overlapped(tc_prep_kernel<4>, dim3((n + 3) / 4), dim3(256), 0, stream, qq,
-                                  kk, pp, qt, kt, B, H, n, fold, a.pos0, a.rotate, wq, err);
-        else
-            e = launch_overlapped(tc_prep_kernel<8>, dim3((n + 7) / 8), dim3(256), 0, stream, qq,
-                                  kk, pp, qt, kt, B, H, n, fold, a.pos0, a.rotate, wq, err);
+        e = launch_overlapped(tc_prep_kernel, dim3(blocks), dim3(256), 0, stream,
+                              (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, pp, qt, kt,
+                              B, H, n, fold, a.pos0, a.rotate, wq, err);
         count_launch();
         if (e != cudaSuccess) return e;
     }

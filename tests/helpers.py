@@ -42,13 +42,14 @@ def record(value: float, what: str = "") -> float:
     return value
 
 
-def slice_rel_err(got, ref, head_axis: int = 2) -> float:
+def slice_rel_err(got, ref, head_axis: int = 2, keep: bool = True) -> float:
     """Norm-wise relative error, worst over (batch, head) slices.
 
     For each (batch, head) slice: max|got - ref| / max|ref|.  This is the
     reading of "max relative error" used for parity: an elementwise ratio is
     meaningless at the many near-zero entries of a retention output.
     Arrays are [B, n, H, d] (head_axis=2) or [B, H, ...] (head_axis=1).
+    keep=False leaves the value out of the run's report of achieved errors.
     """
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
@@ -60,6 +61,5 @@ def slice_rel_err(got, ref, head_axis: int = 2) -> float:
     num = np.abs(g - r).max(axis=-1)
     den = np.abs(r).max(axis=-1)
     den = np.where(den == 0, 1.0, den)
-    if not np.all(np.isfinite(g)):
-        return record(float("inf"), "slice")
-    return record(float((num / den).max()), "slice")
+    err = float("inf") if not np.all(np.isfinite(g)) else float((num / den).max())
+    return record(err, "slice") if keep else err

@@ -245,13 +245,13 @@ def test_groupnorm_output_moments():
 # ------------------------------------------------------- parity measure
 def test_slice_rel_err_measure():
     ref = _rand(2, 5, 3, 4)
-    assert slice_rel_err(ref, ref) == 0.0
+    assert slice_rel_err(ref, ref, keep=False) == 0.0
     bad = ref.copy()
     bad[1, 2, 2, 3] += 0.5 * np.abs(ref[1, :, 2, :]).max()
-    assert abs(slice_rel_err(bad, ref) - 0.5) < 1e-12
+    assert abs(slice_rel_err(bad, ref, keep=False) - 0.5) < 1e-12
     nan = ref.copy()
     nan[0, 0, 0, 0] = np.nan
-    assert slice_rel_err(nan, ref) == float("inf")
+    assert slice_rel_err(nan, ref, keep=False) == float("inf")
 
 
 # ---------------------------------------------------------------- gradients

@@ -9,7 +9,9 @@ one it wants.  This model replays the roles' barrier operations in the
 order the kernels issue them (ring items per work item: the query tile, the
 key tiles, the state halves, the value tiles, the gate/output tile), under
 random interleavings and random arrival times of the loads, and checks that
-every run finishes without a deadlock or an over-arrival.
+every run finishes without a deadlock or an over-arrival.  The single CTA's
+MMA waits also state the number of completions they need, so a wait that
+passes on an older phase of the same parity is reported when it happens.
 
 It also keeps, as `aliasing=True`, the protocol the kernels had before: the
 gate tile counted on its slot's full barrier (single CTA) and raw q counted
@@ -52,9 +54,14 @@ class OverArrival(Exception):
     pass
 
 
+class StaleWait(Exception):
+    """A wait given the number of completions it needs passed before them."""
+
+
 def simulate(roles, inflight, rng, limit=400000):
-    """Run generator roles that yield (barrier, parity) waits; None on success,
-    else a description of the deadlock."""
+    """Run generator roles that yield (barrier, parity) waits, or (barrier,
+    parity, completions needed) to have a stale pass reported; None on
+    success, else a description of the deadlock."""
     waiting = [None] * len(roles)
     alive = list(range(len(roles)))
     for _ in range(limit):
@@ -70,9 +77,11 @@ def simulate(roles, inflight, rng, limit=400000):
         rng.shuffle(order)
         for i in order:
             if waiting[i] is not None:
-                bar, par = waiting[i]
+                bar, par = waiting[i][0], waiting[i][1]
                 if not bar.passed(par):
                     continue
+                if len(waiting[i]) > 2 and bar.phase < waiting[i][2]:
+                    raise StaleWait(bar.name)   # passed on an older phase of the same parity
                 waiting[i] = None
             try:
                 waiting[i] = next(roles[i])
@@ -136,14 +145,16 @@ def single_cta(items, gate, aliasing, rng, slots=3):
     def mma():
         it = nqk = npv = 0
         par = [0] * slots
+        ops = [0] * slots                       # operand phases of each slot taken so far
 
         def take():
             s = it % slots
-            if aliasing:
-                yield B[f"full{s}"], (it // slots) & 1
-            else:
-                yield B[f"full{s}"], par[s]
+            if aliasing:                        # every ring item is a phase of its slot
+                yield B[f"full{s}"], (it // slots) & 1, it // slots + 1
+            else:                               # only the slot's operand tiles are
+                yield B[f"full{s}"], par[s], ops[s] + 1
                 par[s] ^= 1
+                ops[s] += 1
 
         for li, (nk, nsp) in enumerate(items):
             written = [False]
@@ -401,6 +412,8 @@ def failures(run, seeds, **kw):
             result = run(items, rng=rng, **kw)
         except OverArrival:
             result = "over-arrival"
+        except StaleWait:
+            result = "stale wait"
         bad += result is not None
     return bad
 
@@ -422,3 +435,4 @@ def test_cta_pair_protocol_has_no_race(fold, gate):
 
 def test_cta_pair_model_finds_the_fold_aliasing_race():
     assert failures(cta_pair, 150, gate=True, fold=True, aliasing=True) > 0
+
