@@ -104,7 +104,7 @@ NCU_TRAFFIC = {
     ("tc_output", "long7b"): {
         "source": "chunkwise_tc.cu", "section": "output pass",
         "headers": ["sm100.cuh", "common.cuh"],
-        "sha256": "cf91a0d29ac40dd6cbee331e2e3db328b08fd927ce53106ddff7716dc18fba0f",
+        "sha256": "97a24651b782322a9322bb14fc605869870f25c184670e922ec1b7406a49dfeb",
         "bytes": 277.98e6,
     },
 }

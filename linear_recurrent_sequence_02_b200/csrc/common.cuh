@@ -141,7 +141,7 @@ __device__ __forceinline__ void grid_dependency_wait() {
 // (retnet_set_launch_overlap; on by default).
 bool launch_overlap_enabled();
 // Host: how the tensor-core output pass runs (retnet_set_output_pairing):
-// 0 single CTAs, 1 CTA pairs folding q themselves (default), 2 CTA pairs
+// 0 single CTAs (default), 1 CTA pairs folding q themselves, 2 CTA pairs
 // reading the prep pass's folded q.
 int output_pairing_mode();
 
