@@ -21,8 +21,8 @@ default line adds two measurements of their own (skip with --no-legs):
 "decode_legs", the decode configuration (H=16, d=256, states seeded by an
 8192-token prefill) at batch 32 and 128, where the state (269 MB, 1.08 GB)
 is beyond L2, each with its HBM roofline; and "secondary", the 200M-layer
-step (B=8, H=4, n=2048, chunk 512, gate) measured the same way as the main
-workload.
+step (B=8, H=4, n=2048, gate) at chunk 512 and at chunk 64, measured the
+same way as the main workload.
 
 The K timed steps are captured once as a CUDA graph and replayed (after one
 warm-up replay), so the GPU runs them back to back without host launch
@@ -87,12 +87,17 @@ def workload_config(w: wl.Workload, chunk: int, form: str = "chunkwise") -> dict
     else:
         what = f"chunk {chunk}" + (" + GroupNorm/swish gate" if w.hidden else "") + \
             " + 1 decode step"
-    return {
+    cfg = {
         "workload": f"{w.name}: B={w.batch} H={w.heads} n={w.seqlen} d={w.d} {w.dtype} " + what,
         "batch": w.batch, "heads": w.heads, "seqlen": w.seqlen, "dk": w.d, "dv": w.d,
         "chunk": chunk if form == "chunkwise" else None, "form": form, "gate": bool(w.hidden),
         "l2": "3 rotating input sets, each beyond 1/3 of the 126 MB L2",
     }
+    if form == "chunkwise" and chunk < 128 and w.dtype == "bf16" and w.d == 256:
+        cfg["computed_as"] = ("128-token chunks on the tensor cores: the chunkwise form's "
+                              "outputs do not depend on the chunk length, so only the "
+                              "rounding order differs from chunk " + str(chunk))
+    return cfg
 
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of a
@@ -373,9 +378,13 @@ def run_ours(args, w, chunk):
         line["decode_legs"] = {f"batch{b}": measure_decode(args, dw, b, 1, dev, world)
                                for b in (32, 128)}
         if w.name != "layer200m":
+            # the 200M-layer step at its chunk 512 and at its second chunk
+            # length, 64 (computed as 128-token chunks on the tensor cores)
             sw = wl.WORKLOADS["layer200m"]
-            line["secondary"] = {"layer200m": measure_prefill(args, sw, sw.chunk, rank, world,
-                                                              dev, full=False)}
+            line["secondary"] = {
+                "layer200m": measure_prefill(args, sw, sw.chunk, rank, world, dev, full=False),
+                "layer200m_chunk64": measure_prefill(args, sw, 64, rank, world, dev, full=False),
+            }
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -599,13 +608,16 @@ def measure_prefill(args, w, chunk, rank, world, dev, full=True):
         avg_s = tot / cnt / 1e3
         th = B * n * H
         if dom in ("tc_output", "simt_output"):
+            # the tensor-core kernels compute chunks below 128 as 128-token
+            # chunks: the work they do is that chunk length's
+            kc = max(chunk, 128) if dom.startswith("tc") else chunk
             flops = (parallel_flops_per_token_head(d, n) if par else
-                     output_kernel_flops_per_token_head(d, chunk)) * th
+                     output_kernel_flops_per_token_head(d, kc)) * th
             achieved = flops / avg_s / 1e12
             if dom.startswith("tc"):
                 # the binding roof of min(tensor peak, HBM bandwidth x intensity):
                 # the larger of the two floors, flops / peak and bytes / bandwidth
-                nbytes = None if par else output_kernel_bytes(B, H, n, d, chunk, bool(w.hidden))
+                nbytes = None if par else output_kernel_bytes(B, H, n, d, kc, bool(w.hidden))
                 tensor = {"achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                           "frac": achieved / peaks["bf16_tflops"], "work_per_launch": flops}
                 hbm = None
@@ -620,7 +632,8 @@ def measure_prefill(args, w, chunk, rank, world, dev, full=True):
                         "traffic": None if par else measured_traffic(dom, w.name),
                         "peak_source": peak_src, "work_per_launch": binding["work_per_launch"],
                         "avg_us": avg_s * 1e6, "tensor": tensor, "hbm": hbm,
-                        "intensity_flop_per_byte": flops / nbytes if nbytes else None}
+                        "intensity_flop_per_byte": flops / nbytes if nbytes else None,
+                        "chunk_computed": None if par else kc}
             else:   # float32 FFMA: 148 SMs x 128 lanes x 2 flop x max SM clock
                 peak = 148 * 128 * 2 * (peaks.get("sm_max_mhz", 1965.0) * 1e6) / 1e12
                 roof = {"kernel": dom, "bound": "alu", "achieved": achieved, "peak": peak,
