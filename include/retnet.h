@@ -339,6 +339,12 @@ RETNET_API retnet_status retnet_linear(const void *x, const void *w, void *y, lo
  *   hidden must be a multiple of 256 and H d a multiple of 256, else
  *   UNSUPPORTED.  y must not overlap x, the weights, the states or the
  *   workspace.
+ *   When the retention takes the tensor-core path (d = 256, chunks up to
+ *   1024, decays that admit the fold), the projection's epilogue applies R
+ *   and the decay fold to q and k and writes them as the prefill's operands,
+ *   so q and k are never stored unrotated; the result matches the
+ *   definition above to rounding (q and k are not rounded to bf16 before
+ *   the rotation).
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
 RETNET_API retnet_status retnet_msr_workspace_size(const retnet_shape *shape, int hidden,
                                                    int chunk, size_t *bytes);

@@ -1584,6 +1584,14 @@ size_t tc_workspace_bytes(int batch, int heads, int seqlen, int chunk) {
     return tc_layout(batch, heads, seqlen, effective_chunk(chunk)).total;
 }
 
+void tc_operand_layout(int batch, int heads, int seqlen, int chunk, size_t *qt, size_t *kt,
+                       int *fold) {
+    const TcLayout l = tc_layout(batch, heads, seqlen, effective_chunk(chunk));
+    *qt = l.qt;
+    *kt = l.kt;
+    *fold = effective_chunk(chunk);
+}
+
 // The parallel form runs the output pass over the whole sequence as one
 // block of whole 128-row tiles.
 static int parallel_span(int n) { return (n + kBlk - 1) / kBlk * kBlk; }
@@ -1668,10 +1676,10 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
     // also folds q itself, and the prep pass writes only Kt.
     const int pair_mode = output_pairing_mode();
     const bool pairs = pair_mode != 0 && C / kBlk >= 2;
-    const bool fold_q = pairs && pair_mode == 1;
+    const bool fold_q = pairs && pair_mode == 1 && !a.prefolded;
     double pp_theta[kD / 2];
     for (int j = 0; j < kD / 2; ++j) pp_theta[j] = std::pow(10000.0, -2.0 * j / kD);
-    {
+    if (!a.prefolded) {
         TcPrepParams pp;
         for (int j = 0; j < kD / 2; ++j) pp.theta[j] = pp_theta[j];
         for (int h = 0; h < kMaxHeads; ++h) pp.log2g[h] = hp.log2g[h];

@@ -51,7 +51,73 @@ struct GemmArgs {
     int n_split;                            // columns per output
     int tiles_m, tiles_n;
     unsigned *err;
+    GemmFold fold;                          // outputs 0 and 1 as Qt, Kt (fold.on)
 };
+
+// Where row `grow` of a tile whose 256 columns go to output `which` at
+// column c_in lands, and, for a folded output, the row's position and
+// decay factor.
+struct GemmRow {
+    __nv_bfloat16 *dst;                     // the row's first column; null: not written
+    bool fold;
+    float scale;
+    const float2 *cs;                       // the row's 128 (cos, sin) pairs
+};
+
+__device__ __forceinline__ GemmRow gemm_row(const GemmArgs &a, long long grow, int which,
+                                            int c_in, bool live) {
+    GemmRow r{nullptr, false, 1.f, nullptr};
+    if (!live) return r;
+    // (a select chain, not a dynamic index, keeps a.out out of local memory)
+    __nv_bfloat16 *base = which == 0   ? a.out[0]
+                          : which == 1 ? a.out[1]
+                          : which == 2 ? a.out[2]
+                                       : a.out[3];
+    if (a.fold.on && which < 2) {
+        const long long b = grow / a.fold.n;
+        const int t = (int)(grow - b * a.fold.n);
+        const int h = c_in / 256;
+        const float e = (float)(t % a.fold.fold + 1) * a.fold.log2g[h];
+        r.scale = exp2f(which == 0 ? e : -e);
+        r.cs = a.fold.table + (size_t)t * 128;
+        r.fold = true;
+        r.dst = base + ((b * a.fold.heads + h) * (long long)a.fold.n + t) * 256;
+    } else {
+        r.dst = base + grow * a.n_split + c_in;
+    }
+    return r;
+}
+
+// Stores columns [32 cb, 32 cb + 32) of the row (bf16), folded if asked:
+// pair j = 16 cb + p turned by the row's (cos, sin) of pair j and scaled.
+__device__ __forceinline__ void gemm_store32(const GemmRow &r, int cb, const uint32_t (&v)[32]) {
+    uint4 *d4 = reinterpret_cast<uint4 *>(r.dst + 32 * cb);
+    if (r.fold) {
+        float4 cs4[8];                      // pairs 16 cb .. 16 cb + 15, two per float4
+        const float4 *src = reinterpret_cast<const float4 *>(r.cs + 16 * cb);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cs4[i] = src[i];
+        uint32_t y[16];
+#pragma unroll
+        for (int p = 0; p < 16; ++p) {
+            const float cc = (p & 1) ? cs4[p / 2].z : cs4[p / 2].x;
+            const float ss = (p & 1) ? cs4[p / 2].w : cs4[p / 2].y;
+            const float c = cc * r.scale, sn = ss * r.scale;
+            const float x0 = __uint_as_float(v[2 * p]), x1 = __uint_as_float(v[2 * p + 1]);
+            y[p] = pack_bf16x2(x0 * c - x1 * sn, x0 * sn + x1 * c);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) d4[q] = make_uint4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+        return;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        d4[q] = make_uint4(
+            pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+            pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+            pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+            pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+}
 
 __device__ __forceinline__ void gemm_tile(const GemmArgs &a, int t, int &mb, int &nb) {
     const int per_group = kGemmGroup * a.tiles_n;
@@ -170,12 +236,7 @@ gemm_bf16_tn_kernel(const __grid_constant__ CUtensorMap tm_x,
             const int which = col0 / a.n_split;
             const int c_in = col0 % a.n_split;
             const bool live = grow < a.m && in_bounds(which, 4, err, kSiteGemm);
-            // (a select chain, not a dynamic index, keeps a.out out of local memory)
-            __nv_bfloat16 *base = which == 0   ? a.out[0]
-                                  : which == 1 ? a.out[1]
-                                  : which == 2 ? a.out[2]
-                                               : a.out[3];
-            __nv_bfloat16 *dst = live ? base + grow * a.n_split + c_in : nullptr;
+            const GemmRow r = gemm_row(a, grow, which, c_in, live);
 #pragma unroll 1
             for (int cb = 0; cb < kGemmN / 32; ++cb) {
                 uint32_t v[32];
@@ -185,16 +246,7 @@ gemm_bf16_tn_kernel(const __grid_constant__ CUtensorMap tm_x,
                     tc_fence_before();
                     mbar_arrive(&acc_free[buf]);
                 }
-                if (live) {
-                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * cb);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        d4[q] = make_uint4(
-                            pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
-                            pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
-                            pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
-                            pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
-                }
+                if (live) gemm_store32(r, cb, v);
             }
         }
     }
@@ -360,11 +412,7 @@ gemm_bf16_tn_pair_kernel(const __grid_constant__ CUtensorMap tm_x,
             const int which = col0 / a.n_split;
             const int c_in = col0 % a.n_split;
             const bool live = grow < a.m && in_bounds(which, 4, err, kSiteGemm);
-            __nv_bfloat16 *base = which == 0   ? a.out[0]
-                                  : which == 1 ? a.out[1]
-                                  : which == 2 ? a.out[2]
-                                               : a.out[3];
-            __nv_bfloat16 *dst = live ? base + grow * a.n_split + c_in : nullptr;
+            const GemmRow r = gemm_row(a, grow, which, c_in, live);
             const uint32_t l_free = mapa_shared(smem_u32(&acc_free[buf]), 0);
 #pragma unroll 1
             for (int cb = 0; cb < kGemmN / 32; ++cb) {
@@ -375,16 +423,7 @@ gemm_bf16_tn_pair_kernel(const __grid_constant__ CUtensorMap tm_x,
                     tc_fence_before();
                     mbar_arrive_cluster(l_free);
                 }
-                if (live) {
-                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * cb);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        d4[q] = make_uint4(
-                            pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
-                            pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
-                            pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
-                            pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
-                }
+                if (live) gemm_store32(r, cb, v);
             }
         }
         if (!ok && lane == 0) abort_both();
@@ -427,7 +466,8 @@ bool gemm_shape_ok(long long m, int n, int k, int n_split) {
 }
 
 cudaError_t launch_gemm_bf16(const void *x, const void *w, void *const *outs, long long m, int n,
-                             int k, int n_split, cudaStream_t stream, const char *timer_name) {
+                             int k, int n_split, cudaStream_t stream, const char *timer_name,
+                             const GemmFold *fold) {
     if (m == 0) return cudaSuccess;
     CUtensorMap tm_x, tm_w;
     {
@@ -449,6 +489,8 @@ cudaError_t launch_gemm_bf16(const void *x, const void *w, void *const *outs, lo
     a.k = k;
     a.n_split = n_split;
     a.tiles_n = n / kGemmN;
+    if (fold) a.fold = *fold;
+    else a.fold.on = 0;
     a.err = device_error_word();
     if (!a.err) return cudaErrorInvalidValue;
     int dev = 0, sms = 148;

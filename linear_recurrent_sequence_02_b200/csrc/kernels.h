@@ -59,6 +59,10 @@ struct ChunkwiseArgs {
     HeadGammas gam;
     void *workspace;
     size_t workspace_bytes;
+    // Tensor-core path only: Qt and Kt are already in the workspace (the MSR
+    // layer's projection GEMM folded them), so the prep pass is skipped and
+    // q, k are not read.
+    bool prefolded = false;
 };
 size_t simt_workspace_bytes(int batch, int heads, int seqlen, int dk, int dv, int chunk);
 cudaError_t launch_chunkwise_simt(const ChunkwiseArgs &a, cudaStream_t stream);
@@ -69,6 +73,11 @@ bool tc_shape_ok(int dk, int dv, retnet_dtype dtype, int chunk);
 // Every head's decay admits the decay fold: gamma > 0 and chunk*log2(1/gamma) <= 100.
 bool tc_gammas_ok(int chunk, const float *gammas, int heads);
 size_t tc_workspace_bytes(int batch, int heads, int seqlen, int chunk);
+// Byte offsets of Qt and Kt ([B*H, n, 256] bf16 each) in the workspace, and
+// the block length their decay is folded over (the chunk, or 128 for chunks
+// below 128).
+void tc_operand_layout(int batch, int heads, int seqlen, int chunk, size_t *qt, size_t *kt,
+                       int *fold);
 // parallel: the parallel form over the whole sequence (a.chunk, state_in and
 // state_out unused; decays must pass tc_gammas_ok at chunk 128).
 cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cudaStream_t stream,
@@ -80,12 +89,26 @@ bool make_tensor_map_bf16(CUtensorMap *m, const void *base, int rank, const cuui
                           const cuuint64_t *strides_bytes, const cuuint32_t *box);
 
 // gemm_tc.cu ---------------------------------------------------------------
+// Rotation and decay fold applied by the GEMM's epilogue to outputs 0 and 1
+// (the MSR layer's Q and K, 256 columns per head): with row r = b n + t,
+// column 2j, 2j+1 of head h is turned by table[t * 128 + j] (the (cos, sin)
+// of (pos0 + t) theta_j, from launch_rotation_table) and scaled by
+// gamma_h^(+(t mod fold + 1)) (output 0) or gamma_h^(-(t mod fold + 1))
+// (output 1), and written as Qt, Kt in the prefill's [b*H + h][t][256]
+// layout instead of [m, n_split].
+struct GemmFold {
+    int on;
+    int n, heads, fold;
+    const float2 *table;           // [n, 128] device
+    float log2g[kMaxHeads];
+};
 // Y = X W^T on the tensor cores: X [m, k], W [n, k], bf16, f32 accumulation.
 // Columns [j n_split, (j+1) n_split) of Y go to outs[j] ([m, n_split], dense).
 // timer_name: the kernel timer's name for this launch (a string literal).
+// fold (optional): outputs 0 and 1 folded as GemmFold describes.
 bool gemm_shape_ok(long long m, int n, int k, int n_split);
 cudaError_t launch_gemm_bf16(const void *x, const void *w, void *const *outs, long long m, int n,
                              int k, int n_split, cudaStream_t stream,
-                             const char *timer_name = "gemm");
+                             const char *timer_name = "gemm", const GemmFold *fold = nullptr);
 
 }  // namespace retnet

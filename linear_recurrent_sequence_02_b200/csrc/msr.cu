@@ -11,6 +11,13 @@
 // with the rotation R, the per-head decays and the GroupNorm of
 // retnet_retention_chunkwise.  Weights use the [out_features, in_features]
 // layout of a linear layer.
+//
+// When the retention runs on the tensor cores, the projection GEMM's
+// epilogue also applies R and the decay fold to Q and K and writes them as
+// the prefill's Qt, Kt operands, so the prefill starts at its state pass:
+// Q and K never go through HBM unfolded.
+#include <cmath>
+
 #include "kernels.h"
 
 namespace retnet {
@@ -19,9 +26,10 @@ namespace {
 size_t align1k(size_t x) { return (x + 1023) & ~(size_t)1023; }
 
 // Workspace of the layer: Q, K, V, G and the retention output Y, each
-// [B*n, H*d] bf16, then the prefill's own workspace.
+// [B*n, H*d] bf16, the prefill's own workspace, then the rotation table
+// [n, 128] (cos, sin) pairs that the projection's epilogue reads.
 struct MsrLayout {
-    size_t q, k, v, g, y, fwd, fwd_bytes, total;
+    size_t q, k, v, g, y, fwd, fwd_bytes, table, total;
 };
 
 retnet_status msr_layout(const retnet_shape *s, int hidden, int chunk, MsrLayout *l) {
@@ -44,7 +52,8 @@ retnet_status msr_layout(const retnet_shape *s, int hidden, int chunk, MsrLayout
     l->y = l->g + part;
     l->fwd = l->y + part;
     l->fwd_bytes = fwd;
-    l->total = l->fwd + fwd;
+    l->table = l->fwd + align1k(fwd);
+    l->total = l->table + align1k((size_t)s->seqlen * 128 * sizeof(float2));
     return RETNET_OK;
 }
 
@@ -107,20 +116,51 @@ retnet_status retnet_msr_layer(const void *x, const void *w_qkvg, const void *w_
     char *ws = (char *)workspace;
     const int hd = shape->heads * shape->dk;
     void *q = ws + l.q, *k = ws + l.k, *v = ws + l.v, *g = ws + l.g, *o = ws + l.y;
-    if (rows > 0) {
-        void *outs[4] = {q, k, v, g};
-        RETNET_CUDA_TRY(launch_gemm_bf16(x, w_qkvg, outs, rows, 4 * hd, hidden, hd, s,
-                                         "gemm_qkvg"));
-    }
     retnet_gate gate;
     gate.g = g;
     gate.weight = gn_weight;
     gate.bias = gn_bias;
     gate.eps = eps;
-    st = retnet_retention_chunkwise(q, k, v, gammas, chunk, o, shape, pos0, 1, state_in,
-                                    state_out, &gate, RETNET_ALGO_AUTO, ws + l.fwd, l.fwd_bytes,
-                                    stream);
-    if (st != RETNET_OK) return st;
+    // the tensor-core prefill, as retnet_retention_chunkwise would choose it
+    const bool fused = rows > 0 && tc_shape_ok(shape->dk, shape->dv, shape->dtype, chunk) &&
+                       tc_gammas_ok(chunk, gammas, shape->heads);
+    if (!fused) {
+        if (rows > 0) {
+            void *outs[4] = {q, k, v, g};
+            RETNET_CUDA_TRY(launch_gemm_bf16(x, w_qkvg, outs, rows, 4 * hd, hidden, hd, s,
+                                             "gemm_qkvg"));
+        }
+        st = retnet_retention_chunkwise(q, k, v, gammas, chunk, o, shape, pos0, 1, state_in,
+                                        state_out, &gate, RETNET_ALGO_AUTO, ws + l.fwd,
+                                        l.fwd_bytes, stream);
+        if (st != RETNET_OK) return st;
+    } else {
+        size_t qt_off = 0, kt_off = 0;
+        GemmFold fold;
+        fold.on = 1;
+        fold.n = shape->seqlen;
+        fold.heads = shape->heads;
+        tc_operand_layout(shape->batch, shape->heads, shape->seqlen, chunk, &qt_off, &kt_off,
+                          &fold.fold);
+        for (int h = 0; h < kMaxHeads; ++h)
+            fold.log2g[h] = h < shape->heads ? (float)std::log2((double)gammas[h]) : 0.f;
+        float2 *table = reinterpret_cast<float2 *>(ws + l.table);
+        RETNET_CUDA_TRY(launch_rotation_table(table, shape->seqlen, 256, pos0, s));
+        fold.table = table;
+        char *fwd = ws + l.fwd;
+        void *outs[4] = {fwd + qt_off, fwd + kt_off, v, g};
+        RETNET_CUDA_TRY(launch_gemm_bf16(x, w_qkvg, outs, rows, 4 * hd, hidden, hd, s,
+                                         "gemm_qkvg", &fold));
+        ChunkwiseArgs a;
+        a.q = nullptr; a.k = nullptr; a.v = v; a.out = o;
+        a.state_in = state_in; a.state_out = state_out; a.gate = &gate;
+        a.batch = shape->batch; a.heads = shape->heads; a.seqlen = shape->seqlen;
+        a.dk = shape->dk; a.dv = shape->dv; a.chunk = chunk; a.dtype = shape->dtype;
+        a.pos0 = pos0; a.rotate = 1; a.workspace = fwd; a.workspace_bytes = l.fwd_bytes;
+        for (int h = 0; h < kMaxHeads; ++h) a.gam.g[h] = h < shape->heads ? gammas[h] : 0.f;
+        a.prefolded = true;
+        RETNET_CUDA_TRY(launch_chunkwise_tc(a, gammas, s));
+    }
     if (rows > 0) {
         void *outs[1] = {y};
         RETNET_CUDA_TRY(launch_gemm_bf16(o, w_o, outs, rows, hidden, hd, hidden, s, "gemm_out"));

@@ -114,3 +114,25 @@ def test_msr_layer_200m_shape(rn):
     got, want, st, ws = _layer(rn, w.batch, w.seqlen, w.hidden, w.heads, w.d, w.chunk, 33)
     assert slice_rel_err(got[:, :, None], want[:, :, None]) < TOL
     assert slice_rel_err(st, ws, head_axis=1) < TOL
+
+
+def test_msr_layer_folded_by_the_single_cta_gemm_at_chunk_64(rn):
+    # 100 rows: the projection runs on single CTAs, whose epilogue rotates and
+    # decay-folds Q and K; chunk 64 is computed with the fold over 128 tokens;
+    # a far position exercises the angle reduction
+    got, want, st, ws = _layer(rn, 1, 100, 256, 1, 256, 64, 34, pos0=5000, state=True)
+    assert slice_rel_err(got[:, :, None], want[:, :, None]) < TOL
+    assert slice_rel_err(st, ws, head_axis=1) < TOL
+
+
+@pytest.mark.parametrize("pairs", [1, 2])
+def test_msr_layer_folded_operands_on_cta_pairs(rn, pairs):
+    # the output pass on CTA pairs; in mode 1 the pairs fold raw q themselves,
+    # which the layer's already folded Qt must not go through again
+    rn.retnet_set_output_pairing(pairs)
+    try:
+        got, want, st, ws = _layer(rn, 1, 1100, 256, 2, 256, 512, 35, pos0=17, state=True)
+    finally:
+        rn.retnet_set_output_pairing(0)
+    assert slice_rel_err(got[:, :, None], want[:, :, None]) < TOL
+    assert slice_rel_err(st, ws, head_axis=1) < TOL
