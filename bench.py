@@ -109,7 +109,7 @@ NCU_TRAFFIC = {
     ("tc_output", "long7b"): {
         "source": "chunkwise_tc.cu", "section": "output pass",
         "headers": ["sm100.cuh", "common.cuh"],
-        "sha256": "97a24651b782322a9322bb14fc605869870f25c184670e922ec1b7406a49dfeb",
+        "sha256": "b8813a88b501781786be145125861691968076f253afbfefdcfe817e3019eaba",
         "bytes": 277.98e6,
     },
 }
