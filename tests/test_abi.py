@@ -299,6 +299,51 @@ def test_bench_work_counts_match_the_formulas():
     assert bench.parallel_flops_per_token_head(d, 2047) == 2 * d * 2048
 
 
+def test_bench_output_pass_bytes_at_the_long_prefill():
+    """Algorithmic bytes of one output-pass launch at B=1, H=16, n=8192,
+    chunk 512: Qt, Kt, V read and O written once (2 B each per element),
+    plus S_prev (d x d bf16) for the 15 chunks after the first."""
+    import bench
+    th = 1 * 16 * 8192
+    want = th * 256 * 2 * 4 + 16 * 15 * 256 * 256 * 2
+    assert bench.output_kernel_bytes(1, 16, 8192, 256, 512, False) == want == 299_892_736
+    # with a gate: G read once more
+    assert bench.output_kernel_bytes(1, 16, 8192, 256, 512, True) == want + th * 256 * 2
+
+
+def test_bench_kernel_hash_covers_its_section_only(tmp_path, monkeypatch):
+    """The stored ncu traffic is keyed by a hash of one banner-delimited
+    section of a .cu file and the headers: it changes with that section and
+    the headers, not with another section."""
+    import bench
+    csrc = tmp_path / "linear_recurrent_sequence_02_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    banner = bench.SECTION_BANNER
+    (csrc / "k.cu").write_text(f"{banner}alpha\nint a;\n{banner}beta\nint b;\n")
+    (csrc / "h.cuh").write_text("int h;\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    base = bench.kernel_source_sha("k.cu", "alpha", ["h.cuh"])
+    assert base is not None
+    (csrc / "k.cu").write_text(f"{banner}alpha\nint a;\n{banner}beta\nint b2;\n")
+    assert bench.kernel_source_sha("k.cu", "alpha", ["h.cuh"]) == base
+    (csrc / "k.cu").write_text(f"{banner}alpha\nint a2;\n{banner}beta\nint b2;\n")
+    assert bench.kernel_source_sha("k.cu", "alpha", ["h.cuh"]) != base
+    (csrc / "k.cu").write_text(f"{banner}alpha\nint a;\n{banner}beta\nint b;\n")
+    (csrc / "h.cuh").write_text("int h2;\n")
+    assert bench.kernel_source_sha("k.cu", "alpha", ["h.cuh"]) != base
+    assert bench.kernel_source_sha("k.cu", "gamma", ["h.cuh"]) is None
+
+
+def test_bench_stored_traffic_matches_the_current_output_pass():
+    """The recorded ncu traffic is reported only while its source hash
+    matches; it does match the output pass as committed."""
+    import bench
+    rec = bench.NCU_TRAFFIC[("tc_output", "long7b")]
+    assert bench.kernel_source_sha(rec["source"], rec["section"], rec["headers"]) == rec["sha256"]
+    assert bench.measured_traffic("tc_output", "long7b") == rec["bytes"]
+    assert bench.measured_traffic("tc_output", "layer200m") is None
+
+
 def test_linear_and_msr_layer_reject_before_launch(lib):
     P = ctypes.c_void_p
     # retnet_linear(x, w, y, rows, in, out, stream)
