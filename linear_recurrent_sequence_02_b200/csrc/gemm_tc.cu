@@ -77,6 +77,10 @@ __device__ __forceinline__ GemmRow gemm_row(const GemmArgs &a, long long grow, i
         const long long b = grow / a.fold.n;
         const int t = (int)(grow - b * a.fold.n);
         const int h = c_in / 256;
+        // debug build: the row of Qt / Kt lies inside the [B*H, n] operand
+        if (!in_bounds((b * a.fold.heads + h) * (long long)a.fold.n + t, a.m * a.fold.heads, a.err,
+                       kSiteGemm))
+            return r;
         const float e = (float)(t % a.fold.fold + 1) * a.fold.log2g[h];
         r.scale = exp2f(which == 0 ? e : -e);
         r.cs = a.fold.table + (size_t)t * 128;
@@ -246,7 +250,7 @@ gemm_bf16_tn_kernel(const __grid_constant__ CUtensorMap tm_x,
                     tc_fence_before();
                     mbar_arrive(&acc_free[buf]);
                 }
-                if (live) gemm_store32(r, cb, v);
+                if (live && r.dst) gemm_store32(r, cb, v);
             }
         }
     }
@@ -423,7 +427,7 @@ gemm_bf16_tn_pair_kernel(const __grid_constant__ CUtensorMap tm_x,
                     tc_fence_before();
                     mbar_arrive_cluster(l_free);
                 }
-                if (live) gemm_store32(r, cb, v);
+                if (live && r.dst) gemm_store32(r, cb, v);
             }
         }
         if (!ok && lane == 0) abort_both();

@@ -115,3 +115,27 @@ def test_index_checks_quiet_and_bits_equal_decode(rn, tokens):
         rn.retnet_check_device_errors()
     assert torch.equal(got[0], want[0])
     assert torch.equal(got[1], want[1])
+
+
+@pytest.mark.parametrize("B,n,chunk", [(1, 100, 64), (2, 700, 256)])
+def test_index_checks_quiet_and_bits_equal_msr_layer(rn, B, n, chunk):
+    # the layer's projection GEMM (single CTAs at 100 rows, CTA pairs at 1400)
+    # with its epilogue rotation and decay fold, and the prefolded prefill
+    H, d, hidden = 2, 256, 512
+    x, wqkvg, wo = (_dev(a) for a in wl.make_msr_inputs(B, n, hidden, H, d, 830 + n))
+    gam = rn.retnet_default_gammas(H)
+    rng = np.random.default_rng(n + 1)
+    s0 = torch.from_numpy(rng.standard_normal((B, H, d, d)).astype(np.float32) * 0.05).cuda()
+
+    def run():
+        st = torch.full((B, H, d, d), float("nan"), device="cuda")
+        y = rn.retnet_msr_layer(x, wqkvg, wo, gam, chunk, pos0=11, state_in=s0, state_out=st)
+        return y, st
+
+    want = run()
+    rn.retnet_check_device_errors()
+    with rn.using_library(rn.DEBUG_LIB_PATH):
+        got = run()
+        rn.retnet_check_device_errors()
+    assert torch.equal(got[0], want[0])
+    assert torch.equal(got[1], want[1])
