@@ -2,6 +2,7 @@
 //
 // Every check runs before anything is enqueued, so a rejected call leaves
 // all buffers untouched and launches nothing.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 
@@ -135,6 +136,31 @@ static BackwardLayout backward_layout(const retnet_shape *s, int chunk, retnet_a
     l.fwd = l.rkh + bk;
     l.fwd_bytes = backward_fwd_bytes(s, chunk, algo, gammas);
     l.total = l.fwd + l.fwd_bytes;
+    return l;
+}
+
+// The tensor-core backward whose retentions run without their prep pass
+// (bf16, d_k = d_v = 256): the three retentions' values and the outputs of
+// the two reversed-time ones, then one prefill workspace per retention,
+// whose Qt and Kt the fold kernel fills.
+struct FusedBackwardLayout {
+    size_t val[3], out2, out3, fwd[3], fwd_bytes, total;
+};
+static bool backward_fusable(const retnet_shape *s, int chunk, retnet_algo algo) {
+    return algo != RETNET_ALGO_SIMT && s->dtype == RETNET_BF16 && s->dk == 256 && s->dv == 256 &&
+           tc_shape_ok(s->dk, s->dv, s->dtype, chunk);
+}
+static FusedBackwardLayout fused_backward_layout(const retnet_shape *s, int chunk) {
+    const size_t b = align1k((size_t)s->batch * s->seqlen * s->heads * 256 * 2);
+    FusedBackwardLayout l;
+    size_t at = 0;
+    for (int i = 0; i < 3; ++i, at += b) l.val[i] = at;
+    l.out2 = at;
+    l.out3 = at + b;
+    at += 2 * b;
+    l.fwd_bytes = align1k(tc_workspace_bytes(s->batch, s->heads, s->seqlen, chunk));
+    for (int i = 0; i < 3; ++i, at += l.fwd_bytes) l.fwd[i] = at;
+    l.total = at;
     return l;
 }
 
@@ -319,9 +345,13 @@ retnet_status retnet_backward_workspace_size(const retnet_shape *shape, int chun
         return RETNET_ERR_INVALID_ARG;
     if (algo == RETNET_ALGO_TENSOR && !tc_shape_ok(shape->dk, shape->dv, shape->dtype, chunk))
         return RETNET_ERR_UNSUPPORTED;
-    *bytes = (long long)shape->batch * shape->seqlen == 0
-                 ? 0
-                 : backward_layout(shape, chunk, algo, nullptr).total;
+    size_t need = 0;
+    if ((long long)shape->batch * shape->seqlen > 0) {
+        need = backward_layout(shape, chunk, algo, nullptr).total;
+        if (backward_fusable(shape, chunk, algo))      // whichever the decays select
+            need = std::max(need, fused_backward_layout(shape, chunk).total);
+    }
+    *bytes = need;
     return RETNET_OK;
 }
 
@@ -355,11 +385,50 @@ retnet_status retnet_retention_backward(const void *q, const void *k, const void
             return RETNET_ERR_UNSUPPORTED;
     }
     if (tokens == 0) return RETNET_OK;
+    const bool fused = ra == RETNET_ALGO_TENSOR && rb == RETNET_ALGO_TENSOR &&
+                       backward_fusable(shape, chunk, algo);
     const BackwardLayout lay = backward_layout(shape, chunk, algo, gammas);
-    if (!workspace || workspace_bytes < lay.total || ((uintptr_t)workspace & 1023u))
+    const size_t need = fused ? fused_backward_layout(shape, chunk).total : lay.total;
+    if (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 1023u))
         return RETNET_ERR_WORKSPACE;
 
     const cudaStream_t s = (cudaStream_t)stream;
+    if (fused) {
+        // the fold kernel writes every retention's operands; the retentions
+        // then run from their Qt, Kt without a prep pass
+        const FusedBackwardLayout fl = fused_backward_layout(shape, chunk);
+        char *ws = (char *)workspace;
+        size_t qt_off = 0, kt_off = 0;
+        int fold = 0;
+        tc_operand_layout(shape->batch, shape->heads, shape->seqlen, chunk, &qt_off, &kt_off,
+                          &fold);
+        void *qt[3], *kt[3], *vals[3];
+        for (int i = 0; i < 3; ++i) {
+            qt[i] = ws + fl.fwd[i] + qt_off;
+            kt[i] = ws + fl.fwd[i] + kt_off;
+            vals[i] = ws + fl.val[i];
+        }
+        RETNET_CUDA_TRY(launch_backward_fold(q, k, v, d_out, qt, kt, vals, gammas,
+                                             shape->batch, shape->heads, shape->seqlen, fold,
+                                             pos0, rotate, s));
+        void *outs[3] = {dq, ws + fl.out2, ws + fl.out3};
+        for (int i = 0; i < 3; ++i) {
+            ChunkwiseArgs a = base;
+            a.q = nullptr; a.k = nullptr; a.v = vals[i]; a.out = outs[i];
+            a.state_in = nullptr; a.state_out = nullptr; a.gate = nullptr;
+            a.batch = shape->batch; a.heads = shape->heads; a.seqlen = shape->seqlen;
+            a.dk = 256; a.dv = 256; a.chunk = chunk; a.dtype = shape->dtype;
+            a.pos0 = 0; a.rotate = 0;
+            a.workspace = ws + fl.fwd[i];
+            a.workspace_bytes = fl.fwd_bytes;
+            a.prefolded = true;
+            RETNET_CUDA_TRY(launch_chunkwise_tc(a, gammas, s));
+        }
+        RETNET_CUDA_TRY(launch_backward_post(dq, ws + fl.out2, ws + fl.out3, dk, dv, shape->batch,
+                                             shape->heads, shape->seqlen, 256, 256,
+                                             shape->dtype, pos0, rotate, s));
+        return RETNET_OK;
+    }
     const int B = shape->batch, n = shape->seqlen, H = shape->heads;
     const int DK = shape->dk, DV = shape->dv;
     const retnet_dtype dt = shape->dtype;

@@ -199,6 +199,110 @@ BackwardThetas backward_thetas(int dk) {
     return th;
 }
 
+// The tensor-core backward (bf16, d = 256): the same reads, but the three
+// retentions' operands are written already in the form their prep pass
+// would give, so that they run without it.  With e = (position mod fold) + 1
+// in each retention's own time order (t forward, p = n-1-t reversed):
+//   ret 1 (dQ^):  Qt = g^e dO,      Kt = g^-e V,       values R k   at t
+//   ret 2 (dK~):  Qt = g^e V,       Kt = g^-e dO,      values R q   at p
+//   ret 3 (dV~):  Qt = g^e (R k),   Kt = g^-e (R q),   values dO    at p
+// Qt, Kt in the prefill's [b*H + h][time][256] layout, values in [B, n, H, 256].
+struct BackwardFold {
+    float log2g[kMaxHeads];
+};
+
+__global__ void __launch_bounds__(kBwdThreads, 2)
+backward_fold_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                     const __nv_bfloat16 *__restrict__ v, const __nv_bfloat16 *__restrict__ dout,
+                     __nv_bfloat16 *__restrict__ qt1, __nv_bfloat16 *__restrict__ kt1,
+                     __nv_bfloat16 *__restrict__ val1, __nv_bfloat16 *__restrict__ qt2,
+                     __nv_bfloat16 *__restrict__ kt2, __nv_bfloat16 *__restrict__ val2,
+                     __nv_bfloat16 *__restrict__ qt3, __nv_bfloat16 *__restrict__ kt3,
+                     __nv_bfloat16 *__restrict__ val3, BackwardThetas th, BackwardFold bf,
+                     int batch, int heads, int n, int fold, long long pos0, int rotate) {
+    constexpr int D = 256, kParts = D / 8;
+    using T = __nv_bfloat16;
+    __shared__ float2 cs[128];
+    const int t = blockIdx.x, p = n - 1 - t;
+    token_table(cs, D, pos0 + t, rotate, th);
+    const float e1 = (float)(t % fold + 1), e2 = (float)(p % fold + 1);
+    const int tasks = batch * heads * kParts;
+    for (int base = threadIdx.x; base < tasks; base += kBwdBatch * kBwdThreads) {
+        Raw8<T> rq[kBwdBatch], rk[kBwdBatch], rvv[kBwdBatch], ro[kBwdBatch];
+#pragma unroll
+        for (int u = 0; u < kBwdBatch; ++u) {
+            const int task = base + u * kBwdThreads;
+            if (task < tasks) {
+                const PartIndex x = part_index(task, kParts, heads, n, t, D);
+                rq[u].load(q + x.at_t);
+                rk[u].load(k + x.at_t);
+                rvv[u].load(v + x.at_t);
+                ro[u].load(dout + x.at_t);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kBwdBatch; ++u) {
+            const int task = base + u * kBwdThreads;
+            if (task >= tasks) continue;
+            const PartIndex x = part_index(task, kParts, heads, n, t, D);
+            const int bh = task / kParts, h = bh % heads;
+            // rows of the [b*H + h][time][256] operands at t and at p
+            const size_t ot = ((size_t)bh * n + t) * D + x.part * 8;
+            const size_t op = ((size_t)bh * n + p) * D + x.part * 8;
+            const float l2 = bf.log2g[h];
+            const float s1 = exp2f(e1 * l2), s1i = exp2f(-e1 * l2);
+            const float s2 = exp2f(e2 * l2), s2i = exp2f(-e2 * l2);
+            float eq[8], ek[8], ev[8], eo[8], y[8];
+            rq[u].to_float(eq);
+            rk[u].to_float(ek);
+            rvv[u].to_float(ev);
+            ro[u].to_float(eo);
+            turn(eq, cs + 4 * x.part, 1.f);
+            turn(ek, cs + 4 * x.part, 1.f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) y[i] = s1 * eo[i];
+            store8(qt1 + ot, y);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) y[i] = s1i * ev[i];
+            store8(kt1 + ot, y);
+            store8(val1 + x.at_t, ek);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) y[i] = s2 * ev[i];
+            store8(qt2 + op, y);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) y[i] = s2i * eo[i];
+            store8(kt2 + op, y);
+            store8(val2 + x.at_rev, eq);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) y[i] = s2 * ek[i];
+            store8(qt3 + op, y);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) y[i] = s2i * eq[i];
+            store8(kt3 + op, y);
+            ro[u].store(val3 + x.at_rev);
+        }
+    }
+}
+
+cudaError_t launch_backward_fold(const void *q, const void *k, const void *v, const void *dout,
+                                 void *const *qt, void *const *kt, void *const *vals,
+                                 const float *gammas, int batch, int heads, int n, int fold,
+                                 long long pos0, int rotate, cudaStream_t stream) {
+    if ((long long)batch * n == 0) return cudaSuccess;
+    const BackwardThetas th = backward_thetas(256);
+    BackwardFold bf;
+    for (int h = 0; h < kMaxHeads; ++h)
+        bf.log2g[h] = h < heads ? (float)std::log2((double)gammas[h]) : 0.f;
+    using T = __nv_bfloat16;
+    KernelTimer timer("backward_prep", stream);
+    backward_fold_kernel<<<n, kBwdThreads, 0, stream>>>(
+        (const T *)q, (const T *)k, (const T *)v, (const T *)dout, (T *)qt[0], (T *)kt[0],
+        (T *)vals[0], (T *)qt[1], (T *)kt[1], (T *)vals[1], (T *)qt[2], (T *)kt[2], (T *)vals[2],
+        th, bf, batch, heads, n, fold, pos0, rotate);
+    count_launch();
+    return cudaGetLastError();
+}
+
 cudaError_t launch_backward_prep(const void *q, const void *k, const void *v, const void *dout,
                                  void *kh, void *rkh, void *rqh, void *rv, void *rdo, int batch,
                                  int heads, int n, int dk, int dv, retnet_dtype dtype,

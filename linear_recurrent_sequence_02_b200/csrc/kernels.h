@@ -25,6 +25,14 @@ cudaError_t launch_backward_prep(const void *q, const void *k, const void *v, co
                                  void *kh, void *rkh, void *rqh, void *rv, void *rdo, int batch,
                                  int heads, int n, int dk, int dv, retnet_dtype dtype,
                                  long long pos0, int rotate, cudaStream_t stream);
+// bf16, d = 256, the tensor-core backward: from q, k, v, dO, the three
+// retentions' Qt, Kt (qt[i], kt[i], each in the prefill's [B*H, n, 256]
+// layout with the decay folded over `fold`) and values (vals[i], [B, n, H,
+// 256]): ret 1 = (dO, V; R k), ret 2 = rev(V, dO; R q), ret 3 = rev(R k, R q; dO).
+cudaError_t launch_backward_fold(const void *q, const void *k, const void *v, const void *dout,
+                                 void *const *qt, void *const *kt, void *const *vals,
+                                 const float *gammas, int batch, int heads, int n, int fold,
+                                 long long pos0, int rotate, cudaStream_t stream);
 // dq <- R^T dq (in place); dk = R^T rev(dk_rev); dv = rev(dv_rev).
 cudaError_t launch_backward_post(void *dq, const void *dk_rev, const void *dv_rev, void *dk,
                                  void *dv, int batch, int heads, int n, int dkd, int dvd,
