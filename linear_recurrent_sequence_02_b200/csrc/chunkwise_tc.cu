@@ -39,7 +39,6 @@ using namespace sm100;
 
 constexpr int kD = 256;            // head dimension served here (dk = dv = 256)
 constexpr int kBlk = 128;          // rows per tile
-constexpr int kTcThreads = 192;    // 6 warps
 constexpr uint32_t kBox = 16384;   // one 128-row x 64-col bf16 box (128-B swizzle)
 
 struct TcHeadParams {
@@ -142,21 +141,29 @@ tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restr
 
 // ------------------------------------------------------------------ state pass
 // One CTA per (sequence, head, 128 x DVC block of S): the d_k half mh and
-// d_v columns [DVC nv, DVC nv + DVC).  DVC = 128 (four CTAs per
-// sequence-head) by default; DVC = 64 (eight) when there are few
-// sequence-heads, so that more SMs stream.  Warp 0 streams Kt and V
-// sub-tiles of 128 tokens through a TMA ring; warp 1 accumulates
-// U_c = Kt_c^T V_c of every chunk into one of two TMEM buffers (M = d_k
-// half, N = DVC, both operands MN-major); warps 2-5 keep the running state
-// row in registers, S <- g^L (S + U_c), hand the buffer back as soon as it
-// is read, and write S_prev of the next chunk (bf16) or the final state
-// (f32).  The tensor core never waits for the state update.
+// d_v columns [DVC nv, DVC nv + DVC).  DVC is 64, 128 or 256 (eight, four
+// or two CTAs per sequence-head), chosen per shape by tc_state_columns.
+// Warp 0 streams Kt and V sub-tiles of kTok tokens (128; 64 at DVC = 256,
+// so that four stages fit) through a TMA ring;
+// warp 1 accumulates U_c = Kt_c^T V_c of every chunk into one of two TMEM
+// buffers (M = d_k half, N = DVC, both operands MN-major); the state
+// warpgroups (one per 128 of the DVC columns) keep the running state row in
+// registers, S <- g^L (S + U_c), hand the buffer back as soon as it is
+// read, and write S_prev of the next chunk (bf16) or the final state (f32).
+// The tensor core never waits for the state update.
 template <int DVC>
 struct TcStateSmem {
+    static constexpr int kTok = DVC == 256 ? 64 : 128;         // tokens per stage
+    static constexpr uint32_t kTokBox = kTok * 128;            // kTok rows x 64 channels
     static constexpr int kVBoxes = DVC / 64;
-    static constexpr uint32_t kStage = (2 + kVBoxes) * kBox;   // Kt 128 x 128 + V 128 x DVC
+    static constexpr uint32_t kStage = (2 + kVBoxes) * kTokBox; // Kt kTok x 128 + V kTok x DVC
     static constexpr int kStages = DVC == 128 ? 3 : 4;
     static constexpr uint32_t kBytes = kStages * kStage + 1024;
+    static constexpr int kGroups = DVC > 128 ? DVC / 128 : 1;  // state warpgroups
+    static constexpr int kCols = DVC / kGroups;                 // d_v columns per state thread
+    static constexpr int kThreads = 64 + 128 * kGroups;
+    static constexpr uint32_t kBufCols = DVC < 128 ? 128 : DVC; // TMEM columns per U buffer
+    static constexpr uint32_t kTmemCols = 2 * kBufCols;
 };
 
 __device__ __forceinline__ void store_bf16_row(__nv_bfloat16 *dst, const float *v, int count) {
@@ -174,7 +181,7 @@ static __device__ int g_hook_skip_first_load = 0;
 #endif
 
 template <int DVC>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(TcStateSmem<DVC>::kThreads, 1)
 tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 TcHeadParams hp, const float *__restrict__ state_in, float *__restrict__ state_out,
                 __nv_bfloat16 *__restrict__ s_prev, int heads, int n, int chunk, int nchunks,
@@ -202,14 +209,14 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(&acc_full[x], 1);
-            mbar_init(&acc_free[x], 128);
+            mbar_init(&acc_free[x], 128 * Smem::kGroups);
         }
         mbar_init(&drain, 1);
         abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(&tmem_slot, 256);
+        tmem_alloc(&tmem_slot, Smem::kTmemCols);
         tmem_relinquish();
     }
     if (warp == 0 && lane == 0) {
@@ -228,7 +235,7 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             for (int c = 0; c < nchunks && !abort_flag; ++c) {
                 const int c0 = c * chunk;
                 const int L = min(chunk, n - c0);
-                for (int st = 0; st * kBlk < L; ++st, ++it) {
+                for (int st = 0; st * Smem::kTok < L; ++st, ++it) {
                     const int s = it % S;
                     if (it >= S && !mbar_wait(&empty[s], ((it / S) - 1) & 1, &abort_flag, err))
                         break;
@@ -240,13 +247,15 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     }
 #endif
                     uint8_t *kb = smem + s * Smem::kStage;
-                    uint8_t *vb = kb + 2 * kBox;
+                    uint8_t *vb = kb + 2 * Smem::kTokBox;
                     mbar_expect_tx(&full[s], Smem::kStage);
-                    const int t0 = c0 + st * kBlk;
+                    const int t0 = c0 + st * Smem::kTok;
                     for (int x = 0; x < 2; ++x)
-                        tma_load_3d(kb + x * kBox, &tm_k, &full[s], 128 * mh + 64 * x, t0, bh);
+                        tma_load_3d(kb + x * Smem::kTokBox, &tm_k, &full[s], 128 * mh + 64 * x, t0,
+                                    bh);
                     for (int x = 0; x < Smem::kVBoxes; ++x)
-                        tma_load_4d(vb + x * kBox, &tm_v, &full[s], DVC * nv + 64 * x, h, t0, b);
+                        tma_load_4d(vb + x * Smem::kTokBox, &tm_v, &full[s], DVC * nv + 64 * x, h,
+                                    t0, b);
                 }
             }
         }
@@ -261,19 +270,20 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 tc_fence_after();
                 const int L = min(chunk, n - c * chunk);
                 uint32_t accumulate = 0;
-                for (int st = 0; st * kBlk < L; ++st, ++it) {
+                for (int st = 0; st * Smem::kTok < L; ++st, ++it) {
                     const int s = it % S;
                     if (!mbar_wait(&full[s], (it / S) & 1, &abort_flag, err)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t kb = smem_u32(smem + s * Smem::kStage);
-                    const uint32_t vb = kb + 2 * kBox;
+                    const uint32_t vb = kb + 2 * Smem::kTokBox;
 #pragma unroll
-                    for (int ks = 0; ks < kBlk / 16; ++ks) {
+                    for (int ks = 0; ks < Smem::kTok / 16; ++ks) {
                         // A = Kt^T (M = d_k, K = tokens), B = V (N = d_v, K = tokens):
-                        // both MN-major; 16 tokens = two 8-row atoms = 2048 B.
-                        const uint64_t ad = smem_desc_sw128(kb + ks * 2048, kBox, 1024);
-                        const uint64_t bd = smem_desc_sw128(vb + ks * 2048, kBox, 1024);
-                        mma_bf16(tmem + 128 * buf, ad, bd, idesc, accumulate);
+                        // both MN-major, 64 channels per box (the leading
+                        // byte offset); 16 tokens = two 8-row atoms = 2048 B.
+                        const uint64_t ad = smem_desc_sw128(kb + ks * 2048, Smem::kTokBox, 1024);
+                        const uint64_t bd = smem_desc_sw128(vb + ks * 2048, Smem::kTokBox, 1024);
+                        mma_bf16(tmem + Smem::kBufCols * buf, ad, bd, idesc, accumulate);
                         accumulate = 1;
                     }
                     mma_commit(&empty[s]);
@@ -282,30 +292,34 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             }
         }
     } else {
-        // state warpgroup: warp w owns TMEM lanes 32*(w%4) .. +31 = rows of the d_k half
+        // state warpgroups: warp w owns TMEM lanes 32*(w%4) .. +31 = rows of
+        // the d_k half; warpgroup wg owns kCols of the CTA's DVC columns
+        constexpr int kCols = Smem::kCols;
+        const int wg = (warp - 2) / 4;
         const int q4 = warp % 4;
         const int row = 32 * q4 + lane;
         const int krow = 128 * mh + row;                     // row of S
+        const int col0 = DVC * nv + kCols * wg;              // first column of S
         const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
-        const size_t sbase = ((size_t)bh * kD + krow) * kD + DVC * nv;
+        const size_t sbase = ((size_t)bh * kD + krow) * kD + col0;
         const long long state_elems = nbh * kD * kD;
         const long long sprev_elems = nbh * nchunks * kD * kD;
-        float st[DVC];
-        if (state_in && in_bounds((long long)sbase + DVC - 1, state_elems, err, kSiteState)) {
+        float st[kCols];
+        if (state_in && in_bounds((long long)sbase + kCols - 1, state_elems, err, kSiteState)) {
             const float4 *src = reinterpret_cast<const float4 *>(state_in + sbase);
 #pragma unroll
-            for (int v4 = 0; v4 < DVC / 4; ++v4) {
+            for (int v4 = 0; v4 < kCols / 4; ++v4) {
                 const float4 f = src[v4];
                 st[4 * v4] = f.x; st[4 * v4 + 1] = f.y; st[4 * v4 + 2] = f.z; st[4 * v4 + 3] = f.w;
             }
         } else {
 #pragma unroll
-            for (int e = 0; e < DVC; ++e) st[e] = 0.f;
+            for (int e = 0; e < kCols; ++e) st[e] = 0.f;
         }
         {
-            const size_t o0 = ((size_t)bh * nchunks * kD + krow) * kD + DVC * nv;
-            if (in_bounds((long long)o0 + DVC - 1, sprev_elems, err, kSiteState))
-                store_bf16_row(s_prev + o0, st, DVC);
+            const size_t o0 = ((size_t)bh * nchunks * kD + krow) * kD + col0;
+            if (in_bounds((long long)o0 + kCols - 1, sprev_elems, err, kSiteState))
+                store_bf16_row(s_prev + o0, st, kCols);
         }
         for (int c = 0; c < nchunks; ++c) {
             const int buf = c & 1;
@@ -314,9 +328,9 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             const bool last = (c == nchunks - 1);
             const float decay = last ? hp.decay_last[h] : hp.decay_chunk[h];
 #pragma unroll
-            for (int cb = 0; cb < DVC / 32; ++cb) {
+            for (int cb = 0; cb < kCols / 32; ++cb) {
                 uint32_t v[32];
-                tmem_ld32(tmem + 128 * buf + lane_off + 32 * cb, v);
+                tmem_ld32(tmem + Smem::kBufCols * buf + lane_off + kCols * wg + 32 * cb, v);
                 tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 32; ++e)
@@ -325,13 +339,13 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             tc_fence_before();
             mbar_arrive(&acc_free[buf]);                     // buffer free for chunk c + 2
             if (!last) {
-                const size_t o1 = (((size_t)bh * nchunks + c + 1) * kD + krow) * kD + DVC * nv;
-                if (in_bounds((long long)o1 + DVC - 1, sprev_elems, err, kSiteState))
-                    store_bf16_row(s_prev + o1, st, DVC);
-            } else if (state_out && in_bounds((long long)sbase + DVC - 1, state_elems, err, kSiteState)) {
+                const size_t o1 = (((size_t)bh * nchunks + c + 1) * kD + krow) * kD + col0;
+                if (in_bounds((long long)o1 + kCols - 1, sprev_elems, err, kSiteState))
+                    store_bf16_row(s_prev + o1, st, kCols);
+            } else if (state_out && in_bounds((long long)sbase + kCols - 1, state_elems, err, kSiteState)) {
                 float4 *o = reinterpret_cast<float4 *>(state_out + sbase);
 #pragma unroll
-                for (int v4 = 0; v4 < DVC / 4; ++v4)
+                for (int v4 = 0; v4 < kCols / 4; ++v4)
                     o[v4] = make_float4(st[4 * v4], st[4 * v4 + 1], st[4 * v4 + 2], st[4 * v4 + 3]);
             }
         }
@@ -352,7 +366,7 @@ tc_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, Smem::kTmemCols);
     }
 }
 
@@ -1596,6 +1610,30 @@ void tc_operand_layout(int batch, int heads, int seqlen, int chunk, size_t *qt, 
 // block of whole 128-row tiles.
 static int parallel_span(int n) { return (n + kBlk - 1) / kBlk * kBlk; }
 
+// d_v columns per state CTA (64, 128 or 256).  A state CTA streams its d_k
+// half of Kt and its columns of V over the whole sequence, 2 (128 + DVC)
+// bytes per token, one ring stage after another, so the pass takes about
+// waves x (t0 + bytes per CTA / rate per CTA).  Measured on B200 over
+// n = 128 .. 8192 (the pass alone, CUDA events): t0 about 10 us and
+// 64-80 GB/s per CTA at every width.  So 16 sequence-heads take 64 columns
+// (128 CTAs), 32 take 128 (128 CTAs), and 40 take 256 (80 CTAs, one wave:
+// 36 us at n = 2048 against 43 us for two waves of 160 CTAs at 128).  The
+// smallest estimate wins, the narrower width on a tie.
+static int tc_state_columns(int seq_heads, int n, int sms) {
+    int best = 64;
+    double best_us = 0.0;
+    for (int dvc = 64; dvc <= kD; dvc *= 2) {
+        const long long ctas = (long long)seq_heads * 2 * (kD / dvc);
+        const long long waves = (ctas + sms - 1) / sms;
+        const double us = (double)waves * (10.0 + (double)n * 2.0 * (128 + dvc) / 70e3);
+        if (dvc == 64 || us < best_us) {
+            best = dvc;
+            best_us = us;
+        }
+    }
+    return best;
+}
+
 size_t tc_parallel_workspace_bytes(int batch, int heads, int seqlen) {
     return seqlen > 0 ? tc_layout(batch, heads, seqlen, parallel_span(seqlen)).total : 0;
 }
@@ -1697,30 +1735,41 @@ cudaError_t launch_chunkwise_tc(const ChunkwiseArgs &a, const float *gammas, cud
         if (e != cudaSuccess) return e;
     }
     if (!parallel) {
-        // d_v columns per state CTA: 128 (four CTAs per sequence-head) unless
-        // eight CTAs per sequence-head still fit in one wave
         int dev = 0, sms = 148;
         if (cudaGetDevice(&dev) == cudaSuccess)
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        const bool narrow = BH * 8 <= sms;
-        KernelTimer timer("tc_state", stream);
-        if (narrow) {
-            const int smem = (int)TcStateSmem<64>::kBytes;
-            e = cudaFuncSetAttribute(tc_state_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     smem);
-            if (e != cudaSuccess) return e;
-            e = launch_overlapped(tc_state_kernel<64>, dim3(BH * 8), dim3(kTcThreads), smem, stream,
-                                  tm_k, tm_v, hp, a.state_in, a.state_out, sp, H, n, C, nchunks,
-                                  err);
-        } else {
-            const int smem = (int)TcStateSmem<128>::kBytes;
-            e = cudaFuncSetAttribute(tc_state_kernel<128>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            if (e != cudaSuccess) return e;
-            e = launch_overlapped(tc_state_kernel<128>, dim3(BH * 4), dim3(kTcThreads), smem,
-                                  stream, tm_k, tm_v, hp, a.state_in, a.state_out, sp, H, n, C,
-                                  nchunks, err);
+        const int dvc = tc_state_columns(BH, n, sms);
+        // Kt and V as the state pass reads them: sub-tiles of 64 tokens at
+        // 256 columns, else the 128-token tiles of the output pass
+        CUtensorMap sk = tm_k, sv = tm_v;
+        if (dvc == 256) {
+            const cuuint32_t rows = (cuuint32_t)TcStateSmem<256>::kTok;
+            cuuint64_t kdims[3] = {kD, (cuuint64_t)n, (cuuint64_t)BH};
+            cuuint64_t kstr[2] = {kD * 2, (cuuint64_t)n * kD * 2};
+            cuuint32_t kbox[3] = {64, rows, 1};
+            cuuint64_t vdims[4] = {kD, (cuuint64_t)H, (cuuint64_t)n, (cuuint64_t)B};
+            cuuint64_t vstr[3] = {kD * 2, (cuuint64_t)H * kD * 2, (cuuint64_t)n * H * kD * 2};
+            cuuint32_t vbox[4] = {64, 1, rows, 1};
+            if (!make_tensor_map_bf16(&sk, kt, 3, kdims, kstr, kbox) ||
+                !make_tensor_map_bf16(&sv, a.v, 4, vdims, vstr, vbox))
+                return cudaErrorInvalidValue;
         }
+        KernelTimer timer("tc_state", stream);
+        auto launch = [&](auto kernel, int smem, int threads) -> cudaError_t {
+            cudaError_t r = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 smem);
+            if (r != cudaSuccess) return r;
+            return launch_overlapped(kernel, dim3(BH * 2 * (kD / dvc)), dim3(threads), smem, stream,
+                                     sk, sv, hp, a.state_in, a.state_out, sp, H, n, C, nchunks, err);
+        };
+        if (dvc == 64)
+            e = launch(tc_state_kernel<64>, (int)TcStateSmem<64>::kBytes, TcStateSmem<64>::kThreads);
+        else if (dvc == 128)
+            e = launch(tc_state_kernel<128>, (int)TcStateSmem<128>::kBytes,
+                       TcStateSmem<128>::kThreads);
+        else
+            e = launch(tc_state_kernel<256>, (int)TcStateSmem<256>::kBytes,
+                       TcStateSmem<256>::kThreads);
         count_launch();
         if (e != cudaSuccess) return e;
     }

@@ -102,6 +102,24 @@ def test_more_work_items_than_sms(rn):
     assert slice_rel_err(st, ws, head_axis=1) < TOL
 
 
+# The state pass splits S into 128 x DVC blocks, one CTA each, with DVC =
+# 64, 128 or 256 chosen from the number of sequence-heads and the SM count
+# (148 on B200): 2 x 3 sequence-heads take 64 columns, 4 x 5 take 128, 3 x 13
+# take 256 (one wave of 78 CTAs), 5 x 16 take 256 over two waves.
+@pytest.mark.parametrize("B,H", [(2, 3), (4, 5), (3, 13), (5, 16)])
+@pytest.mark.parametrize("n,chunk", [(300, 128), (700, 256)])
+def test_state_pass_widths(rn, B, H, n, chunk):
+    q, k, v, _ = inputs(B, n, H, 71 + B * H + n)
+    rng = np.random.default_rng(72 + n)
+    s0 = rng.standard_normal((B, H, 256, 256)) * 0.05
+    gam = rn.retnet_default_gammas(H)
+    want, ws = oracle.retention_prefill(q, k, v, np.float32(gam), chunk, pos0=9,
+                                        state_in=np.float32(s0))
+    got, st = run(rn, q, k, v, gam, chunk, pos0=9, state_in=s0)
+    assert slice_rel_err(got, want) < TOL
+    assert slice_rel_err(st, ws, head_axis=1) < TOL
+
+
 def test_tensor_matches_simt_path(rn):
     B, n, H = 1, 1024, 4
     q, k, v, g = inputs(B, n, H, 31, gate_width=256)
