@@ -61,12 +61,13 @@ struct GemmRow {
     __nv_bfloat16 *dst;                     // the row's first column; null: not written
     bool fold;
     float scale;
-    const float2 *cs;                       // the row's 128 (cos, sin) pairs
+    const float2 *cs;                       // 128 (cos, sin) pairs at the base position tb
+    float delta;                            // t - tb, below kFoldTableStride
 };
 
 __device__ __forceinline__ GemmRow gemm_row(const GemmArgs &a, long long grow, int which,
                                             int c_in, bool live) {
-    GemmRow r{nullptr, false, 1.f, nullptr};
+    GemmRow r{nullptr, false, 1.f, nullptr, 0.f};
     if (!live) return r;
     // (a select chain, not a dynamic index, keeps a.out out of local memory)
     __nv_bfloat16 *base = which == 0   ? a.out[0]
@@ -83,7 +84,8 @@ __device__ __forceinline__ GemmRow gemm_row(const GemmArgs &a, long long grow, i
             return r;
         const float e = (float)(t % a.fold.fold + 1) * a.fold.log2g[h];
         r.scale = exp2f(which == 0 ? e : -e);
-        r.cs = a.fold.table + (size_t)t * 128;
+        r.cs = a.fold.table + (size_t)(t / kFoldTableStride) * 128;
+        r.delta = (float)(t % kFoldTableStride);
         r.fold = true;
         r.dst = base + ((b * a.fold.heads + h) * (long long)a.fold.n + t) * 256;
     } else {
@@ -92,8 +94,16 @@ __device__ __forceinline__ GemmRow gemm_row(const GemmArgs &a, long long grow, i
     return r;
 }
 
+// log2 of theta_{j+1} / theta_j = 10000^(-1/128), and that ratio.
+constexpr float kLog2ThetaStep = -0.10381025296523007f;
+constexpr float kThetaStep = 0.930572040929699f;
+
 // Stores columns [32 cb, 32 cb + 32) of the row (bf16), folded if asked:
-// pair j = 16 cb + p turned by the row's (cos, sin) of pair j and scaled.
+// pair j = 16 cb + p turned by the angle (pos0 + t) theta_j and scaled.  The
+// (cos, sin) of (pos0 + tb) theta_j come from the table (one row per 32
+// positions, so the 32 rows of a warp read the same entries); those of
+// (t - tb) theta_j, an angle below 32, from the fast sine and cosine, whose
+// error there (a few 1e-6) is far below the bf16 rounding of the result.
 __device__ __forceinline__ void gemm_store32(const GemmRow &r, int cb, const uint32_t (&v)[32]) {
     uint4 *d4 = reinterpret_cast<uint4 *>(r.dst + 32 * cb);
     if (r.fold) {
@@ -101,12 +111,17 @@ __device__ __forceinline__ void gemm_store32(const GemmRow &r, int cb, const uin
         const float4 *src = reinterpret_cast<const float4 *>(r.cs + 16 * cb);
 #pragma unroll
         for (int i = 0; i < 8; ++i) cs4[i] = src[i];
+        float th = exp2f((float)(16 * cb) * kLog2ThetaStep);  // theta_{16 cb}
         uint32_t y[16];
 #pragma unroll
         for (int p = 0; p < 16; ++p) {
-            const float cc = (p & 1) ? cs4[p / 2].z : cs4[p / 2].x;
-            const float ss = (p & 1) ? cs4[p / 2].w : cs4[p / 2].y;
-            const float c = cc * r.scale, sn = ss * r.scale;
+            float sd, cd;
+            __sincosf(r.delta * th, &sd, &cd);
+            th *= kThetaStep;
+            const float cb0 = (p & 1) ? cs4[p / 2].z : cs4[p / 2].x;
+            const float sb0 = (p & 1) ? cs4[p / 2].w : cs4[p / 2].y;
+            const float c = (cb0 * cd - sb0 * sd) * r.scale;
+            const float sn = (sb0 * cd + cb0 * sd) * r.scale;
             const float x0 = __uint_as_float(v[2 * p]), x1 = __uint_as_float(v[2 * p + 1]);
             y[p] = pack_bf16x2(x0 * c - x1 * sn, x0 * sn + x1 * c);
         }

@@ -8,9 +8,9 @@
 namespace retnet {
 
 // rotate.cu ---------------------------------------------------------------
-// table[t * (d/2) + j] = (cos, sin) of (pos0 + t) * theta_j, t < n.
-cudaError_t launch_rotation_table(float2 *table, int n, int d, long long pos0,
-                                  cudaStream_t stream);
+// table[t * (d/2) + j] = (cos, sin) of (pos0 + t * stride) * theta_j, t < rows.
+cudaError_t launch_rotation_table(float2 *table, int rows, int d, long long pos0,
+                                  cudaStream_t stream, int stride = 1);
 cudaError_t launch_xpos_rotate(const void *x, void *y, long long rows_bt, int heads, int d,
                                retnet_dtype dtype, int seqlen, long long pos0,
                                cudaStream_t stream);
@@ -99,15 +99,19 @@ bool make_tensor_map_bf16(CUtensorMap *m, const void *base, int rank, const cuui
 // gemm_tc.cu ---------------------------------------------------------------
 // Rotation and decay fold applied by the GEMM's epilogue to outputs 0 and 1
 // (the MSR layer's Q and K, 256 columns per head): with row r = b n + t,
-// column 2j, 2j+1 of head h is turned by table[t * 128 + j] (the (cos, sin)
-// of (pos0 + t) theta_j, from launch_rotation_table) and scaled by
-// gamma_h^(+(t mod fold + 1)) (output 0) or gamma_h^(-(t mod fold + 1))
-// (output 1), and written as Qt, Kt in the prefill's [b*H + h][t][256]
-// layout instead of [m, n_split].
+// column 2j, 2j+1 of head h is turned by the angle (pos0 + t) theta_j,
+// theta_j = 10000^(-j/128), and scaled by gamma_h^(+(t mod fold + 1))
+// (output 0) or gamma_h^(-(t mod fold + 1)) (output 1), and written as Qt,
+// Kt in the prefill's [b*H + h][t][256] layout instead of [m, n_split].
+// The angle is split as (pos0 + tb) theta_j + (t - tb) theta_j with
+// tb = t rounded down to a multiple of kFoldTableStride: the first part's
+// (cos, sin) is table[(t / kFoldTableStride) * 128 + j] (launch_rotation_table
+// with that stride), the second (below 32 theta_j) is formed in registers.
+constexpr int kFoldTableStride = 32;
 struct GemmFold {
     int on;
     int n, heads, fold;
-    const float2 *table;           // [n, 128] device
+    const float2 *table;           // [ceil(n / kFoldTableStride), 128] device
     float log2g[kMaxHeads];
 };
 // Y = X W^T on the tensor cores: X [m, k], W [n, k], bf16, f32 accumulation.

@@ -145,7 +145,9 @@ retnet_status retnet_msr_layer(const void *x, const void *w_qkvg, const void *w_
         for (int h = 0; h < kMaxHeads; ++h)
             fold.log2g[h] = h < shape->heads ? (float)std::log2((double)gammas[h]) : 0.f;
         float2 *table = reinterpret_cast<float2 *>(ws + l.table);
-        RETNET_CUDA_TRY(launch_rotation_table(table, shape->seqlen, 256, pos0, s));
+        RETNET_CUDA_TRY(launch_rotation_table(
+            table, (shape->seqlen + kFoldTableStride - 1) / kFoldTableStride, 256, pos0, s,
+            kFoldTableStride));
         fold.table = table;
         char *fwd = ws + l.fwd;
         void *outs[4] = {fwd + qt_off, fwd + kt_off, v, g};

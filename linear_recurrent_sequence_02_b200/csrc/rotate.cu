@@ -9,30 +9,33 @@
 
 namespace retnet {
 
-// Grid (ceil(n / kTablePositions), ceil(half / 128)): each thread owns one
-// pair index j, forms theta_j once and fills kTablePositions positions, so
-// the float64 power is paid once per 32 table entries.
+// Grid (ceil(rows / kTablePositions), ceil(half / 128)): each thread owns one
+// pair index j, forms theta_j once and fills kTablePositions rows, so the
+// float64 power is paid once per 32 table entries.  Row t holds position
+// pos0 + t * stride.
 constexpr int kTablePositions = 32;
 
 __global__ void __launch_bounds__(128)
-rotation_table_kernel(float2 *__restrict__ table, int n, int half, int d, long long pos0) {
+rotation_table_kernel(float2 *__restrict__ table, int rows, int half, int d, long long pos0,
+                      int stride) {
     const int j = blockIdx.y * 128 + threadIdx.x;
     if (j >= half) return;
     const double theta = pow(10000.0, -2.0 * (double)j / (double)d);
     const int t0 = blockIdx.x * kTablePositions;
-    const int t1 = min(n, t0 + kTablePositions);
-    for (int t = t0; t < t1; ++t) table[(size_t)t * half + j] = rotation_cs(pos0 + t, theta);
+    const int t1 = min(rows, t0 + kTablePositions);
+    for (int t = t0; t < t1; ++t)
+        table[(size_t)t * half + j] = rotation_cs(pos0 + (long long)t * stride, theta);
 }
 
-cudaError_t launch_rotation_table(float2 *table, int n, int d, long long pos0,
-                                  cudaStream_t stream) {
+cudaError_t launch_rotation_table(float2 *table, int rows, int d, long long pos0,
+                                  cudaStream_t stream, int stride) {
     const int half = d / 2;
-    if (n == 0 || half == 0) return cudaSuccess;
-    dim3 grid((unsigned)((n + kTablePositions - 1) / kTablePositions),
+    if (rows == 0 || half == 0) return cudaSuccess;
+    dim3 grid((unsigned)((rows + kTablePositions - 1) / kTablePositions),
               (unsigned)((half + 127) / 128));
     {
         KernelTimer timer("rotation_table", stream);
-        rotation_table_kernel<<<grid, 128, 0, stream>>>(table, n, half, d, pos0);
+        rotation_table_kernel<<<grid, 128, 0, stream>>>(table, rows, half, d, pos0, stride);
     }
     count_launch();
     return cudaGetLastError();

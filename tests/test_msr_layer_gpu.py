@@ -136,3 +136,13 @@ def test_msr_layer_folded_operands_on_cta_pairs(rn, pairs):
         rn.retnet_set_output_pairing(0)
     assert slice_rel_err(got[:, :, None], want[:, :, None]) < TOL
     assert slice_rel_err(st, ws, head_axis=1) < TOL
+
+
+def test_msr_layer_fold_angles_far_and_straddling(rn):
+    # The fold forms each row's angle (pos0 + t) theta_j from a table row every
+    # 32 positions plus the remainder; n = 1100 is no multiple of 32, so the
+    # 32 rows of a warp straddle two table rows, and pos0 = 123457 puts the
+    # table's angles far from zero.
+    got, want, st, ws = _layer(rn, 2, 1100, 512, 2, 256, 512, 37, pos0=123457, state=True)
+    assert slice_rel_err(got[:, :, None], want[:, :, None]) < TOL
+    assert slice_rel_err(st, ws, head_axis=1) < TOL
