@@ -5,24 +5,24 @@
 // pos * theta_j, theta_j = 10000^(-2j/d).  Relative position then enters
 // through (R_n q) . (R_m k), which depends only on n - m; the per-head
 // decay takes the place of xPos's length scaling.
+#include <algorithm>
+
 #include "kernels.h"
 
 namespace retnet {
 
-// Grid (ceil(rows / kTablePositions), ceil(half / 128)): each thread owns one
-// pair index j, forms theta_j once and fills kTablePositions rows, so the
-// float64 power is paid once per 32 table entries.  Row t holds position
+// Grid (ceil(rows / per_thread), ceil(half / 128)): each thread owns one
+// pair index j, forms theta_j once and fills per_thread rows, so the float64
+// power is paid once per per_thread table entries.  Row t holds position
 // pos0 + t * stride.
-constexpr int kTablePositions = 32;
-
 __global__ void __launch_bounds__(128)
 rotation_table_kernel(float2 *__restrict__ table, int rows, int half, int d, long long pos0,
-                      int stride) {
+                      int stride, int per_thread) {
     const int j = blockIdx.y * 128 + threadIdx.x;
     if (j >= half) return;
     const double theta = pow(10000.0, -2.0 * (double)j / (double)d);
-    const int t0 = blockIdx.x * kTablePositions;
-    const int t1 = min(rows, t0 + kTablePositions);
+    const int t0 = blockIdx.x * per_thread;
+    const int t1 = min(rows, t0 + per_thread);
     for (int t = t0; t < t1; ++t)
         table[(size_t)t * half + j] = rotation_cs(pos0 + (long long)t * stride, theta);
 }
@@ -31,11 +31,14 @@ cudaError_t launch_rotation_table(float2 *table, int rows, int d, long long pos0
                                   cudaStream_t stream, int stride) {
     const int half = d / 2;
     if (rows == 0 || half == 0) return cudaSuccess;
-    dim3 grid((unsigned)((rows + kTablePositions - 1) / kTablePositions),
-              (unsigned)((half + 127) / 128));
+    // 32 rows per thread for long tables; short ones spread one row per
+    // thread, so the grid still covers the SMs
+    const int per_thread = std::max(1, std::min(32, rows / 256));
+    dim3 grid((unsigned)((rows + per_thread - 1) / per_thread), (unsigned)((half + 127) / 128));
     {
         KernelTimer timer("rotation_table", stream);
-        rotation_table_kernel<<<grid, 128, 0, stream>>>(table, rows, half, d, pos0, stride);
+        rotation_table_kernel<<<grid, 128, 0, stream>>>(table, rows, half, d, pos0, stride,
+                                                        per_thread);
     }
     count_launch();
     return cudaGetLastError();
