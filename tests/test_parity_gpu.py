@@ -197,6 +197,28 @@ def test_simt_head_dims_with_state_and_gate(rn, dk, dv):
     assert slice_rel_err(st, wst, head_axis=1) < TOL["f32"]
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_simt_and_decode_at_the_maximum_head_count(rn, dtype):
+    # 256 heads (the most the library accepts) on the SIMT prefill, then one
+    # decode step continuing from its state
+    rng = np.random.default_rng(8)
+    B, n, H, d, chunk = 1, 70, 256, 64, 64
+    q, k, v = (wl.normal(rng, (B, n + 1, H, d), 0.125, dtype) for _ in range(3))
+    gam = rn.retnet_default_gammas(H)
+    want, wstate = oracle.retention_prefill(q[:, :n], k[:, :n], v[:, :n], np.float32(gam),
+                                            chunk, pos0=1)
+    got, st = run_prefill(rn, q[:, :n], k[:, :n], v[:, :n], dtype, gam, chunk, "simt", pos0=1)
+    assert slice_rel_err(got, want) < TOL[dtype]
+    assert slice_rel_err(st, wstate, head_axis=1) < TOL[dtype]
+    qr = oracle.xpos_rotate(q[:, n:], 1 + n)[:, 0]
+    kr = oracle.xpos_rotate(k[:, n:], 1 + n)[:, 0]
+    o_ref, _ = oracle.retention_step(qr, kr, v[:, n], np.float32(gam), wstate)
+    s_dev = torch.from_numpy(np.float32(st)).cuda()
+    o = rn.retnet_retention_step(dev(q[:, n], dtype), dev(k[:, n], dtype), dev(v[:, n], dtype),
+                                 gam, s_dev, 1 + n)
+    assert slice_rel_err(host(o)[:, None], o_ref[:, None]) < TOL[dtype]
+
+
 def test_simt_split_prefill_and_decode_continue(rn):
     rng = np.random.default_rng(8)
     B, n, H, d, m = 2, 160, 2, 64, 96

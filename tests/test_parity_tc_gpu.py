@@ -252,3 +252,17 @@ def test_output_pass_on_pairs_and_single(rn, pairs, B, n, H, chunk):
         rn.retnet_set_output_pairing(0)
     assert slice_rel_err(got, want) < TOL
     assert slice_rel_err(st, ws, head_axis=1) < TOL
+
+
+def test_maximum_head_count(rn):
+    # 256 heads, the most the library accepts: the decay constants reach
+    # gamma = 1 in float32, the state pass runs several waves of CTAs and the
+    # output pass more items than it has CTAs; n = 300 leaves a ragged chunk.
+    B, n, H = 1, 300, 256
+    q, k, v, _ = inputs(B, n, H, 81)
+    gam = rn.retnet_default_gammas(H)
+    assert gam[-1] == 1.0
+    want, ws = oracle.retention_prefill(q, k, v, np.float32(gam), 128, pos0=2)
+    got, st = run(rn, q, k, v, gam, 128, pos0=2)
+    assert slice_rel_err(got, want) < TOL
+    assert slice_rel_err(st, ws, head_axis=1) < TOL
