@@ -59,7 +59,7 @@ typedef struct CUstream_st *retnet_stream_t;
 typedef enum retnet_status {
     RETNET_OK = 0,
     RETNET_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size or dtype */
-    RETNET_ERR_UNSUPPORTED = 2,  /* well-formed request this build does not implement */
+    RETNET_ERR_UNSUPPORTED = 2,  /* well-formed request the library does not implement */
     RETNET_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
     RETNET_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up */
     RETNET_ERR_WORKSPACE = 5,    /* workspace missing or smaller than required */
