@@ -171,6 +171,22 @@ def parallel_flops_per_token_head(d: int, n: int) -> int:
     return 2 * d * (n + 1)
 
 
+def executed_flops_per_token_head(d: int, chunk: int, n: int, parallel: bool = False) -> float:
+    """Flops the tensor-core prefill executes per token-head (the tensor
+    path, n a multiple of the chunk): 128-key tiles up to the diagonal,
+    the diagonal tile whole, upper tiles skipped.  A row block r of a chunk
+    runs r + 1 tiles of Q K^T and P V, 4 * 128 * d flops per row each, so a
+    chunk of R = C / 128 row blocks averages 256 d (R + 1) per token; the
+    chunkwise form adds Qt S_prev (2 d^2) for every chunk after the first
+    and the state pass's Kt^T V (2 d^2).  Chunks below 128 are computed as
+    128; the parallel form is one chunk of ceil(n / 128) row blocks."""
+    if parallel:
+        return 256.0 * d * ((n + 127) // 128 + 1)
+    c = max(chunk, 128)
+    nchunks = (n + c - 1) // c
+    return 256.0 * d * (c // 128 + 1) + 2.0 * d * d * (nchunks - 1) / nchunks + 2.0 * d * d
+
+
 class ClockSampler:
     """Samples SM clock and throttle reasons through NVML on a thread."""
 
@@ -665,6 +681,10 @@ def measure_prefill(args, w, chunk, rank, world, dev, full=True):
         prefill_info = {"tokens_per_s": B * n / (pre_ms / 1e3), "ms": pre_ms,
                         "tflops_algorithmic": alg / (pre_ms / 1e3) / 1e12,
                         "frac_of_bf16_peak": alg / (pre_ms / 1e3) / 1e12 / peaks["bf16_tflops"]}
+        if d == 256 and w.dtype == "bf16" and args.algo != "simt":   # the tensor-core path
+            exe = executed_flops_per_token_head(d, chunk, n, par) * B * n * H
+            prefill_info["flop_executed_per_token_head"] = exe / (B * n * H)
+            prefill_info["tflops_executed"] = exe / (pre_ms / 1e3) / 1e12
     step_decode = None
     if "retention_step" in kern_warm:
         tot, cnt = kern_warm["retention_step"]

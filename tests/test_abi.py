@@ -380,3 +380,19 @@ def test_linear_and_msr_layer_reject_before_launch(lib):
     assert call(ws=None) == 5
     assert call(wsb=1024) == 5
     assert call(ws=1024 + 256) == 5
+
+
+def test_bench_executed_flops_count_tiles_up_to_the_diagonal():
+    # chunk 512 = 4 row blocks of 128: 1 + 2 + 3 + 4 = 10 key tiles per chunk,
+    # each 4 * 128 * 256 flops per row (Q K^T and P V), 2.5 tiles per row on
+    # average; plus Qt S_prev for 15 of 16 chunks and the state pass's Kt^T V
+    import bench
+    tiles = 4 * 128 * 256 * (1 + 2 + 3 + 4) / 4
+    want = tiles + 2 * 256 * 256 * 15 / 16 + 2 * 256 * 256
+    assert bench.executed_flops_per_token_head(256, 512, 8192) == want == 581_632
+    # chunks below 128 are computed as 128: one tile per row block
+    want64 = 4 * 128 * 256 * 1 + 2 * 256 * 256 * 15 / 16 + 2 * 256 * 256
+    assert bench.executed_flops_per_token_head(256, 64, 2048) == want64
+    # the parallel form: one chunk of n / 128 row blocks, no state terms
+    assert bench.executed_flops_per_token_head(256, 0, 1024, parallel=True) == \
+        4 * 128 * 256 * sum(range(1, 9)) / 8
