@@ -47,10 +47,13 @@ def _prefill(rn, q, k, v, gam, chunk, gate=None, state_in=None, pos0=0):
     return y, st
 
 
-def test_timeout_path_reports_and_the_context_stays_usable(rn):
+# (B, H): the state pass at 64, 128 and 256 columns per CTA (6, 20 and 39
+# sequence-heads on 148 SMs); the skipped load is in its first CTA
+@pytest.mark.parametrize("B,H", [(1, 1), (4, 5), (3, 13)])
+def test_timeout_path_reports_and_the_context_stays_usable(rn, B, H):
     q, k, v, _ = (None if x is None else _dev(x)
-                  for x in wl.make_prefill_inputs(1, 1, 256, 256, "bf16", 1 / 16, 801))
-    gam = rn.retnet_default_gammas(1)
+                  for x in wl.make_prefill_inputs(B, H, 256, 256, "bf16", 1 / 16, 801))
+    gam = rn.retnet_default_gammas(H)
     ref_y, ref_s = _prefill(rn, q, k, v, gam, 128)          # default library
     rn.retnet_check_device_errors()
     with rn.using_library(rn.DEBUG_LIB_PATH):
@@ -75,7 +78,7 @@ def test_timeout_path_reports_and_the_context_stays_usable(rn):
 
 
 @pytest.mark.parametrize("B,n,H,chunk", [(2, 1101, 3, 256), (1, 77, 2, 512), (3, 300, 2, 64),
-                                         (1, 2048, 16, 512)])
+                                         (1, 2048, 16, 512), (4, 700, 5, 256), (3, 300, 13, 128)])
 def test_index_checks_quiet_and_bits_equal_prefill(rn, B, n, H, chunk):
     q, k, v, g = (_dev(x) for x in wl.make_prefill_inputs(B, H, n, 256, "bf16", 1 / 16,
                                                           810 + n, hidden=256))
