@@ -16,17 +16,19 @@
 //
 // Kernels (all bf16 operands, f32 accumulation):
 //   tc_prep    rotation + decay fold of q and k into Qt, Kt [B*H, n, 256]
-//   tc_state   per (sequence, head, 128x128 quarter of S): walks the chunks,
-//              accumulating Kt^T V onto the state in TMEM, scaling by g^L,
-//              and writing S_prev of every chunk (bf16) and the final state
-//   tc_output  per (sequence, head, chunk, 128-row block): S = Qt Kt^T in
-//              TMEM, causal mask in registers, P (bf16) to shared memory,
-//              O += P V; then O += Qt S_prev; epilogue writes O, or
-//              swish(G) * GroupNorm(O) when a gate is given.
+//   tc_state   per (sequence, head, 128 x DVC block of S, DVC = 64, 128 or
+//              256): walks the chunks, accumulating each chunk's Kt^T V in
+//              TMEM, carrying S <- g^L (S + Kt^T V) in registers, and writing
+//              S_prev of every chunk (bf16) and the final state (f32)
+//   tc_output  persistent, work items (sequence, head, chunk, 128-row
+//              block): S = Qt Kt^T in TMEM, causal mask in registers, P
+//              (bf16) to shared memory, O += P V; then O += Qt S_prev; the
+//              epilogue writes O, or swish(G) * GroupNorm(O) when a gate is
+//              given.
 // Roles inside a CTA: warp 0 issues TMA loads, warp 1 allocates TMEM and
-// issues tcgen05.mma, warps 2-5 move data between TMEM, registers and
-// memory.  Every mbarrier wait is bounded (about 2 s); on timeout the CTA
-// records kDevErrTimeout and unwinds.
+// issues tcgen05.mma, the remaining warps move data between TMEM, registers
+// and memory.  Every mbarrier wait is bounded (about 2 s); on timeout the
+// CTA records kDevErrTimeout and unwinds.
 #include <algorithm>
 #include <cmath>
 
