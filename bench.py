@@ -109,8 +109,8 @@ NCU_TRAFFIC = {
     ("tc_output", "long7b"): {
         "source": "chunkwise_tc.cu", "section": "output pass",
         "headers": ["sm100.cuh", "common.cuh"],
-        "sha256": "b8813a88b501781786be145125861691968076f253afbfefdcfe817e3019eaba",
-        "bytes": 277.98e6,
+        "sha256": "2135b4b483203581f984438dece09b44b415da3e3335562b3b0a0389e1c1b9af",
+        "bytes": 277.97e6,
     },
 }
 SECTION_BANNER = "// " + "-" * 66 + " "
@@ -164,6 +164,11 @@ def output_kernel_flops_per_token_head(d: int, chunk: int) -> int:
 
 def state_kernel_flops_per_token_head(d: int) -> int:
     return 2 * d * d
+
+
+def prep_kernel_bytes_per_token_head(d: int) -> int:
+    # the rotation and decay fold: q and k read, Qt and Kt written, bf16
+    return 4 * d * 2
 
 
 def parallel_flops_per_token_head(d: int, n: int) -> int:
@@ -665,6 +670,13 @@ def measure_prefill(args, w, chunk, rank, world, dev, full=True):
             roof = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak,
                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
                     "peak_source": peak_src, "work_per_launch": flops, "avg_us": avg_s * 1e6}
+        elif dom == "tc_prep":
+            # q and k read, Qt and Kt written once (bf16)
+            nbytes = prep_kernel_bytes_per_token_head(d) * th
+            gbs = nbytes / avg_s / 1e9
+            roof = {"kernel": dom, "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                    "peak_source": peak_src, "work_per_launch": nbytes, "avg_us": avg_s * 1e6}
         else:
             roof = {"kernel": dom, "bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"],
                     "unit": "GB/s", "frac": None, "traffic": None, "peak_source": peak_src}

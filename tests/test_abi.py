@@ -296,6 +296,7 @@ def test_bench_work_counts_match_the_formulas():
     assert bench.algorithmic_flops_per_token_head(d, C) == 524_800          # (dk+dv)(C+1) + 4 dk dv
     assert bench.output_kernel_flops_per_token_head(d, C) == 2 * d * (C + 1) + 2 * d * d
     assert bench.state_kernel_flops_per_token_head(d) == 2 * d * d
+    assert bench.prep_kernel_bytes_per_token_head(d) == 2048                 # q, k in; Qt, Kt out
     assert bench.parallel_flops_per_token_head(d, 2047) == 2 * d * 2048
 
 
