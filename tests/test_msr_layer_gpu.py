@@ -37,9 +37,12 @@ def host(t):
 
 
 @pytest.mark.parametrize("m,k,n", [(128, 64, 256), (1000, 1024, 512), (300, 2560, 2560),
-                                   (4097, 1024, 4096), (1, 128, 256)])
+                                   (4097, 1024, 4096), (1, 128, 256), (300, 192, 256),
+                                   (513, 64, 512)])
 def test_linear_against_oracle(rn, m, k, n):
-    # up to 128 rows: single CTAs (128 x 256 tiles); above: CTA pairs (256 x 256)
+    # up to 128 rows: single CTAs (128 x 256 tiles); above: CTA pairs (256 x 256),
+    # whose stages hold two 64-wide K steps: K = 192 and 64 leave the last
+    # stage's second step past the end of K (read as zeros)
     rng = np.random.default_rng(m + k + n)
     x = wl.normal(rng, (m, k), 1.0, "bf16")
     w = wl.normal(rng, (n, k), 1.0 / np.sqrt(k), "bf16")
