@@ -76,6 +76,12 @@ def test_backward_tensor_path(rn, n, chunk):
     check(rn, "bf16", 2, n, 3, 256, 256, chunk, pos0=5, algo="tensor", seed=n)
 
 
+def test_backward_with_the_widest_state_pass(rn):
+    # 3 x 13 = 39 sequence-heads: the three retentions' state passes take 256
+    # d_v columns per CTA (78 CTAs in one wave on 148 SMs)
+    check(rn, "bf16", 3, 300, 13, 256, 256, 128, pos0=2, algo="tensor", seed=77)
+
+
 def test_backward_tensor_path_no_rotation_ragged(rn):
     check(rn, "bf16", 1, 333, 2, 256, 256, 128, rotate=False, algo="tensor", seed=3)
 

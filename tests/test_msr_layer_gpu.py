@@ -149,3 +149,11 @@ def test_msr_layer_fold_angles_far_and_straddling(rn):
     got, want, st, ws = _layer(rn, 2, 1100, 512, 2, 256, 512, 37, pos0=123457, state=True)
     assert slice_rel_err(got[:, :, None], want[:, :, None]) < TOL
     assert slice_rel_err(st, ws, head_axis=1) < TOL
+
+
+def test_msr_layer_with_the_widest_state_pass(rn):
+    # 3 x 13 = 39 sequence-heads (hidden 13 x 256): the prefill's state pass
+    # takes 256 d_v columns per CTA, fed by the projection's folded operands
+    got, want, st, ws = _layer(rn, 3, 300, 3328, 13, 256, 128, 38, pos0=3, state=True)
+    assert slice_rel_err(got[:, :, None], want[:, :, None]) < TOL
+    assert slice_rel_err(st, ws, head_axis=1) < TOL
